@@ -1,0 +1,446 @@
+"""Benchmark of the KDA operator on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload I] [--impl reference]
+
+One step = one ``kda_forward`` call (varlen index + chunked prefill, every
+step of the hot path) over the prefill workload ``--workload`` (default 1:
+bf16, B=2, T=4096, H=16, d_k=d_v=128, chunk 64).  The timed region is K
+steps between a barrier + synchronize on both sides; each step's kernels
+are bracketed by CUDA events on the launching stream and L2 is flushed
+(256 MiB write) between steps outside those brackets.  Multi-GPU runs are
+independent replicas (the operator needs no collective): each rank runs the
+same workload on its own GPU and rank 0 reports the total over ranks divided
+by the slowest rank's time.
+
+The JSON line also carries: ``e2e`` (the same metric through the public
+Python API from pinned host buffers, with the host<->device copies inside
+the timed region), ``roofline`` (algorithmic bytes of the dominant kernel
+over its measured duration against the measured HBM copy bandwidth),
+``cpu_baseline`` (the fp64 CPU oracle on a bounded sample, rank 0), a
+``decode`` object (64 recurrent steps of the decode workload) and the SM
+clocks sampled during the timed region.
+
+``--impl reference``: the reference arm is the fp64 CPU oracle (there is no
+other implementation of this operator to run); it times K steps of a
+bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from gated_delta_rule_113_b200.inputs import WORKLOADS, decode_inputs, forward_inputs  # noqa: E402
+
+METRIC = "KDA tokens/sec/GPU (prefill and decode) + % of tensor-pipe / HBM roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# --------------------------------------------------------------------------
+# accounting
+# --------------------------------------------------------------------------
+def _es(dtype):
+    return 4 if dtype == torch.float32 else 2
+
+
+def prefill_bytes(T, N, H, Dk, Dv, io_dtype, gate_dtype, has_s0):
+    """Algorithmic HBM bytes of one prefill: every input read once, every output written once."""
+    e, g = _es(io_dtype), _es(gate_dtype)
+    per_token_head = 2 * Dk * e + Dv * e + Dk * g + g + Dv * e
+    states = N * H * Dk * Dv * 4 * (2 if has_s0 else 1)
+    return T * H * per_token_head + states + 4 * (N + 1)
+
+
+def prefill_flops(T, H, Dk, Dv, C=64):
+    """Algorithmic flops per prefill: 6*Dk*Dv + C*(3*Dk + 2*Dv) per token-head (triangles once)."""
+    return T * H * (6 * Dk * Dv + C * (3 * Dk + 2 * Dv))
+
+
+def decode_bytes(N, H, Dk, Dv, io_dtype):
+    e = _es(io_dtype)
+    return N * H * (2 * Dk * Dv * 4 + 3 * Dk * e + Dv * e + e + Dv * e)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def traffic_record(kernel):
+    """DRAM bytes per launch from a committed ncu capture, if the kernel's source is unchanged."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        recs = json.load(f)
+    rec = recs.get(kernel)
+    if not rec:
+        return None
+    src = os.path.join(ROOT, rec["source"])
+    if not os.path.exists(src):
+        return None
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    return rec["bytes_per_launch"] if sha == rec.get("source_sha") else None
+
+
+# --------------------------------------------------------------------------
+# clocks sampled during the timed region
+# --------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.dev)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.t.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------
+# CPU baseline: the fp64 oracle on a bounded sample
+# --------------------------------------------------------------------------
+def oracle_sample(w, inp, max_tokens):
+    """First ``max_tokens`` tokens of every sequence, all heads (same chains, truncated)."""
+    cu = inp["cu_seqlens"].numpy()
+    idx, lens = [], []
+    for n in range(len(cu) - 1):
+        L = min(int(cu[n + 1] - cu[n]), max_tokens)
+        idx.extend(range(int(cu[n]), int(cu[n]) + L))
+        lens.append(L)
+    idx = torch.tensor(idx, dtype=torch.long)
+    sub = {k: inp[k][idx].contiguous() for k in ("q", "k", "v", "log_alpha", "beta")}
+    sub["S0"] = inp["S0"]
+    sub["cu_seqlens"] = np.concatenate([[0], np.cumsum(lens)])
+    return sub, int(sum(lens))
+
+
+def run_oracle_timed(sub):
+    import oracle
+    t0 = time.perf_counter()
+    oracle.forward(sub["q"], sub["k"], sub["v"], sub["log_alpha"], sub["beta"], sub["S0"],
+                   sub["cu_seqlens"])
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(w, inp, max_tokens):
+    import oracle
+    sub, ntok = oracle_sample(w, inp, max_tokens)
+    dt = run_oracle_timed(sub)
+    return {"value": ntok / dt, "unit": "tokens/s", "cores": oracle.default_threads(),
+            "kind": "oracle",
+            "sample": f"first {max_tokens} tokens of each of the {len(inp['lengths'])} sequences, "
+                      f"all {w.H} heads ({ntok} tokens, {dt:.2f} s, fp64 token-by-token)"}
+
+
+# --------------------------------------------------------------------------
+# distributed plumbing (replicas)
+# --------------------------------------------------------------------------
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------------------
+# arms
+# --------------------------------------------------------------------------
+def bench_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    w = WORKLOADS[args.workload]
+    inp = forward_inputs(w)
+    sub, ntok = oracle_sample(w, inp, args.ref_tokens)
+    for _ in range(args.warmup):
+        run_oracle_timed(sub)
+    times = [run_oracle_timed(sub) for _ in range(args.steps)]
+    total = sum(times)
+    value = ntok * args.steps / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "sample_tokens": ntok, "H": w.H, "Dk": w.Dk, "Dv": w.Dv},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.default_threads(),
+                         "kind": "oracle",
+                         "sample": f"first {args.ref_tokens} tokens of each sequence, all heads"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def bench_kda(args):
+    import gated_delta_rule_113_b200 as kda
+    world, rank, local = dist_setup()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    kda.load_library()
+    w = WORKLOADS[args.workload]
+    inp = forward_inputs(w)
+    N, T, H, Dk, Dv = len(inp["lengths"]), int(inp["cu_seqlens"][-1]), w.H, w.Dk, w.Dv
+    d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    out = torch.empty((T, H, Dv), dtype=w.torch_dtype, device=dev)
+    sf = torch.empty((N, H, Dk, Dv), dtype=torch.float32, device=dev)
+    ws = torch.empty(kda.forward_workspace_size(N, T, H, Dk, Dv, w.torch_dtype), dtype=torch.uint8,
+                     device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        kda.forward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["S0"], d["cu_seqlens"],
+                    out=out, S_final=sf, workspace=ws)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    if kda.workspace_status(ws) != 0:
+        raise RuntimeError("device status not OK after warm-up")
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier(world)
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            flush.zero_()
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        barrier(world)
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = max_over_ranks(sum(step_ms), world)
+    value = world * T * args.steps / (total_ms * 1e-3)
+
+    # ---- end to end through the public API from pinned host buffers -------
+    names = ("q", "k", "v", "log_alpha", "beta")
+    host = {k: inp[k].pin_memory() for k in names}
+    host["S0"] = inp["S0"].pin_memory() if inp["S0"] is not None else None
+    host_cu = inp["cu_seqlens"].pin_memory()
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    sf_h = torch.empty(sf.shape, dtype=sf.dtype).pin_memory()
+    dd = {k: torch.empty_like(d[k]) for k in names}
+    s0d = torch.empty_like(d["S0"]) if d["S0"] is not None else None
+    cud = torch.empty_like(d["cu_seqlens"])
+    h2d = sum(host[k].numel() * host[k].element_size() for k in names) + \
+        (host["S0"].numel() * 4 if host["S0"] is not None else 0) + host_cu.numel() * 4
+    d2h = out_h.numel() * out_h.element_size() + sf_h.numel() * 4
+
+    def e2e_step():
+        for k in names:
+            dd[k].copy_(host[k], non_blocking=True)
+        if s0d is not None:
+            s0d.copy_(host["S0"], non_blocking=True)
+        cud.copy_(host_cu, non_blocking=True)
+        kda.forward(dd["q"], dd["k"], dd["v"], dd["log_alpha"], dd["beta"], s0d, cud, out=out,
+                    S_final=sf, workspace=ws)
+        out_h.copy_(out, non_blocking=True)
+        sf_h.copy_(sf, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    e2e_value = world * T * args.steps / (e2e_ms * 1e-3)
+
+    # ---- decode workload: 64 recurrent steps ------------------------------
+    dec = None
+    if not args.no_decode:
+        dec = bench_decode(kda, dev, stream, world, args)
+
+    # ---- roofline of the dominant kernel (prefill) -------------------------
+    peaks, peaks_kind = load_peaks()
+    alg_bytes = prefill_bytes(T, N, H, Dk, Dv, w.torch_dtype, w.torch_dtype, inp["S0"] is not None)
+    alg_flops = prefill_flops(T, H, Dk, Dv)
+    mean_ms = sum(step_ms) / len(step_ms)
+    achieved = alg_bytes / (mean_ms * 1e-3) / 1e9
+    roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / peaks["hbm_gbs"], "traffic": traffic_record("kda_prefill"),
+            "peak_kind": f"{peaks_kind} HBM copy", "kernel": "kda_forward (varlen index + prefill)",
+            "algorithmic_bytes": alg_bytes, "algorithmic_flops": alg_flops,
+            "tensor_frac_algorithmic": alg_flops / (mean_ms * 1e-3) / 1e12 / peaks["bf16_tflops"]}
+
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            cpu = cpu_baseline(w, inp, args.cpu_tokens)
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if w.torch_dtype == torch.bfloat16 else "f32",
+            "data": "synthetic (seeded generator; q,k L2-normalised, log_alpha uniform)",
+            "config": {"workload": w.name, "num_seqs": N, "total_tokens": T, "H": H, "Dk": Dk,
+                       "Dv": Dv, "chunk": 64, "state": "fp32",
+                       "l2": "256 MiB flush between steps, outside the timed spans",
+                       "parallelism": f"replicas x{world}"},
+            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": 2 * args.steps,
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "decode": dec,
+            "clocks": clk.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def bench_decode(kda, dev, stream, world, args):
+    w = WORKLOADS[4]
+    steps = w.decode_steps
+    inp = decode_inputs(w)
+    N, H, Dk, Dv = len(w.lengths), w.H, w.Dk, w.Dv
+    x = {k: inp[k].to(dev) for k in ("q", "k", "v", "log_alpha", "beta")}
+    S = inp["S"].to(dev)
+    out = torch.empty((N, H, Dv), dtype=w.torch_dtype, device=dev)
+
+    def run64():
+        for t in range(steps):
+            kda.decode_step(x["q"][t], x["k"][t], x["v"][t], x["log_alpha"][t], x["beta"][t], S,
+                            out=out)
+
+    for _ in range(3):
+        run64()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = 3
+    e0.record(stream)
+    for _ in range(reps):
+        run64()
+    e1.record(stream)
+    barrier(world)
+    ms = max_over_ranks(e0.elapsed_time(e1), world) / (reps * steps)
+    peaks, kind = load_peaks()
+    b = decode_bytes(N, H, Dk, Dv, w.torch_dtype)
+    gbs = b / (ms * 1e-3) / 1e9
+    return {"workload": w.name, "value": world * N / (ms * 1e-3), "unit": "tokens/s",
+            "us_per_step": ms * 1e3, "gpu_launches": reps * steps,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm_gbs"], "frac_of_8TBs_nominal": gbs / 8000.0,
+                         "traffic": traffic_record("kda_decode"), "algorithmic_bytes": b,
+                         "peak_kind": f"{kind} HBM copy"},
+            "state": "512 MiB fp32, larger than L2: no flush needed"}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", type=int, default=1, choices=[0, 1, 2, 3])
+    ap.add_argument("--impl", default="kda", choices=["kda", "reference"])
+    ap.add_argument("--cpu-tokens", type=int, default=4096,
+                    help="oracle sample: first N tokens of each sequence")
+    ap.add_argument("--ref-tokens", type=int, default=512,
+                    help="reference arm: tokens per sequence in each timed step")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return bench_reference(args)
+    return bench_kda(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

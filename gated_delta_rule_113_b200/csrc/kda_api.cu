@@ -1,0 +1,147 @@
+// kda_api.cu -- the C ABI declared in include/kda.h: host validation,
+// workspace layout, device selection and kernel dispatch.
+#include <string.h>
+
+#include "kda_internal.cuh"
+
+namespace {
+
+using kda::kWsHeader;
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool dtype_ok(int32_t d) { return d == KDA_F32 || d == KDA_BF16; }
+bool width_ok(int32_t d) { return d == 64 || d == 128; }
+
+kda_status check_common(const kda_params *p) {
+    if (!p) return KDA_ERR_INVALID;
+    if (p->num_seqs < 0 || p->H <= 0) return KDA_ERR_INVALID;
+    if (!dtype_ok(p->io_dtype) || !dtype_ok(p->gate_dtype)) return KDA_ERR_UNSUPPORTED;
+    if (!width_ok(p->Dk) || !width_ok(p->Dv)) return KDA_ERR_UNSUPPORTED;
+    if (p->flags & ~KDA_FLAG_FORCE_SIMT) return KDA_ERR_INVALID;
+    return KDA_OK;
+}
+
+// Pointers must be device (or managed) memory of one device; make that
+// device current for the launches.  Host memory would fault on the GPU.
+kda_status select_device(const void *const *ptrs, int n) {
+    int dev = -1;
+    for (int i = 0; i < n; ++i) {
+        if (!ptrs[i]) continue;
+        cudaPointerAttributes at;
+        if (cudaPointerGetAttributes(&at, ptrs[i]) != cudaSuccess) {
+            cudaGetLastError();
+            return KDA_ERR_INVALID;
+        }
+        if (at.type != cudaMemoryTypeDevice && at.type != cudaMemoryTypeManaged)
+            return KDA_ERR_INVALID;
+        if (dev < 0) dev = at.device;
+        else if (dev != at.device) return KDA_ERR_INVALID;
+    }
+    if (dev < 0) return KDA_OK;
+    int cur = -1;
+    if (cudaGetDevice(&cur) != cudaSuccess) return KDA_ERR_CUDA;
+    if (cur != dev && cudaSetDevice(dev) != cudaSuccess) return KDA_ERR_CUDA;
+    return KDA_OK;
+}
+
+size_t workspace_bytes(const kda_params *p) {
+    return kWsHeader + round_up(sizeof(int32_t) * (size_t)p->num_seqs, 256);
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t kda_abi_version(void) { return KDA_ABI_VERSION; }
+
+const char *kda_status_string(kda_status s) {
+    switch (s) {
+    case KDA_OK: return "KDA_OK";
+    case KDA_ERR_INVALID: return "KDA_ERR_INVALID: invalid argument";
+    case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED: unsupported shape or dtype";
+    case KDA_ERR_ALIGN: return "KDA_ERR_ALIGN: tensor not 16-byte aligned";
+    case KDA_ERR_WORKSPACE: return "KDA_ERR_WORKSPACE: workspace missing, misaligned or too small";
+    case KDA_ERR_CUDA: return "KDA_ERR_CUDA: CUDA call or launch failed";
+    case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT: bounded device wait gave up";
+    case KDA_ERR_SEQLENS: return "KDA_ERR_SEQLENS: cu_seqlens not monotone from 0 to total_tokens";
+    }
+    return "KDA_ERR_UNKNOWN";
+}
+
+size_t kda_forward_workspace_size(const kda_params *p) {
+    if (check_common(p) != KDA_OK) return 0;
+    return workspace_bytes(p);
+}
+
+kda_status kda_forward(const void *q, const void *k, const void *v, const void *log_alpha,
+                       const void *beta, const float *S0, const int32_t *cu_seqlens, void *out,
+                       float *S_final, const kda_params *p, void *workspace, size_t ws_bytes,
+                       void *stream) {
+    kda_status st = check_common(p);
+    if (st != KDA_OK) return st;
+    if (p->chunk != kda::kChunk || p->total_tokens < 0) return KDA_ERR_UNSUPPORTED;
+    if (p->num_seqs == 0) return p->total_tokens == 0 ? KDA_OK : KDA_ERR_INVALID;
+    if (!cu_seqlens) return KDA_ERR_INVALID;
+    if (p->total_tokens > 0 && (!q || !k || !v || !log_alpha || !beta || !out))
+        return KDA_ERR_INVALID;
+    const void *ptrs[] = {q, k, v, log_alpha, beta, S0, cu_seqlens, out, S_final, workspace};
+    for (const void *x : ptrs)
+        if (x && !aligned16(x)) return KDA_ERR_ALIGN;
+    if (!workspace || ((uintptr_t)workspace & 255u) || ws_bytes < workspace_bytes(p))
+        return KDA_ERR_WORKSPACE;
+    // grid = N * H * (Dv / 32) CTAs must fit in gridDim.x
+    if ((long long)p->num_seqs * p->H * (p->Dv / 32) > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+    st = select_device(ptrs, 10);
+    if (st != KDA_OK) return st;
+
+    kda::ForwardArgs a;
+    a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta;
+    a.S0 = S0; a.cu_seqlens = cu_seqlens; a.out = out; a.S_final = S_final;
+    a.N = p->num_seqs; a.T = p->total_tokens; a.H = p->H; a.Dk = p->Dk; a.Dv = p->Dv;
+    a.io_dtype = p->io_dtype; a.gate_dtype = p->gate_dtype;
+    a.status = reinterpret_cast<int32_t *>(workspace);
+    a.order = reinterpret_cast<int32_t *>(static_cast<char *>(workspace) + kWsHeader);
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (kda::launch_varlen_index(a, s) != cudaSuccess) return KDA_ERR_CUDA;
+    if (kda::launch_prefill_simt(a, s) != cudaSuccess) return KDA_ERR_CUDA;
+    return KDA_OK;
+}
+
+kda_status kda_decode_step(const void *q, const void *k, const void *v, const void *log_alpha,
+                           const void *beta, float *S, void *out, const kda_params *p,
+                           void *stream) {
+    kda_status st = check_common(p);
+    if (st != KDA_OK) return st;
+    if (p->num_seqs == 0) return KDA_OK;
+    if (!q || !k || !v || !log_alpha || !beta || !S || !out) return KDA_ERR_INVALID;
+    const void *ptrs[] = {q, k, v, log_alpha, beta, S, out};
+    for (const void *x : ptrs)
+        if (!aligned16(x)) return KDA_ERR_ALIGN;
+    if ((long long)p->num_seqs * p->H * (p->Dv / 64) > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+    st = select_device(ptrs, 7);
+    if (st != KDA_OK) return st;
+
+    kda::DecodeArgs a;
+    a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta; a.S = S; a.out = out;
+    a.N = p->num_seqs; a.H = p->H; a.Dk = p->Dk; a.Dv = p->Dv;
+    a.io_dtype = p->io_dtype; a.gate_dtype = p->gate_dtype;
+    if (kda::launch_decode(a, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    return KDA_OK;
+}
+
+kda_status kda_workspace_status(const void *workspace, int32_t *status, void *stream) {
+    if (!workspace || !status) return KDA_ERR_INVALID;
+    const void *ptrs[] = {workspace};
+    kda_status st = select_device(ptrs, 1);
+    if (st != KDA_OK) return st;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return KDA_ERR_CUDA;
+    if (cudaMemcpy(status, workspace, sizeof(int32_t), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    return KDA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,65 @@
+// kda_internal.cuh -- shared declarations of the KDA CUDA library (not public).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kda.h"
+
+namespace kda {
+
+constexpr int kChunk = 64;          // tokens per chunk of the prefill
+constexpr size_t kWsHeader = 256;   // bytes: status word + padding
+constexpr int kSortMax = 4096;      // sequences ordered longest-first up to this N
+
+// Everything a prefill launch needs, already validated on the host.
+struct ForwardArgs {
+    const void *q, *k, *v, *log_alpha, *beta;
+    const float *S0;
+    const int32_t *cu_seqlens;
+    void *out;
+    float *S_final;
+    int N, T, H, Dk, Dv;
+    int io_dtype, gate_dtype;
+    int32_t *status;   // device status word (workspace)
+    int32_t *order;    // device work order [N] (workspace)
+};
+
+struct DecodeArgs {
+    const void *q, *k, *v, *log_alpha, *beta;
+    float *S;
+    void *out;
+    int N, H, Dk, Dv;
+    int io_dtype, gate_dtype;
+};
+
+cudaError_t launch_varlen_index(const ForwardArgs &a, cudaStream_t s);
+cudaError_t launch_prefill_simt(const ForwardArgs &a, cudaStream_t s);
+cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
+
+// ---------------------------------------------------------------------------
+// small device helpers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+// Record the first error code seen by any thread; later codes are dropped.
+__device__ __forceinline__ void set_status(int32_t *status, int32_t code) {
+    if (status) atomicCAS(status, 0, code);
+}
+
+// Token range of sequence n, or false when cu_seqlens is malformed there.
+__device__ __forceinline__ bool seq_range(const int32_t *cu, int n, int T, int &t0, int &t1) {
+    t0 = cu[n];
+    t1 = cu[n + 1];
+    return t0 >= 0 && t1 >= t0 && t1 <= T;
+}
+
+}  // namespace kda

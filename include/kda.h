@@ -1,0 +1,162 @@
+/*
+ * kda.h -- C ABI of the B200 (sm_100a) Kimi Delta Attention library.
+ *
+ * The operator.  The page "Kimi K3: Open Frontier Intelligence and
+ * Implementation Framework" (section "Technical Architecture and Scaling
+ * Efficiency", sub-section "Hybrid Attention Mechanism", KDA bullet)
+ * describes Kimi Delta Attention as the delta-rule recurrence extended with
+ * a channel-wise forget gate whose decay is bounded below, which lets the
+ * diagonal and off-diagonal tiles of a chunked evaluation run as dense
+ * tensor-core products.  Per head, with a d_k x d_v state S:
+ *
+ *     S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T
+ *     o_t = S_t^T q_t,            alpha_t = exp(log_alpha_t) per channel.
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the
+ *     library never allocates, frees or retains them.  Every tensor is dense
+ *     row-major and its base address must be 16-byte aligned.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Work is enqueued asynchronously; the call returns once it is
+ *     enqueued.
+ *   - Host-side validation (NULL pointers, alignment, sizes, dtypes) is done
+ *     before anything is enqueued and returns a kda_status synchronously;
+ *     nothing runs on the device when a call returns an error.
+ *   - Launch failures return KDA_ERR_CUDA.  Problems only the device can see
+ *     (malformed cu_seqlens contents) are written to a status word in the
+ *     workspace, read back with kda_workspace_status().
+ *   - Token axis: sequences are packed back to back along a token axis of
+ *     length total_tokens and delimited by cu_seqlens.
+ *   - Supported shapes: Dk, Dv in {64, 128}; chunk == 64; H >= 1.
+ *   - The factorisation exp(g_r - g_s) = exp(g_r) * exp(-g_s) used inside a
+ *     chunk needs the in-chunk cumulative log-decay of every channel to stay
+ *     above -80 (fp32 exponent range): e.g. alpha >= exp(-1.25) per token at
+ *     chunk 64.  That is the lower bound on the decay the method relies on;
+ *     the library does not clamp log_alpha.
+ */
+#ifndef KDA_H
+#define KDA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define KDA_ABI_VERSION 1
+
+typedef enum kda_status {
+    KDA_OK = 0,
+    KDA_ERR_INVALID = 1,      /* NULL pointer, non-positive size, bad value      */
+    KDA_ERR_UNSUPPORTED = 2,  /* Dk/Dv/chunk/dtype combination not implemented    */
+    KDA_ERR_ALIGN = 3,        /* a tensor base address is not 16-byte aligned     */
+    KDA_ERR_WORKSPACE = 4,    /* workspace NULL, misaligned or too small          */
+    KDA_ERR_CUDA = 5,         /* a CUDA runtime call or kernel launch failed      */
+    KDA_ERR_TIMEOUT = 6,      /* a bounded device-side wait gave up               */
+    KDA_ERR_SEQLENS = 7       /* device saw cu_seqlens not 0..total_tokens monotone */
+} kda_status;
+
+typedef enum kda_dtype {
+    KDA_F32 = 0,
+    KDA_BF16 = 1
+} kda_dtype;
+
+/* Problem description shared by kda_forward and kda_decode_step. */
+typedef struct kda_params {
+    int32_t num_seqs;      /* N: number of sequences (prefill) or decode rows   */
+    int32_t total_tokens;  /* T_tot: packed token count (prefill); ignored by decode */
+    int32_t H;             /* heads                                            */
+    int32_t Dk;            /* key / query width: 64 or 128                     */
+    int32_t Dv;            /* value width: 64 or 128                           */
+    int32_t chunk;         /* prefill chunk length; must be 64                 */
+    int32_t io_dtype;      /* kda_dtype of q, k, v and out                     */
+    int32_t gate_dtype;    /* kda_dtype of log_alpha and beta                  */
+    int32_t flags;         /* 0, or KDA_FLAG_* bits below                      */
+} kda_params;
+
+/* Evaluate a bf16 problem with the fp32 CUDA-core prefill instead of the
+ * tensor-core one (slower; for cross-checking the two kernels). */
+#define KDA_FLAG_FORCE_SIMT 1
+
+/*
+ * kda_forward_workspace_size -- bytes of device workspace kda_forward needs
+ * for this problem (a status word, the per-sequence work order).  Returns 0
+ * when `p` is NULL or invalid.  The workspace must be 256-byte aligned; its
+ * contents need no initialisation and are overwritten by every call.
+ */
+size_t kda_forward_workspace_size(const kda_params *p);
+
+/*
+ * kda_forward -- chunked (chunk = 64) prefill over packed sequences.
+ *
+ * Computes, for every sequence n in [0, N) and head h, the recurrence above
+ * over tokens cu_seqlens[n] .. cu_seqlens[n+1]-1 starting from S0[n,h]
+ * (zero when S0 is NULL), writing o_t for every token and the state after
+ * the sequence's last token to S_final[n,h] (skipped when S_final is NULL).
+ * A zero-length sequence leaves S_final[n,h] = S0[n,h].
+ *
+ *   q, k       [T_tot, H, Dk]  io_dtype
+ *   v          [T_tot, H, Dv]  io_dtype
+ *   log_alpha  [T_tot, H, Dk]  gate_dtype   (natural log of the decay, <= 0)
+ *   beta       [T_tot, H]      gate_dtype   (write strength, usually in [0,1])
+ *   S0         [N, H, Dk, Dv]  fp32, or NULL for a zero initial state
+ *   cu_seqlens [N + 1]         int32, device; 0 = c_0 <= c_1 <= ... <= c_N = T_tot
+ *   out        [T_tot, H, Dv]  io_dtype, written
+ *   S_final    [N, H, Dk, Dv]  fp32, written, or NULL
+ *   workspace  device scratch of ws_bytes >= kda_forward_workspace_size(p)
+ *
+ * Aliasing: out and S_final must not overlap any input.  S_final may be the
+ * same buffer as S0 (in-place continuation of a chain); any other partial
+ * overlap is undefined.  Calls that share a workspace must be ordered on the
+ * same stream.
+ *
+ * Errors: KDA_ERR_INVALID / _UNSUPPORTED / _ALIGN / _WORKSPACE from host
+ * validation; KDA_ERR_CUDA if a launch fails.  If cu_seqlens is malformed
+ * the kernels skip the offending sequences (no out-of-range access) and
+ * record KDA_ERR_SEQLENS in the workspace status word.
+ */
+kda_status kda_forward(const void *q, const void *k, const void *v,
+                       const void *log_alpha, const void *beta,
+                       const float *S0, const int32_t *cu_seqlens,
+                       void *out, float *S_final, const kda_params *p,
+                       void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * kda_decode_step -- one recurrent token for N independent sequences.
+ *
+ * For every n < N (= p->num_seqs) and head h, applies one token of the
+ * recurrence to S[n,h] in place and writes its output:
+ *
+ *   q, k, log_alpha [N, H, Dk]  (io_dtype for q/k, gate_dtype for log_alpha)
+ *   v               [N, H, Dv]  io_dtype
+ *   beta            [N, H]      gate_dtype
+ *   S               [N, H, Dk, Dv] fp32, read and overwritten
+ *   out             [N, H, Dv]  io_dtype, written
+ *
+ * p->total_tokens and p->chunk are ignored.  S must not overlap any other
+ * argument.  The state of each (n, h) is read once and written once per call.
+ */
+kda_status kda_decode_step(const void *q, const void *k, const void *v,
+                           const void *log_alpha, const void *beta, float *S,
+                           void *out, const kda_params *p, void *stream);
+
+/*
+ * kda_workspace_status -- synchronise `stream`, then copy the device status
+ * word of a kda_forward workspace into *status (KDA_OK when the last call
+ * that used this workspace saw nothing wrong).  Returns KDA_ERR_INVALID for
+ * NULL arguments and KDA_ERR_CUDA if the copy fails.
+ */
+kda_status kda_workspace_status(const void *workspace, int32_t *status, void *stream);
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char *kda_status_string(kda_status s);
+
+/* KDA_ABI_VERSION of the loaded library. */
+int32_t kda_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H */

@@ -1,0 +1,113 @@
+"""Host-only checks of the C ABI (no GPU): the library loads, exports every
+function ``include/kda.h`` declares, and rejects malformed calls with the
+documented status codes before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import gated_delta_rule_113_b200 as kda
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
+
+
+def _declared_functions():
+    names = set()
+    for fn in os.listdir(HEADER):
+        if fn.endswith(".h"):
+            text = open(os.path.join(HEADER, fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(kda_[a-z0-9_]+)\s*\(", text))
+    return sorted(names)
+
+
+def test_library_loads_and_exports_every_declared_symbol():
+    lib = kda.load_library()
+    declared = _declared_functions()
+    assert declared, "no declarations parsed from include/*.h"
+    for name in declared:
+        assert hasattr(lib, name), f"{name} declared in include/ but not exported"
+    assert set(kda.EXPORTED_SYMBOLS) <= set(declared)
+    assert lib.kda_abi_version() == 1
+
+
+def test_status_strings():
+    lib = kda.load_library()
+    for code in range(0, 8):
+        assert lib.kda_status_string(code).startswith(b"KDA_")
+    assert lib.kda_status_string(1234) == b"KDA_ERR_UNKNOWN"
+
+
+def _params(**kw):
+    base = dict(num_seqs=2, total_tokens=128, H=4, Dk=128, Dv=128, chunk=64,
+                io_dtype=1, gate_dtype=1, flags=0)
+    base.update(kw)
+    return kda.Params(**base)
+
+
+def test_workspace_size():
+    lib = kda.load_library()
+    p = _params(num_seqs=1000)
+    assert lib.kda_forward_workspace_size(ctypes.byref(p)) >= 256 + 4 * 1000
+    assert lib.kda_forward_workspace_size(None) == 0
+    assert lib.kda_forward_workspace_size(ctypes.byref(_params(Dk=96))) == 0
+
+
+FAKE = 0x10000  # 16-byte aligned non-null address; never dereferenced on these paths
+
+
+def _fwd(lib, p, **over):
+    args = dict(q=FAKE, k=FAKE, v=FAKE, la=FAKE, beta=FAKE, S0=None, cu=FAKE, out=FAKE,
+                Sf=None, ws=0x20000, ws_bytes=1 << 20)
+    args.update(over)
+    vp = ctypes.c_void_p
+    return lib.kda_forward(vp(args["q"]), vp(args["k"]), vp(args["v"]), vp(args["la"]),
+                           vp(args["beta"]), vp(args["S0"]), vp(args["cu"]), vp(args["out"]),
+                           vp(args["Sf"]), ctypes.byref(p), vp(args["ws"]), args["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("over,params,code", [
+    (dict(q=None), {}, 1),
+    (dict(cu=None), {}, 1),
+    (dict(out=None), {}, 1),
+    ({}, dict(H=0), 1),
+    ({}, dict(num_seqs=-1), 1),
+    ({}, dict(flags=8), 1),
+    ({}, dict(Dk=96), 2),
+    ({}, dict(Dv=256), 2),
+    ({}, dict(chunk=32), 2),
+    ({}, dict(io_dtype=5), 2),
+    (dict(q=FAKE + 4), {}, 3),
+    (dict(S0=FAKE + 8), {}, 3),
+    (dict(ws=None), {}, 4),
+    (dict(ws=0x20010), {}, 4),
+    (dict(ws_bytes=16), {}, 4),
+])
+def test_forward_host_validation(over, params, code):
+    lib = kda.load_library()
+    assert _fwd(lib, _params(**params), **over) == code
+
+
+def test_forward_empty_problem_is_noop():
+    lib = kda.load_library()
+    assert _fwd(lib, _params(num_seqs=0, total_tokens=0), q=None, cu=None, out=None, ws=None) == 0
+    assert _fwd(lib, _params(num_seqs=0, total_tokens=5)) == 1
+
+
+def test_decode_host_validation():
+    lib = kda.load_library()
+    vp = ctypes.c_void_p
+    call = lambda p, **o: lib.kda_decode_step(*(vp(o.get(n, FAKE)) for n in
+                                                ("q", "k", "v", "la", "b", "S", "out")),
+                                              ctypes.byref(p), None)
+    assert call(_params(Dk=32)) == 2
+    assert call(_params(), S=None) == 1
+    assert call(_params(), out=FAKE + 2) == 3
+    assert call(_params(num_seqs=0)) == 0
+
+
+def test_workspace_status_null_args():
+    lib = kda.load_library()
+    st = ctypes.c_int32(0)
+    assert lib.kda_workspace_status(None, ctypes.byref(st), None) == 1

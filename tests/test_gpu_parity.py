@@ -1,0 +1,212 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the
+same seeded inputs.  Small cases compare every element; full-size workloads
+compare every output of sampled (sequence, head) chains, which the oracle
+computes exactly as it would inside the full problem (chains are
+independent)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import gated_delta_rule_113_b200 as kda
+import oracle
+from gated_delta_rule_113_b200.inputs import WORKLOADS, decode_inputs, forward_inputs
+from helpers import as_np, err, head_slice, rel_fro, to_dev, tol
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(inp, force_simt=False, **kw):
+    d = to_dev(inp)
+    out, sf = kda.forward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["S0"],
+                          d["cu_seqlens"], force_simt=force_simt, **kw)
+    torch.cuda.synchronize()
+    return out, sf
+
+
+def _oracle(inp):
+    return oracle.forward(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"],
+                          inp["S0"], inp["cu_seqlens"].numpy())
+
+
+def _check(inp, out, sf, io_dtype, heads=None):
+    ref = head_slice(inp, heads) if heads is not None else inp
+    ro, rs = _oracle(ref)
+    go, gs = as_np(out), as_np(sf)
+    if heads is not None:
+        go, gs = go[:, list(heads)], gs[:, list(heads)]
+    e_o, e_s = err(go, ro, io_dtype), err(gs, rs, io_dtype)
+    assert e_o <= tol(io_dtype), f"out error {e_o:.3e}"
+    assert e_s <= tol(io_dtype), f"S_final error {e_s:.3e}"
+    return e_o, e_s
+
+
+# ---------------------------------------------------------------- small cases
+def test_workload0_fp32_full():
+    w = WORKLOADS[0]
+    inp = forward_inputs(w)
+    out, sf = _run(inp)
+    _check(inp, out, sf, torch.float32)
+
+
+@pytest.mark.parametrize("force_simt", [False, True])
+def test_bf16_ragged_multi_chunk(force_simt):
+    w = WORKLOADS[1]
+    inp = forward_inputs(w, lengths=[300, 201], H=4)
+    out, sf = _run(inp, force_simt=force_simt)
+    _check(inp, out, sf, torch.bfloat16)
+
+
+@pytest.mark.parametrize("dtype_idx", [0, 1])
+def test_varlen_edge_lengths(dtype_idx):
+    w = WORKLOADS[dtype_idx]
+    lens = [1, 63, 64, 65, 0, 130, 128, 2]
+    inp = forward_inputs(w, lengths=lens, H=2, s0=True)
+    out, sf = _run(inp)
+    _check(inp, out, sf, w.torch_dtype)
+    # zero-length sequence: S_final == S0 exactly
+    assert torch.equal(sf[4].cpu(), inp["S0"][4])
+
+
+@pytest.mark.parametrize("dk,dv", [(64, 128), (128, 64)])
+def test_mixed_widths(dk, dv):
+    import dataclasses
+    w = dataclasses.replace(WORKLOADS[1], Dk=dk, Dv=dv)
+    inp = forward_inputs(w, lengths=[190, 64], H=3)
+    out, sf = _run(inp)
+    _check(inp, out, sf, torch.bfloat16)
+
+
+def test_fp32_io_bf16_gates_and_no_initial_state():
+    w = WORKLOADS[0]
+    inp = forward_inputs(w, lengths=[150], H=2, s0=False)
+    inp["log_alpha"] = inp["log_alpha"].to(torch.bfloat16)
+    inp["beta"] = inp["beta"].to(torch.bfloat16)
+    out, sf = _run(inp)
+    _check(inp, out, sf, torch.float32)
+
+
+def test_split_chain_gpu():
+    w = WORKLOADS[1]
+    inp = forward_inputs(w, lengths=[384], H=2)
+    d = to_dev(inp)
+    out, sf = kda.forward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["S0"])
+    t0 = 192  # chunk-aligned split
+    sl = lambda x, a, b: x[a:b].contiguous()
+    o1, s1 = kda.forward(*(sl(d[n], 0, t0) for n in ("q", "k", "v", "log_alpha", "beta")), d["S0"])
+    o2, s2 = kda.forward(*(sl(d[n], t0, 384) for n in ("q", "k", "v", "log_alpha", "beta")), s1)
+    assert rel_fro(as_np(torch.cat([o1, o2])), as_np(out)) < 1e-2
+    assert rel_fro(as_np(s2), as_np(sf)) < 1e-2
+
+
+def test_in_place_state_continuation():
+    """S_final may be the same buffer as S0."""
+    w = WORKLOADS[0]
+    inp = forward_inputs(w, lengths=[100, 37], H=2, s0=True)
+    d = to_dev(inp)
+    ref_o, ref_s = kda.forward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["S0"],
+                               d["cu_seqlens"])
+    S = d["S0"].clone()
+    o, s = kda.forward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], S, d["cu_seqlens"],
+                       S_final=S)
+    torch.cuda.synchronize()
+    assert torch.equal(o, ref_o) and torch.equal(S, ref_s)
+
+
+def test_exact_write_invariant_gpu():
+    """beta = 1, q = k = unit coordinate axis: the output reproduces v (any decay)."""
+    T, H, D = 200, 2, 128
+    g = torch.Generator().manual_seed(5)
+    idx = torch.randint(0, D, (T, H), generator=g)
+    k = torch.nn.functional.one_hot(idx, D).to(torch.bfloat16)
+    v = torch.randn(T, H, D, generator=g).to(torch.bfloat16)
+    la = (torch.rand(T, H, D, generator=g) * math.log(0.9)).to(torch.bfloat16)
+    beta = torch.ones(T, H, dtype=torch.bfloat16)
+    S0 = 0.02 * torch.randn(1, H, D, D, generator=g)
+    inp = dict(q=k.clone(), k=k, v=v, log_alpha=la, beta=beta, S0=S0,
+               cu_seqlens=torch.tensor([0, T], dtype=torch.int32))
+    out, _ = _run(inp)
+    assert rel_fro(as_np(out), as_np(v)) < 1e-2
+
+
+def test_value_channel_permutation():
+    w = WORKLOADS[1]
+    inp = forward_inputs(w, lengths=[130], H=2)
+    perm = torch.randperm(128, generator=torch.Generator().manual_seed(1))
+    out, sf = _run(inp)
+    inp2 = dict(inp, v=inp["v"][..., perm].contiguous(), S0=inp["S0"][..., perm].contiguous())
+    out2, sf2 = _run(inp2)
+    assert rel_fro(as_np(out2), as_np(out[..., perm.cuda()])) < 1e-3
+    assert rel_fro(as_np(sf2), as_np(sf[..., perm.cuda()])) < 1e-3
+
+
+def test_deterministic_reruns():
+    w = WORKLOADS[1]
+    inp = forward_inputs(w, lengths=[257, 64], H=4)
+    a = _run(inp)
+    b = _run(inp)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+def test_malformed_seqlens_reported_not_faulting():
+    w = WORKLOADS[1]
+    inp = forward_inputs(w, lengths=[64, 64], H=2)
+    d = to_dev(inp)
+    bad = torch.tensor([0, 100, 90], dtype=torch.int32, device="cuda")  # decreasing, wrong end
+    ws = torch.empty(kda.forward_workspace_size(2, 128, 2, 128, 128), dtype=torch.uint8,
+                     device="cuda")
+    kda.forward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["S0"], bad, workspace=ws)
+    assert kda.workspace_status(ws) == 7
+    good = d["cu_seqlens"]
+    kda.forward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["S0"], good, workspace=ws)
+    assert kda.workspace_status(ws) == 0
+
+
+# ------------------------------------------------------------------- decode
+def test_decode_small_all_elements():
+    w = WORKLOADS[4]
+    inp = decode_inputs(w, steps=6, N=8, H=4)
+    S = inp["S"].cuda()
+    S_ref = inp["S"].double().numpy()
+    for t in range(6):
+        args = [inp[n][t].cuda() for n in ("q", "k", "v", "log_alpha", "beta")]
+        out = kda.decode_step(*args, S)
+        ro, S_ref = oracle.decode_step(*(inp[n][t] for n in ("q", "k", "v", "log_alpha", "beta")),
+                                       S_ref)
+        assert rel_fro(as_np(out), ro) < 2e-2
+    assert rel_fro(as_np(S), S_ref) < 2e-2
+
+
+def test_decode_fp32_all_elements():
+    import dataclasses
+    w = dataclasses.replace(WORKLOADS[4], io_dtype="f32", Dk=64, Dv=128)
+    inp = decode_inputs(w, steps=4, N=3, H=2)
+    S = inp["S"].cuda()
+    S_ref = inp["S"].double().numpy()
+    for t in range(4):
+        out = kda.decode_step(*(inp[n][t].cuda() for n in ("q", "k", "v", "log_alpha", "beta")), S)
+        ro, S_ref = oracle.decode_step(*(inp[n][t] for n in ("q", "k", "v", "log_alpha", "beta")),
+                                       S_ref)
+        assert np.max(np.abs(as_np(out) - ro)) / np.max(np.abs(ro)) < 1e-4
+    assert np.max(np.abs(as_np(S) - S_ref)) / np.max(np.abs(S_ref)) < 1e-4
+
+
+def test_decode_equals_prefill():
+    """64 decode steps from S equal one prefill over those 64 tokens from S0 = S."""
+    w = WORKLOADS[4]
+    steps, N, H = 64, 4, 2
+    inp = decode_inputs(w, steps=steps, N=N, H=H)
+    S = inp["S"].cuda()
+    outs = []
+    for t in range(steps):
+        outs.append(kda.decode_step(*(inp[n][t].cuda() for n in ("q", "k", "v", "log_alpha",
+                                                                  "beta")), S))
+    dec_out = torch.stack(outs, 1)  # [N, steps, H, Dv]
+    pk = lambda n: inp[n].transpose(0, 1).reshape(N * steps, *inp[n].shape[2:]).contiguous().cuda()
+    cu = torch.arange(0, N * steps + 1, steps, dtype=torch.int32, device="cuda")
+    p_out, p_s = kda.forward(pk("q"), pk("k"), pk("v"), pk("log_alpha"), pk("beta"),
+                             inp["S"].cuda(), cu)
+    torch.cuda.synchronize()
+    assert rel_fro(as_np(dec_out.reshape(N * steps, H, -1)), as_np(p_out)) < 1e-2
+    assert rel_fro(as_np(S), as_np(p_s)) < 1e-2

@@ -129,6 +129,11 @@ class ClockSampler:
         for line in self.proc.stdout:
             self.lines.append(line.strip())
 
+    def wait_first(self, timeout=3.0):
+        t0 = time.time()
+        while self.proc is not None and not self.lines and time.time() - t0 < timeout:
+            time.sleep(0.02)
+
     def __exit__(self, *exc):
         if self.proc is not None:
             self.proc.terminate()
@@ -289,8 +294,16 @@ def bench_kda(args):
 
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    barrier(world)
     with ClockSampler(local) as clk:
+        # keep the GPU busy (untimed) until the sampler reports, so the clock
+        # samples describe the loaded GPU around the timed region
+        clk.wait_first()
+        t_end = time.time() + 0.3
+        while time.time() < t_end:
+            flush.zero_()
+            step()
+            torch.cuda.synchronize()
+        barrier(world)
         for i in range(args.steps):
             flush.zero_()
             starts[i].record(stream)

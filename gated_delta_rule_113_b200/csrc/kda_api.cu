@@ -106,7 +106,9 @@ kda_status kda_forward(const void *q, const void *k, const void *v, const void *
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (kda::launch_varlen_index(a, s) != cudaSuccess) return KDA_ERR_CUDA;
-    if (kda::launch_prefill_simt(a, s) != cudaSuccess) return KDA_ERR_CUDA;
+    const bool tc = !(p->flags & KDA_FLAG_FORCE_SIMT) && kda::prefill_tc_supported(a);
+    if ((tc ? kda::launch_prefill_tc(a, s) : kda::launch_prefill_simt(a, s)) != cudaSuccess)
+        return KDA_ERR_CUDA;
     return KDA_OK;
 }
 

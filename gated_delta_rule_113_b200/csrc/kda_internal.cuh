@@ -36,6 +36,8 @@ struct DecodeArgs {
 
 cudaError_t launch_varlen_index(const ForwardArgs &a, cudaStream_t s);
 cudaError_t launch_prefill_simt(const ForwardArgs &a, cudaStream_t s);
+bool prefill_tc_supported(const ForwardArgs &a);
+cudaError_t launch_prefill_tc(const ForwardArgs &a, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
 
 // ---------------------------------------------------------------------------

@@ -53,13 +53,34 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
+// As above, but the waiting thread may stay suspended (not issuing) for up
+// to `hint_ns` nanoseconds while the phase is incomplete.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity,
+                                                    uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+
 // Bounded wait for the phase with the given parity.  ~2^22 polls, each of
 // which may itself block for a hardware-defined interval, is seconds of
 // wall time: far beyond any legitimate wait in these kernels.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
     for (uint32_t i = 0; i < (1u << 22); ++i) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (i > 64) __nanosleep(64);
+        if (i >= (1u << 14)) __nanosleep(128);
     }
     return false;
 }
@@ -223,6 +244,10 @@ __device__ __forceinline__ uint32_t to_tf32(float x) {
     return r;
 }
 
+// tf32 operand from an fp32 value without a conversion instruction: the MMA
+// reads only the sign, exponent and top 10 mantissa bits (round toward zero).
+__device__ __forceinline__ uint32_t tf32_bits(float x) { return __float_as_uint(x); }
+
 __device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], const uint32_t (&a)[4],
                                                 const uint32_t (&b)[2]) {
     asm volatile(
@@ -232,11 +257,41 @@ __device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], const uint32_t (&
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
+// ------------------------------------------------------ fast scalar math
+// Hardware approximations (MUFU): 2^x and 1/x, flushing denormals.
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Elementwise product of two packed bf16 pairs, rounded to nearest.
+__device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
 // ---------------------------------------------------------------- bf16 pack
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     uint32_t r;
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
     return r;
+}
+
+// Round-to-nearest-even bf16 packing on the integer ALU (keeps the
+// conversion pipe free); finite inputs only.
+__device__ __forceinline__ uint32_t pack_bf16_alu(float lo, float hi) {
+    const uint32_t a = __float_as_uint(lo), b = __float_as_uint(hi);
+    const uint32_t ra = a + 0x7FFFu + ((a >> 16) & 1u);
+    const uint32_t rb = b + 0x7FFFu + ((b >> 16) & 1u);
+    return __byte_perm(ra, rb, 0x7632);
 }
 
 __device__ __forceinline__ float bf16lo(uint32_t x) { return __uint_as_float(x << 16); }

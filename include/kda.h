@@ -123,6 +123,39 @@ kda_status kda_forward(const void *q, const void *k, const void *v,
                        void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * kda_forward_noalloc -- kda_forward for callers that cannot allocate device
+ * memory.  The KDA description has no counterpart to this; it is a
+ * convenience of this library.
+ *
+ * Some callers cannot hand kda_forward a workspace: engines whose device
+ * memory is planned once up front and that forbid allocation while serving,
+ * plug-ins running inside an application that owns the allocator, or
+ * latency-critical paths that cannot take cudaMalloc's implicit device
+ * synchronisation.  This entry point takes the same arguments as kda_forward
+ * minus the workspace and uses a fixed scratch array held by the library:
+ *
+ *   - the array holds a status word and KDA_NOALLOC_MAX_SEQS int32 entries;
+ *     every GPU that loads the library keeps it (about 64 KB) until exit;
+ *   - p->num_seqs > KDA_NOALLOC_MAX_SEQS is rejected with
+ *     KDA_ERR_UNSUPPORTED before anything is enqueued;
+ *   - the first call on a device looks up the array's device address (with
+ *     that device current); make that first call before any stream capture;
+ *   - every call shares the array and rewrites it before use; calls whose
+ *     work overlaps on the GPU race on it, so order them on one stream;
+ *   - it allocates nothing (no cudaMalloc, cudaFree or allocating library
+ *     call) and runs exactly the kernels of kda_forward.
+ *
+ * Returns the same codes as kda_forward.  Malformed cu_seqlens contents are
+ * still skipped safely on the device, but this path has no status readback.
+ */
+#define KDA_NOALLOC_MAX_SEQS 16384
+kda_status kda_forward_noalloc(const void *q, const void *k, const void *v,
+                               const void *log_alpha, const void *beta,
+                               const float *S0, const int32_t *cu_seqlens,
+                               void *out, float *S_final, const kda_params *p,
+                               void *stream);
+
+/*
  * kda_decode_step -- one recurrent token for N independent sequences.
  *
  * For every n < N (= p->num_seqs) and head h, applies one token of the

@@ -26,6 +26,7 @@ EXPORTED_SYMBOLS = ("kda_forward_workspace_size", "kda_forward", "kda_decode_ste
 
 KDA_F32, KDA_BF16 = 0, 1
 FLAG_FORCE_SIMT = 1
+FLAG_FUSED_TC = 2
 CHUNK = 64
 
 _lock = threading.Lock()
@@ -114,12 +115,14 @@ def forward_workspace_size(N: int, T: int, H: int, Dk: int, Dv: int,
 
 
 def forward(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, *, out=None, S_final=None,
-            workspace=None, output_final_state=True, force_simt=False):
+            workspace=None, output_final_state=True, force_simt=False, fused_tc=False):
     """Chunked KDA prefill through ``kda_forward``.
 
     q, k, log_alpha [T, H, Dk]; v [T, H, Dv]; beta [T, H]; S0 [N, H, Dk, Dv]
     fp32 or None; cu_seqlens int32 [N+1] on the device (None: one sequence).
     Returns (out [T, H, Dv] in q's dtype, S_final [N, H, Dk, Dv] fp32 or None).
+    ``force_simt`` / ``fused_tc`` select the CUDA-core or the single-kernel
+    tensor-core prefill instead of the default (for cross-checks).
     """
     lib = load_library()
     dev = q.device
@@ -142,7 +145,7 @@ def forward(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, *, out=None, S_f
     if S_final is None and output_final_state:
         S_final = torch.empty((N, H, Dk, Dv), dtype=torch.float32, device=dev)
     p = Params(N, T, H, Dk, Dv, CHUNK, _dt(q), _dt(log_alpha),
-               FLAG_FORCE_SIMT if force_simt else 0)
+               (FLAG_FORCE_SIMT if force_simt else 0) | (FLAG_FUSED_TC if fused_tc else 0))
     ws_bytes = int(lib.kda_forward_workspace_size(ctypes.byref(p)))
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)

@@ -19,7 +19,7 @@ kda_status check_common(const kda_params *p) {
     if (p->num_seqs < 0 || p->H <= 0) return KDA_ERR_INVALID;
     if (!dtype_ok(p->io_dtype) || !dtype_ok(p->gate_dtype)) return KDA_ERR_UNSUPPORTED;
     if (!width_ok(p->Dk) || !width_ok(p->Dv)) return KDA_ERR_UNSUPPORTED;
-    if (p->flags & ~KDA_FLAG_FORCE_SIMT) return KDA_ERR_INVALID;
+    if (p->flags & ~(KDA_FLAG_FORCE_SIMT | KDA_FLAG_FUSED_TC)) return KDA_ERR_INVALID;
     return KDA_OK;
 }
 
@@ -46,8 +46,26 @@ kda_status select_device(const void *const *ptrs, int n) {
     return KDA_OK;
 }
 
+// Workspace layout: [status header][order: N int32][chunk_off: N+1 int32]
+// [operand packets].  The first two parts are always needed; the last two
+// only by the two-pass tensor-core prefill.
 size_t workspace_bytes(const kda_params *p) {
     return kWsHeader + round_up(sizeof(int32_t) * (size_t)p->num_seqs, 256);
+}
+
+bool tc_shape(const kda_params *p) {
+    return p->io_dtype == KDA_BF16 && p->gate_dtype == KDA_BF16 && p->Dk == 128 && p->Dv == 128;
+}
+
+size_t chunk_off_offset(const kda_params *p) { return workspace_bytes(p); }
+
+size_t packets_offset(const kda_params *p) {
+    return chunk_off_offset(p) + round_up(sizeof(int32_t) * ((size_t)p->num_seqs + 1), 256);
+}
+
+size_t workspace_bytes_two_pass(const kda_params *p) {
+    return packets_offset(p) +
+           kda::packet_slots_bound(p->total_tokens, p->num_seqs, p->H) * kda::kPacketBytes;
 }
 
 }  // namespace
@@ -72,6 +90,9 @@ const char *kda_status_string(kda_status s) {
 
 size_t kda_forward_workspace_size(const kda_params *p) {
     if (check_common(p) != KDA_OK) return 0;
+    if (tc_shape(p) && !(p->flags & (KDA_FLAG_FORCE_SIMT | KDA_FLAG_FUSED_TC)) &&
+        p->total_tokens >= 0)
+        return workspace_bytes_two_pass(p);
     return workspace_bytes(p);
 }
 
@@ -103,12 +124,28 @@ kda_status kda_forward(const void *q, const void *k, const void *v, const void *
     a.io_dtype = p->io_dtype; a.gate_dtype = p->gate_dtype;
     a.status = reinterpret_cast<int32_t *>(workspace);
     a.order = reinterpret_cast<int32_t *>(static_cast<char *>(workspace) + kWsHeader);
+    a.chunk_off = nullptr;
+    a.packets = nullptr;
+    a.packet_slots = 0;
 
+    // bf16 with Dk = Dv = 128: tensor cores, two-pass when the workspace holds
+    // the operand packets, else the single fused kernel; otherwise CUDA cores.
+    const bool tc = !(p->flags & KDA_FLAG_FORCE_SIMT) && kda::prefill_tc_supported(a);
+    const bool two_pass =
+        tc && !(p->flags & KDA_FLAG_FUSED_TC) && ws_bytes >= workspace_bytes_two_pass(p);
+    if (two_pass) {
+        char *ws = static_cast<char *>(workspace);
+        a.chunk_off = reinterpret_cast<int32_t *>(ws + chunk_off_offset(p));
+        a.packets = reinterpret_cast<unsigned char *>(ws + packets_offset(p));
+        a.packet_slots = kda::packet_slots_bound(p->total_tokens, p->num_seqs, p->H);
+    }
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (kda::launch_varlen_index(a, s) != cudaSuccess) return KDA_ERR_CUDA;
-    const bool tc = !(p->flags & KDA_FLAG_FORCE_SIMT) && kda::prefill_tc_supported(a);
-    if ((tc ? kda::launch_prefill_tc(a, s) : kda::launch_prefill_simt(a, s)) != cudaSuccess)
-        return KDA_ERR_CUDA;
+    cudaError_t e;
+    if (two_pass) e = kda::launch_prefill_two_pass(a, s);
+    else if (tc) e = kda::launch_prefill_tc(a, s);
+    else e = kda::launch_prefill_simt(a, s);
+    if (e != cudaSuccess) return KDA_ERR_CUDA;
     return KDA_OK;
 }
 

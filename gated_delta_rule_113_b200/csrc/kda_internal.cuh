@@ -1,6 +1,7 @@
 // kda_internal.cuh -- shared declarations of the KDA CUDA library (not public).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -24,6 +25,9 @@ struct ForwardArgs {
     int io_dtype, gate_dtype;
     int32_t *status;   // device status word (workspace)
     int32_t *order;    // device work order [N] (workspace)
+    int32_t *chunk_off;    // device [N+1] exclusive prefix of per-sequence chunk counts, or null
+    unsigned char *packets;  // device per-(chunk, head) key-side operand packets, or null
+    size_t packet_slots;     // number of packets the workspace holds
 };
 
 struct DecodeArgs {
@@ -39,6 +43,19 @@ cudaError_t launch_prefill_simt(const ForwardArgs &a, cudaStream_t s);
 bool prefill_tc_supported(const ForwardArgs &a);
 cudaError_t launch_prefill_tc(const ForwardArgs &a, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
+cudaError_t launch_prefill_two_pass(const ForwardArgs &a, cudaStream_t s);
+
+// Two-pass tensor-core prefill: bytes of one key-side operand packet and the
+// number of packets a problem can need (one per 64-token chunk and head).
+constexpr size_t kPacketBytes = 66560;
+inline size_t packet_slots_bound(int64_t T, int64_t N, int64_t H) {
+    return (size_t)((T + kChunk - 1) / kChunk + N) * (size_t)H;
+}
+
+// TMA descriptor of a bf16 [T, H, D] tensor with a box of {box_x, 1, 64}
+// (innermost first) and a 32/64/128-byte swizzle (0 = none).
+bool make_tmap_bf16_3d(CUtensorMap *m, const void *base, int T, int H, int D, int box_x,
+                       int swizzle_bytes);
 
 // ---------------------------------------------------------------------------
 // small device helpers

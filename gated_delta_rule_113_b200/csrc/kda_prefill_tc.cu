@@ -37,12 +37,14 @@
 #include <cuda.h>
 
 #include "kda_internal.cuh"
+#include "kda_tc_common.cuh"
 #include "sm100.cuh"
 
 namespace kda {
 namespace {
 
 using namespace sm100;
+using namespace tc;
 
 // Optional per-chunk timeline of CTA 0 (clock64 per pipeline event), compiled
 // in only with -DKDA_TRACE for profiling builds; a no-op otherwise.
@@ -60,10 +62,6 @@ __device__ unsigned long long g_kda_trace[64 * 32];
 
 constexpr int kWarps = 19;
 constexpr int kThreads = kWarps * 32;
-constexpr int kDK = 128;           // key width handled by this kernel
-constexpr int kDV = 128;           // value width handled by this kernel
-constexpr int kLDL = 68;           // fp32 row stride of the solve scratch
-constexpr int kPrepThreads = 256;
 
 enum Role { kChain0 = 0, kPrep0 = 4, kSolve0 = 12, kTma = 16, kMmaK = 17, kMmaC = 18 };
 enum NamedBar { kBarPrep = 1, kBarSolve = 2 };
@@ -135,61 +133,6 @@ struct TcParams {
     int N, T, H;
 };
 
-__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity,
-                                              volatile int *abort_flag, int32_t *status) {
-    // Waiting threads stay suspended in try_wait (no issue slots taken from
-    // the warps doing work) and wake when the phase completes; a wait that
-    // outlasts 2 s of wall time gives up and flags the whole CTA.
-    if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t start = globaltimer_ns();
-    for (;;) {
-        if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
-        if (*abort_flag) return false;
-        if (globaltimer_ns() - start > 2000000000ull) break;
-    }
-    *abort_flag = 1;
-    set_status(status, KDA_ERR_TIMEOUT);
-    return false;
-}
-
-// 16-byte shared store / load helpers
-__device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
-                                       uint32_t d) {
-    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
-                 "r"(d)
-                 : "memory");
-}
-__device__ __forceinline__ uint4 lds128(uint32_t addr) {
-    uint4 v;
-    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "r"(addr)
-                 : "memory");
-    return v;
-}
-
-template <int VS>
-__device__ __forceinline__ uint32_t vs_off(uint32_t row, uint32_t chunk) {
-    return VS == 32 ? sw64_off(row, chunk) : sw128_off(row, chunk);
-}
-
-// B-operand descriptor of a VS-wide MN-major tile (rows = K) at K step 0;
-// step ks adds vs_step(ks) (start address field, in 16-byte units).
-template <int VS>
-__device__ __forceinline__ uint64_t vs_desc(uint32_t base, uint32_t rows) {
-    return VS == 32 ? smem_desc(base, rows * 64, 512, kSw64)
-                    : smem_desc(base, rows * 128, 1024, kSw128);
-}
-template <int VS>
-__device__ __forceinline__ uint64_t vs_step(int ks) {
-    return (uint64_t)(VS == 32 ? ks * 1024 : ks * 2048) >> 4;
-}
-// K-major 128B-swizzled operand with two 64-wide K atoms `atom` bytes apart
-__device__ __forceinline__ uint64_t kmaj_step(int ks, uint32_t atom) {
-    return (uint64_t)((ks >> 2) * atom + (ks & 3) * 32) >> 4;
-}
-
-__device__ __forceinline__ uint32_t pack2(float lo, float hi) { return pack_bf16(lo, hi); }
 
 template <int VS>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -305,114 +248,14 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         // ----------------------------------------------------------- prep
         // thread = (row group rg of 4 rows, channel group cg of 8 channels)
         const int t = tid - kPrep0 * 32;
-        const int cg = t & 15, rg = t >> 4;
-        const int a = cg >> 3, ch = cg & 7;
-        constexpr float kLog2e = 1.4426950408889634f;
         for (int n = 0; n < nchunks; ++n) {
             const int s = n & 1;
             const int c0 = t0 + n * kChunk;
             const int L = min(kChunk, t1 - c0);
             if (!wait_or_abort(&bars[bRawFull + s], (n >> 1) & 1, abort_flag, p.status)) break;
             if (t == 0) KDA_TRACE_EVENT(n, 1);
-            const uint32_t kq = sbase + Ly::kKQ + s * 32768 + a * 16384;
-            const uint32_t ki = sbase + Ly::kKI + s * 16384 + a * 8192;
-            // pass 0: alpha = 2^(la log2 e); in-group prefix and suffix products
-            float pre[4][8], suf[4][8];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int r = rg * 4 + i;
-                uint4 raw = lds128(ki + sw128_off(r, ch));
-                if (r >= L) raw = make_uint4(0, 0, 0, 0);  // past the end: alpha = 1
-                const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float la = (e & 1) ? bf16hi(w4[e >> 1]) : bf16lo(w4[e >> 1]);
-                    pre[i][e] = ex2_approx(la * kLog2e);   // alpha for now
-                }
-            }
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                float sx = 1.f;
-#pragma unroll
-                for (int i = 3; i >= 0; --i) {
-                    suf[i][e] = sx;          // prod_{j > i} alpha_j (within the group)
-                    sx *= pre[i][e];
-                }
-                float px = 1.f;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    px *= pre[i][e];
-                    pre[i][e] = px;          // prod_{j <= i} alpha_j
-                }
-            }
-            {
-                float *gpp = sGP + rg * 128 + cg * 8;
-                *reinterpret_cast<float4 *>(gpp) = make_float4(pre[3][0], pre[3][1], pre[3][2], pre[3][3]);
-                *reinterpret_cast<float4 *>(gpp + 4) = make_float4(pre[3][4], pre[3][5], pre[3][6], pre[3][7]);
-            }
-            if (t == 0) KDA_TRACE_EVENT(n, 29);
-            named_bar(kBarPrep, kPrepThreads);
-            // scan over the 16 row groups, one thread per channel:
-            // sGP <- exclusive prefix, sSUF <- exclusive suffix, sGL <- total
-            if (t < 128) {
-                float gv[16];
-#pragma unroll
-                for (int g = 0; g < 16; ++g) gv[g] = sGP[g * 128 + t];
-                float px = 1.f;
-#pragma unroll
-                for (int g = 0; g < 16; ++g) {
-                    sGP[g * 128 + t] = px;
-                    px *= gv[g];
-                }
-                sGL[s * 128 + t] = px;
-                float sx = rcp_approx(px);   // 1/Gam_L, once per channel
-#pragma unroll
-                for (int g = 15; g >= 0; --g) {
-                    sSUF[g * 128 + t] = sx;
-                    sx *= gv[g];
-                }
-            } else if (t < 128 + kChunk) {
-                const int r = t - 128;
-                sB[s * 64 + r] = r < L ? __bfloat162float(p.beta[(size_t)(c0 + r) * p.H + h]) : 0.f;
-            }
-            named_bar(kBarPrep, kPrepThreads);
-            // pass 1: Gam_r = pre_group * pre[i]; 1/Gam_r = (1/Gam_L) suf_group suf[i]
-            float ef[8], ci[8];
-            {
-                const float4 *pp = reinterpret_cast<const float4 *>(sGP + rg * 128 + cg * 8);
-                const float4 *sp = reinterpret_cast<const float4 *>(sSUF + rg * 128 + cg * 8);
-                const float4 p0 = pp[0], p1 = pp[1], q0 = sp[0], q1 = sp[1];
-                ef[0] = p0.x; ef[1] = p0.y; ef[2] = p0.z; ef[3] = p0.w;
-                ef[4] = p1.x; ef[5] = p1.y; ef[6] = p1.z; ef[7] = p1.w;
-                ci[0] = q0.x; ci[1] = q0.y; ci[2] = q0.z; ci[3] = q0.w;
-                ci[4] = q1.x; ci[5] = q1.y; ci[6] = q1.z; ci[7] = q1.w;
-            }
-            // the next chunk's pass 0 overwrites sGP: everyone must have read it
-            named_bar(kBarPrep, kPrepThreads);
-            if (t == 0) KDA_TRACE_EVENT(n, 30);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int r = rg * 4 + i;
-                uint32_t gb[4], gib[4];
-#pragma unroll
-                for (int e2 = 0; e2 < 4; ++e2) {
-                    gb[e2] = pack_bf16_alu(ef[2 * e2] * pre[i][2 * e2], ef[2 * e2 + 1] * pre[i][2 * e2 + 1]);
-                    gib[e2] = pack_bf16_alu(ci[2 * e2] * suf[i][2 * e2], ci[2 * e2 + 1] * suf[i][2 * e2 + 1]);
-                }
-                if (r >= L) {  // rows past the end of the sequence are zero
-#pragma unroll
-                    for (int e2 = 0; e2 < 4; ++e2) gb[e2] = gib[e2] = 0u;
-                }
-                const uint32_t ka = kq + sw128_off(r, ch), qa = ka + 8192;
-                const uint4 kr = lds128(ka), qr = lds128(qa);
-                sts128(ki + sw128_off(r, ch), mul_bf16x2(kr.x, gib[0]), mul_bf16x2(kr.y, gib[1]),
-                       mul_bf16x2(kr.z, gib[2]), mul_bf16x2(kr.w, gib[3]));
-                sts128(ka, mul_bf16x2(kr.x, gb[0]), mul_bf16x2(kr.y, gb[1]), mul_bf16x2(kr.z, gb[2]),
-                       mul_bf16x2(kr.w, gb[3]));
-                sts128(qa, mul_bf16x2(qr.x, gb[0]), mul_bf16x2(qr.y, gb[1]), mul_bf16x2(qr.z, gb[2]),
-                       mul_bf16x2(qr.w, gb[3]));
-            }
-            fence_proxy_async();
+            prep_chunk(t, sbase + Ly::kKQ + s * 32768, sbase + Ly::kKI + s * 16384, sGP, sSUF,
+                       sGL + s * 128, sB + s * 64, p.beta, c0, L, p.H, h, kBarPrep);
             __syncwarp();
             if (t == 0) KDA_TRACE_EVENT(n, 2);
             if (lane == 0) mbar_arrive(&bars[bKqFull + s]);
@@ -421,202 +264,13 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         // ---------------------------------------------------------- solve
         const int sw = warp - kSolve0;        // 0..3, TMEM lanes 32*sw..
         const int t = tid - kSolve0 * 32;     // 0..127
-        const int g = lane >> 2, tq = lane & 3;
         for (int n = 0; n < nchunks; ++n) {
             const int s = n & 1;
             if (!wait_or_abort(&bars[bApFull], n & 1, abort_flag, p.status)) break;
             tc_fence_after();
             if (t == 0) KDA_TRACE_EVENT(n, 4);
-            const uint32_t tp = sbase + Ly::kTP + s * 24576;
-            {
-                const int r = 32 * (sw & 1) + lane;  // row within A (sw<2) or P (sw>=2)
-                uint32_t v0[32], v1[32];
-                tmem_ld32(tmem_addr(tmem, 32 * sw, Ly::kTmAP), v0);
-                tmem_ld32(tmem_addr(tmem, 32 * sw, Ly::kTmAP + 32), v1);
-                tmem_wait_ld();
-                if (t == 0) KDA_TRACE_EVENT(n, 24);
-                if (sw < 2) {
-                    // L = strict_lower(diag(b) A)
-                    const float br = sB[s * 64 + r];
-                    float *Lr = sL + r * kLDL;
-#pragma unroll
-                    for (int c = 0; c < 64; c += 4) {
-                        const uint32_t *src = c < 32 ? &v0[c] : &v1[c - 32];
-                        float4 w;
-                        w.x = (c + 0 < r) ? br * __uint_as_float(src[0]) : 0.f;
-                        w.y = (c + 1 < r) ? br * __uint_as_float(src[1]) : 0.f;
-                        w.z = (c + 2 < r) ? br * __uint_as_float(src[2]) : 0.f;
-                        w.w = (c + 3 < r) ? br * __uint_as_float(src[3]) : 0.f;
-                        *reinterpret_cast<float4 *>(Lr + c) = w;
-                    }
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        uint32_t o[4];
-#pragma unroll
-                        for (int e2 = 0; e2 < 4; ++e2) {
-                            const int c = 8 * j + 2 * e2;
-                            const uint32_t *src = c < 32 ? &v0[c] : &v1[c - 32];
-                            const float x0 = (c <= r) ? __uint_as_float(src[0]) : 0.f;
-                            const float x1 = (c + 1 <= r) ? __uint_as_float(src[1]) : 0.f;
-                            o[e2] = pack2(x0, x1);
-                        }
-                        sts128(tp + 16384 + sw128_off(r, j), o[0], o[1], o[2], o[3]);
-                    }
-                }
-            }
-            if (t == 0) KDA_TRACE_EVENT(n, 25);
-            tc_fence_before();
-            named_bar(kBarSolve, 128);
-            if (t == 0) mbar_arrive(&bars[bApFree]);
-            if (t == 0) KDA_TRACE_EVENT(n, 5);
-
-            // phase 1: invert the four 16x16 diagonal blocks, one block per
-            // warp, one column per lane (lanes 0-15)
-            if (lane < 16) {
-                const int o = 16 * sw, j = lane;
-                float col[16];
-#pragma unroll
-                for (int aa = 0; aa < 16; ++aa) col[aa] = 0.f;
-#pragma unroll
-                for (int aa = 0; aa < 16; ++aa) {
-                    float acc = 0.f;
-#pragma unroll
-                    for (int m4 = 0; m4 < aa; m4 += 4) {
-                        const float4 l = *reinterpret_cast<const float4 *>(sL + (o + aa) * kLDL + o + m4);
-                        acc = fmaf(l.x, col[m4], acc);
-                        if (m4 + 1 < aa) acc = fmaf(l.y, col[m4 + 1], acc);
-                        if (m4 + 2 < aa) acc = fmaf(l.z, col[m4 + 2], acc);
-                        if (m4 + 3 < aa) acc = fmaf(l.w, col[m4 + 3], acc);
-                    }
-                    col[aa] = (aa == j) ? 1.f : -acc;
-                }
-#pragma unroll
-                for (int aa = 0; aa < 16; ++aa) sT[(o + aa) * kLDL + o + j] = col[aa];
-                if (t == 0) KDA_TRACE_EVENT(n, 26);
-            }
-            named_bar(kBarSolve, 128);
-            if (t == 0) KDA_TRACE_EVENT(n, 6);
-
-            // phase 2: 32x32 blocks: T21 = -T22 (L21 T11), one 16x8 tile per warp
-            {
-                const int pb = sw >> 1, nt = sw & 1;
-                const int R1 = 32 * pb + 16, C0 = 32 * pb;
-                float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int kk = 0; kk < 16; kk += 8) {
-                    const uint32_t af[4] = {
-                        tf32_bits(sL[(R1 + g) * kLDL + C0 + kk + tq]),
-                        tf32_bits(sL[(R1 + g + 8) * kLDL + C0 + kk + tq]),
-                        tf32_bits(sL[(R1 + g) * kLDL + C0 + kk + tq + 4]),
-                        tf32_bits(sL[(R1 + g + 8) * kLDL + C0 + kk + tq + 4])};
-                    const uint32_t bfr[2] = {tf32_bits(sT[(C0 + kk + tq) * kLDL + C0 + 8 * nt + g]),
-                                             tf32_bits(sT[(C0 + kk + tq + 4) * kLDL + C0 + 8 * nt + g])};
-                    mma_tf32_16x8x8(acc, af, bfr);
-                }
-                float *xw = sXw + sw * 16 * 9;
-                xw[g * 9 + 2 * tq] = acc[0];
-                xw[g * 9 + 2 * tq + 1] = acc[1];
-                xw[(g + 8) * 9 + 2 * tq] = acc[2];
-                xw[(g + 8) * 9 + 2 * tq + 1] = acc[3];
-                __syncwarp();
-                float d[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int kk = 0; kk < 16; kk += 8) {
-                    const uint32_t af[4] = {
-                        tf32_bits(sT[(R1 + g) * kLDL + R1 + kk + tq]),
-                        tf32_bits(sT[(R1 + g + 8) * kLDL + R1 + kk + tq]),
-                        tf32_bits(sT[(R1 + g) * kLDL + R1 + kk + tq + 4]),
-                        tf32_bits(sT[(R1 + g + 8) * kLDL + R1 + kk + tq + 4])};
-                    const uint32_t bfr[2] = {tf32_bits(xw[(kk + tq) * 9 + g]),
-                                             tf32_bits(xw[(kk + tq + 4) * 9 + g])};
-                    mma_tf32_16x8x8(d, af, bfr);
-                }
-                float *o = sT + R1 * kLDL + C0 + 8 * nt;
-                o[g * kLDL + 2 * tq] = -d[0];
-                o[g * kLDL + 2 * tq + 1] = -d[1];
-                o[(g + 8) * kLDL + 2 * tq] = -d[2];
-                o[(g + 8) * kLDL + 2 * tq + 1] = -d[3];
-            }
-            named_bar(kBarSolve, 128);
-            if (t == 0) KDA_TRACE_EVENT(n, 7);
-
-            // phase 3: 64x64: T_BA = -T_B (L_BA T_A); warp = (m tile, pair of n
-            // tiles).  Blocks above the diagonal blocks of T are zero.
-            {
-                const int mt = sw & 1, nb = 2 * (sw >> 1);
-                const int rr = 32 + 16 * mt;
-                float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-                for (int kk = 0; kk < 32; kk += 8) {
-                    const uint32_t af[4] = {tf32_bits(sL[(rr + g) * kLDL + kk + tq]),
-                                            tf32_bits(sL[(rr + g + 8) * kLDL + kk + tq]),
-                                            tf32_bits(sL[(rr + g) * kLDL + kk + tq + 4]),
-                                            tf32_bits(sL[(rr + g + 8) * kLDL + kk + tq + 4])};
-#pragma unroll
-                    for (int q = 0; q < 2; ++q) {
-                        const int c = 8 * (nb + q) + g;
-                        const uint32_t bfr[2] = {tf32_bits(sT[(kk + tq) * kLDL + c]),
-                                                 tf32_bits(sT[(kk + tq + 4) * kLDL + c])};
-                        mma_tf32_16x8x8(acc[q], af, bfr);
-                    }
-                }
-#pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    float *o = sX + (16 * mt) * 36 + 8 * (nb + q);
-                    o[g * 36 + 2 * tq] = acc[q][0];
-                    o[g * 36 + 2 * tq + 1] = acc[q][1];
-                    o[(g + 8) * 36 + 2 * tq] = acc[q][2];
-                    o[(g + 8) * 36 + 2 * tq + 1] = acc[q][3];
-                }
-                if (t == 0) KDA_TRACE_EVENT(n, 27);
-                named_bar(kBarSolve, 128);
-                float d[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-                for (int kk = 0; kk < 32; kk += 8) {
-                    const uint32_t af[4] = {tf32_bits(sT[(rr + g) * kLDL + 32 + kk + tq]),
-                                            tf32_bits(sT[(rr + g + 8) * kLDL + 32 + kk + tq]),
-                                            tf32_bits(sT[(rr + g) * kLDL + 32 + kk + tq + 4]),
-                                            tf32_bits(sT[(rr + g + 8) * kLDL + 32 + kk + tq + 4])};
-#pragma unroll
-                    for (int q = 0; q < 2; ++q) {
-                        const int cc = 8 * (nb + q);
-                        const uint32_t bfr[2] = {tf32_bits(sX[(kk + tq) * 36 + cc + g]),
-                                                 tf32_bits(sX[(kk + tq + 4) * 36 + cc + g])};
-                        mma_tf32_16x8x8(d[q], af, bfr);
-                    }
-                }
-#pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    float *o = sT + rr * kLDL + 8 * (nb + q);
-                    o[g * kLDL + 2 * tq] = -d[q][0];
-                    o[g * kLDL + 2 * tq + 1] = -d[q][1];
-                    o[(g + 8) * kLDL + 2 * tq] = -d[q][2];
-                    o[(g + 8) * kLDL + 2 * tq + 1] = -d[q][3];
-                }
-            }
-            named_bar(kBarSolve, 128);
-            if (t == 0) KDA_TRACE_EVENT(n, 8);
-
-            // Tb = T diag(b) -> bf16, rows 0..63 of the Tb|0|P tile
-            {
-                const int r = t >> 1, half = t & 1;
-                const float *Tr = sT + r * kLDL + 32 * half;
-                const float *bs = sB + s * 64 + 32 * half;
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const float4 t0v = *reinterpret_cast<const float4 *>(Tr + 8 * j);
-                    const float4 t1v = *reinterpret_cast<const float4 *>(Tr + 8 * j + 4);
-                    const float4 b0v = *reinterpret_cast<const float4 *>(bs + 8 * j);
-                    const float4 b1v = *reinterpret_cast<const float4 *>(bs + 8 * j + 4);
-                    sts128(tp + sw128_off(r, 4 * half + j), pack2(t0v.x * b0v.x, t0v.y * b0v.y),
-                           pack2(t0v.z * b0v.z, t0v.w * b0v.w), pack2(t1v.x * b1v.x, t1v.y * b1v.y),
-                           pack2(t1v.z * b1v.z, t1v.w * b1v.w));
-                }
-            }
-            if (t == 0) KDA_TRACE_EVENT(n, 28);
-            fence_proxy_async();
-            named_bar(kBarSolve, 128);
+            solve_chunk(sw, lane, tmem, Ly::kTmAP, sbase + Ly::kTP + s * 24576, sL, sT, sX, sXw,
+                        sB + s * 64, &bars[bApFree], kBarSolve);
             if (t == 0) mbar_arrive(&bars[bTbFull + s]);
             if (t == 0) KDA_TRACE_EVENT(n, 9);
 
@@ -625,29 +279,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 if (!wait_or_abort(&bars[bWaccFull], n & 1, abort_flag, p.status)) break;
                 tc_fence_after();
                 if (t == 0) KDA_TRACE_EVENT(n, 11);
-                const int r = 32 * sw + lane;
-                const uint32_t kq = sbase + Ly::kKQ + s * 32768;
-#pragma unroll
-                for (int blk = 0; blk < 4; ++blk) {
-                    uint32_t v[32];
-                    tmem_ld32(tmem_addr(tmem, 32 * sw, Ly::kTmW + 32 * blk), v);
-                    tmem_wait_ld();
-                    const int aa = blk >> 1;
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        uint32_t o[4];
-#pragma unroll
-                        for (int e2 = 0; e2 < 4; ++e2) {
-                            const int c = 8 * j + 2 * e2;
-                            o[e2] = pack2(-__uint_as_float(v[c]), -__uint_as_float(v[c + 1]));
-                        }
-                        const int chunk = 4 * (blk & 1) + j;
-                        sts128(kq + aa * 16384 + sw128_off(r, chunk), o[0], o[1], o[2], o[3]);
-                    }
-                }
-                fence_proxy_async();
-                tc_fence_before();
-                __syncwarp();
+                convert_w(sw, lane, tmem, Ly::kTmW, sbase + Ly::kKQ + s * 32768);
                 if (lane == 0) mbar_arrive(&bars[bWReady + s]);
                 if (t == 0) KDA_TRACE_EVENT(n, 12);
             }
@@ -886,49 +518,14 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     }
 }
 
-// ---------------------------------------------------------------- host side
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
-                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
-                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void *ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
-                cudaSuccess ||
-            q != cudaDriverEntryPointSuccess)
-            return nullptr;
-        fn = reinterpret_cast<EncodeTiledFn>(ptr);
-    }
-    return fn;
-}
-
-// [T, H, D] bf16 tensor; box = {bx channels, 1 head, 64 tokens}
-bool make_map(CUtensorMap *m, const void *base, int T, int H, int D, int bx,
-              CUtensorMapSwizzle swz) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T};
-    const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
-    const cuuint32_t box[3] = {(cuuint32_t)bx, 1, (cuuint32_t)kChunk};
-    const cuuint32_t estr[3] = {1, 1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
-              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int VS>
 cudaError_t launch_vs(const ForwardArgs &a, cudaStream_t s) {
     CUtensorMap mq, mk, mla, mv;
     const int T = a.T > 0 ? a.T : 1;
-    if (!make_map(&mq, a.q, T, a.H, kDK, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&mk, a.k, T, a.H, kDK, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&mla, a.log_alpha, T, a.H, kDK, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&mv, a.v, T, a.H, kDV, VS,
-                  VS == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B))
+    if (!make_tmap_bf16_3d(&mq, a.q, T, a.H, kDK, 64, 128) ||
+        !make_tmap_bf16_3d(&mk, a.k, T, a.H, kDK, 64, 128) ||
+        !make_tmap_bf16_3d(&mla, a.log_alpha, T, a.H, kDK, 64, 128) ||
+        !make_tmap_bf16_3d(&mv, a.v, T, a.H, kDV, VS, VS * 2))
         return cudaErrorInvalidValue;
     TcParams p;
     p.beta = static_cast<const __nv_bfloat16 *>(a.beta);
@@ -953,7 +550,8 @@ cudaError_t launch_vs(const ForwardArgs &a, cudaStream_t s) {
 }  // namespace
 
 bool prefill_tc_supported(const ForwardArgs &a) {
-    return a.io_dtype == KDA_BF16 && a.gate_dtype == KDA_BF16 && a.Dk == kDK && a.Dv == kDV;
+    return a.io_dtype == KDA_BF16 && a.gate_dtype == KDA_BF16 && a.Dk == tc::kDK &&
+           a.Dv == tc::kDV;
 }
 
 cudaError_t launch_prefill_tc(const ForwardArgs &a, cudaStream_t s) {

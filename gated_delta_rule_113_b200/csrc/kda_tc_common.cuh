@@ -1,0 +1,431 @@
+// kda_tc_common.cuh -- key-side building blocks shared by the tensor-core
+// prefill kernels: gate prep (Qg, Kg, Ki, Gam_L over one 64-token chunk),
+// the unit-lower-triangular inverse (Tb, masked P) and the -W operand.
+//
+// Tile layouts (shared memory, 128-byte swizzle, K-major rows of 64 channels):
+//   KQ stage  [katom 0..1][Kg/-W rows 0..63 | Qg rows 0..63]   2 x 16 KB
+//   KI stage  [katom 0..1][Ki rows 0..63]                       2 x 8 KB
+//   TP stage  Tb rows 0..63 | zero rows 64..127 | P rows 128..191 (24 KB)
+// and in TMEM: D_AP (lanes 0-63 = A, lanes 64-127 = P, 64 columns) and D_W
+// (lanes 0-63 = W, 128 columns).
+#pragma once
+
+#include "kda_internal.cuh"
+#include "sm100.cuh"
+
+namespace kda {
+namespace tc {
+
+using namespace sm100;
+
+constexpr int kDK = 128;           // key width handled by the tensor-core kernels
+constexpr int kDV = 128;           // value width handled by the tensor-core kernels
+constexpr int kLDL = 68;           // fp32 row stride of the solve scratch
+constexpr int kPrepThreads = 256;  // threads running prep_chunk
+constexpr int kSolveThreads = 128; // threads running solve_chunk (4 warps, lane quarters 0..3)
+constexpr float kLog2e = 1.4426950408889634f;
+
+// Bounded wait on an mbarrier phase.  Waiting threads stay suspended in
+// try_wait (no issue slots taken from working warps) and wake when the phase
+// completes; a wait that outlasts 2 s gives up, records KDA_ERR_TIMEOUT and
+// raises the CTA's abort flag so every role winds down.
+__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity,
+                                              volatile int *abort_flag, int32_t *status) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t start = globaltimer_ns();
+    for (;;) {
+        if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+        if (*abort_flag) return false;
+        if (globaltimer_ns() - start > 2000000000ull) break;
+    }
+    *abort_flag = 1;
+    set_status(status, KDA_ERR_TIMEOUT);
+    return false;
+}
+
+// 16-byte shared store / load helpers
+__device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                       uint32_t d) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+                 "r"(d)
+                 : "memory");
+}
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr)
+                 : "memory");
+    return v;
+}
+
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) { return pack_bf16(lo, hi); }
+
+// Byte offset of 16-byte chunk `chunk` of row `row` in a VS-wide MN-major tile.
+template <int VS>
+__device__ __forceinline__ uint32_t vs_off(uint32_t row, uint32_t chunk) {
+    return VS == 32 ? sw64_off(row, chunk) : sw128_off(row, chunk);
+}
+
+// B-operand descriptor of a VS-wide MN-major tile (rows = K) at K step 0;
+// step ks adds vs_step(ks) (start address field, in 16-byte units).
+template <int VS>
+__device__ __forceinline__ uint64_t vs_desc(uint32_t base, uint32_t rows) {
+    return VS == 32 ? smem_desc(base, rows * 64, 512, kSw64)
+                    : smem_desc(base, rows * 128, 1024, kSw128);
+}
+template <int VS>
+__device__ __forceinline__ uint64_t vs_step(int ks) {
+    return (uint64_t)(VS == 32 ? ks * 1024 : ks * 2048) >> 4;
+}
+// K-major 128B-swizzled operand with two 64-wide K atoms `atom` bytes apart
+__device__ __forceinline__ uint64_t kmaj_step(int ks, uint32_t atom) {
+    return (uint64_t)((ks >> 2) * atom + (ks & 3) * 32) >> 4;
+}
+
+// ---------------------------------------------------------------------------
+// Gate prep for one chunk, run by kPrepThreads threads (t = 0..255) that
+// synchronise on named barrier `bar_id`.  On entry the KQ stage holds raw k
+// (rows 0-63) and q (rows 64-127) and the KI stage raw log_alpha, as the TMA
+// left them.  On exit (after a proxy fence) they hold Kg, Qg and Ki; rows at
+// or past L are zero.  sGL_s receives Gam_L (128 channels), sB_s beta (64
+// rows, zero past L).  sGP / sSUF are [16][128] fp32 scratch.
+//
+// alpha = 2^(log_alpha log2 e) once per element; Gam_r is the running product
+// of alpha inside the chunk and 1/Gam_r = (1/Gam_L) prod_{j>r} alpha_j, so no
+// element needs a second exponential or a division.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void prep_chunk(int t, uint32_t kq_stage, uint32_t ki_stage,
+                                           float *sGP, float *sSUF, float *sGL_s, float *sB_s,
+                                           const __nv_bfloat16 *beta, int c0, int L, int H, int h,
+                                           uint32_t bar_id) {
+    const int cg = t & 15, rg = t >> 4;   // 8-channel group, 4-row group
+    const int a = cg >> 3, ch = cg & 7;
+    const uint32_t kq = kq_stage + a * 16384;
+    const uint32_t ki = ki_stage + a * 8192;
+    // pass 0: alpha; in-group prefix and suffix products
+    float pre[4][8], suf[4][8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int r = rg * 4 + i;
+        uint4 raw = lds128(ki + sw128_off(r, ch));
+        if (r >= L) raw = make_uint4(0, 0, 0, 0);  // past the end: alpha = 1
+        const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const float la = (e & 1) ? bf16hi(w4[e >> 1]) : bf16lo(w4[e >> 1]);
+            pre[i][e] = ex2_approx(la * kLog2e);   // alpha for now
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        float sx = 1.f;
+#pragma unroll
+        for (int i = 3; i >= 0; --i) {
+            suf[i][e] = sx;          // prod_{j > i} alpha_j (within the group)
+            sx *= pre[i][e];
+        }
+        float px = 1.f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            px *= pre[i][e];
+            pre[i][e] = px;          // prod_{j <= i} alpha_j
+        }
+    }
+    {
+        float *gpp = sGP + rg * 128 + cg * 8;
+        *reinterpret_cast<float4 *>(gpp) = make_float4(pre[3][0], pre[3][1], pre[3][2], pre[3][3]);
+        *reinterpret_cast<float4 *>(gpp + 4) = make_float4(pre[3][4], pre[3][5], pre[3][6], pre[3][7]);
+    }
+    named_bar(bar_id, kPrepThreads);
+    // scan over the 16 row groups, one thread per channel:
+    // sGP <- exclusive prefix, sSUF <- (1/Gam_L) exclusive suffix, sGL <- Gam_L
+    if (t < 128) {
+        float gv[16];
+#pragma unroll
+        for (int g = 0; g < 16; ++g) gv[g] = sGP[g * 128 + t];
+        float px = 1.f;
+#pragma unroll
+        for (int g = 0; g < 16; ++g) {
+            sGP[g * 128 + t] = px;
+            px *= gv[g];
+        }
+        sGL_s[t] = px;
+        float sx = rcp_approx(px);   // 1/Gam_L, once per channel
+#pragma unroll
+        for (int g = 15; g >= 0; --g) {
+            sSUF[g * 128 + t] = sx;
+            sx *= gv[g];
+        }
+    } else if (t < 128 + kChunk) {
+        const int r = t - 128;
+        sB_s[r] = r < L ? __bfloat162float(beta[(size_t)(c0 + r) * H + h]) : 0.f;
+    }
+    named_bar(bar_id, kPrepThreads);
+    // pass 1: Gam_r = pre_group * pre[i]; 1/Gam_r = (1/Gam_L) suf_group suf[i]
+    float ef[8], ci[8];
+    {
+        const float4 *pp = reinterpret_cast<const float4 *>(sGP + rg * 128 + cg * 8);
+        const float4 *sp = reinterpret_cast<const float4 *>(sSUF + rg * 128 + cg * 8);
+        const float4 p0 = pp[0], p1 = pp[1], q0 = sp[0], q1 = sp[1];
+        ef[0] = p0.x; ef[1] = p0.y; ef[2] = p0.z; ef[3] = p0.w;
+        ef[4] = p1.x; ef[5] = p1.y; ef[6] = p1.z; ef[7] = p1.w;
+        ci[0] = q0.x; ci[1] = q0.y; ci[2] = q0.z; ci[3] = q0.w;
+        ci[4] = q1.x; ci[5] = q1.y; ci[6] = q1.z; ci[7] = q1.w;
+    }
+    // the next chunk's pass 0 overwrites sGP: everyone must have read it
+    named_bar(bar_id, kPrepThreads);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int r = rg * 4 + i;
+        uint32_t gb[4], gib[4];
+#pragma unroll
+        for (int e2 = 0; e2 < 4; ++e2) {
+            gb[e2] = pack_bf16_alu(ef[2 * e2] * pre[i][2 * e2], ef[2 * e2 + 1] * pre[i][2 * e2 + 1]);
+            gib[e2] = pack_bf16_alu(ci[2 * e2] * suf[i][2 * e2], ci[2 * e2 + 1] * suf[i][2 * e2 + 1]);
+        }
+        if (r >= L) {  // rows past the end of the sequence are zero
+#pragma unroll
+            for (int e2 = 0; e2 < 4; ++e2) gb[e2] = gib[e2] = 0u;
+        }
+        const uint32_t ka = kq + sw128_off(r, ch), qa = ka + 8192;
+        const uint4 kr = lds128(ka), qr = lds128(qa);
+        sts128(ki + sw128_off(r, ch), mul_bf16x2(kr.x, gib[0]), mul_bf16x2(kr.y, gib[1]),
+               mul_bf16x2(kr.z, gib[2]), mul_bf16x2(kr.w, gib[3]));
+        sts128(ka, mul_bf16x2(kr.x, gb[0]), mul_bf16x2(kr.y, gb[1]), mul_bf16x2(kr.z, gb[2]),
+               mul_bf16x2(kr.w, gb[3]));
+        sts128(qa, mul_bf16x2(qr.x, gb[0]), mul_bf16x2(qr.y, gb[1]), mul_bf16x2(qr.z, gb[2]),
+               mul_bf16x2(qr.w, gb[3]));
+    }
+    fence_proxy_async();
+}
+
+// ---------------------------------------------------------------------------
+// Solve for one chunk, run by 4 warps (sw = 0..3 owns TMEM lanes 32 sw..) that
+// synchronise on named barrier `bar_id`.  Reads D_AP from TMEM (column
+// tm_ap), writes L = strict_lower(diag(b) A) to sL and the masked bf16 P into
+// TP rows 128..191, arrives once on `ap_free` when D_AP may be overwritten,
+// then builds T = (I + L)^{-1} (16x16 diagonal blocks by substitution, 32x32
+// and 64x64 merges with mma.sync tf32) and writes Tb = T diag(b) as bf16 into
+// TP rows 0..63.  Blocks of sT above the diagonal blocks must be zero on
+// entry (they are never written).  Ends with a proxy fence and a barrier.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void solve_chunk(int sw, int lane, uint32_t tmem, uint32_t tm_ap,
+                                            uint32_t tp, float *sL, float *sT, float *sX,
+                                            float *sXw, const float *sB_s, uint64_t *ap_free,
+                                            uint32_t bar_id) {
+    const int t = sw * 32 + lane;
+    const int g = lane >> 2, tq = lane & 3;
+    {
+        const int r = 32 * (sw & 1) + lane;  // row within A (sw<2) or P (sw>=2)
+        uint32_t v0[32], v1[32];
+        tmem_ld32(tmem_addr(tmem, 32 * sw, tm_ap), v0);
+        tmem_ld32(tmem_addr(tmem, 32 * sw, tm_ap + 32), v1);
+        tmem_wait_ld();
+        if (sw < 2) {
+            // L = strict_lower(diag(b) A)
+            const float br = sB_s[r];
+            float *Lr = sL + r * kLDL;
+#pragma unroll
+            for (int c = 0; c < 64; c += 4) {
+                const uint32_t *src = c < 32 ? &v0[c] : &v1[c - 32];
+                float4 w;
+                w.x = (c + 0 < r) ? br * __uint_as_float(src[0]) : 0.f;
+                w.y = (c + 1 < r) ? br * __uint_as_float(src[1]) : 0.f;
+                w.z = (c + 2 < r) ? br * __uint_as_float(src[2]) : 0.f;
+                w.w = (c + 3 < r) ? br * __uint_as_float(src[3]) : 0.f;
+                *reinterpret_cast<float4 *>(Lr + c) = w;
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                uint32_t o[4];
+#pragma unroll
+                for (int e2 = 0; e2 < 4; ++e2) {
+                    const int c = 8 * j + 2 * e2;
+                    const uint32_t *src = c < 32 ? &v0[c] : &v1[c - 32];
+                    const float x0 = (c <= r) ? __uint_as_float(src[0]) : 0.f;
+                    const float x1 = (c + 1 <= r) ? __uint_as_float(src[1]) : 0.f;
+                    o[e2] = pack2(x0, x1);
+                }
+                sts128(tp + 16384 + sw128_off(r, j), o[0], o[1], o[2], o[3]);
+            }
+        }
+    }
+    tc_fence_before();
+    named_bar(bar_id, kSolveThreads);
+    if (t == 0) mbar_arrive(ap_free);
+
+    // phase 1: invert the four 16x16 diagonal blocks, one block per warp, one
+    // column per lane (lanes 0-15)
+    if (lane < 16) {
+        const int o = 16 * sw, j = lane;
+        float col[16];
+#pragma unroll
+        for (int aa = 0; aa < 16; ++aa) col[aa] = 0.f;
+#pragma unroll
+        for (int aa = 0; aa < 16; ++aa) {
+            float acc = 0.f;
+#pragma unroll
+            for (int m4 = 0; m4 < aa; m4 += 4) {
+                const float4 l = *reinterpret_cast<const float4 *>(sL + (o + aa) * kLDL + o + m4);
+                acc = fmaf(l.x, col[m4], acc);
+                if (m4 + 1 < aa) acc = fmaf(l.y, col[m4 + 1], acc);
+                if (m4 + 2 < aa) acc = fmaf(l.z, col[m4 + 2], acc);
+                if (m4 + 3 < aa) acc = fmaf(l.w, col[m4 + 3], acc);
+            }
+            col[aa] = (aa == j) ? 1.f : -acc;
+        }
+#pragma unroll
+        for (int aa = 0; aa < 16; ++aa) sT[(o + aa) * kLDL + o + j] = col[aa];
+    }
+    named_bar(bar_id, kSolveThreads);
+
+    // phase 2: 32x32 blocks: T21 = -T22 (L21 T11), one 16x8 tile per warp
+    {
+        const int pb = sw >> 1, nt = sw & 1;
+        const int R1 = 32 * pb + 16, C0 = 32 * pb;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int kk = 0; kk < 16; kk += 8) {
+            const uint32_t af[4] = {tf32_bits(sL[(R1 + g) * kLDL + C0 + kk + tq]),
+                                    tf32_bits(sL[(R1 + g + 8) * kLDL + C0 + kk + tq]),
+                                    tf32_bits(sL[(R1 + g) * kLDL + C0 + kk + tq + 4]),
+                                    tf32_bits(sL[(R1 + g + 8) * kLDL + C0 + kk + tq + 4])};
+            const uint32_t bfr[2] = {tf32_bits(sT[(C0 + kk + tq) * kLDL + C0 + 8 * nt + g]),
+                                     tf32_bits(sT[(C0 + kk + tq + 4) * kLDL + C0 + 8 * nt + g])};
+            mma_tf32_16x8x8(acc, af, bfr);
+        }
+        float *xw = sXw + sw * 16 * 9;
+        xw[g * 9 + 2 * tq] = acc[0];
+        xw[g * 9 + 2 * tq + 1] = acc[1];
+        xw[(g + 8) * 9 + 2 * tq] = acc[2];
+        xw[(g + 8) * 9 + 2 * tq + 1] = acc[3];
+        __syncwarp();
+        float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int kk = 0; kk < 16; kk += 8) {
+            const uint32_t af[4] = {tf32_bits(sT[(R1 + g) * kLDL + R1 + kk + tq]),
+                                    tf32_bits(sT[(R1 + g + 8) * kLDL + R1 + kk + tq]),
+                                    tf32_bits(sT[(R1 + g) * kLDL + R1 + kk + tq + 4]),
+                                    tf32_bits(sT[(R1 + g + 8) * kLDL + R1 + kk + tq + 4])};
+            const uint32_t bfr[2] = {tf32_bits(xw[(kk + tq) * 9 + g]),
+                                     tf32_bits(xw[(kk + tq + 4) * 9 + g])};
+            mma_tf32_16x8x8(d, af, bfr);
+        }
+        float *o = sT + R1 * kLDL + C0 + 8 * nt;
+        o[g * kLDL + 2 * tq] = -d[0];
+        o[g * kLDL + 2 * tq + 1] = -d[1];
+        o[(g + 8) * kLDL + 2 * tq] = -d[2];
+        o[(g + 8) * kLDL + 2 * tq + 1] = -d[3];
+    }
+    named_bar(bar_id, kSolveThreads);
+
+    // phase 3: 64x64: T_BA = -T_B (L_BA T_A); warp = (m tile, pair of n tiles).
+    // Blocks above the diagonal blocks of T are zero.
+    {
+        const int mt = sw & 1, nb = 2 * (sw >> 1);
+        const int rr = 32 + 16 * mt;
+        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+        for (int kk = 0; kk < 32; kk += 8) {
+            const uint32_t af[4] = {tf32_bits(sL[(rr + g) * kLDL + kk + tq]),
+                                    tf32_bits(sL[(rr + g + 8) * kLDL + kk + tq]),
+                                    tf32_bits(sL[(rr + g) * kLDL + kk + tq + 4]),
+                                    tf32_bits(sL[(rr + g + 8) * kLDL + kk + tq + 4])};
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                const int c = 8 * (nb + q) + g;
+                const uint32_t bfr[2] = {tf32_bits(sT[(kk + tq) * kLDL + c]),
+                                         tf32_bits(sT[(kk + tq + 4) * kLDL + c])};
+                mma_tf32_16x8x8(acc[q], af, bfr);
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            float *o = sX + (16 * mt) * 36 + 8 * (nb + q);
+            o[g * 36 + 2 * tq] = acc[q][0];
+            o[g * 36 + 2 * tq + 1] = acc[q][1];
+            o[(g + 8) * 36 + 2 * tq] = acc[q][2];
+            o[(g + 8) * 36 + 2 * tq + 1] = acc[q][3];
+        }
+        named_bar(bar_id, kSolveThreads);
+        float d[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+        for (int kk = 0; kk < 32; kk += 8) {
+            const uint32_t af[4] = {tf32_bits(sT[(rr + g) * kLDL + 32 + kk + tq]),
+                                    tf32_bits(sT[(rr + g + 8) * kLDL + 32 + kk + tq]),
+                                    tf32_bits(sT[(rr + g) * kLDL + 32 + kk + tq + 4]),
+                                    tf32_bits(sT[(rr + g + 8) * kLDL + 32 + kk + tq + 4])};
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                const int cc = 8 * (nb + q);
+                const uint32_t bfr[2] = {tf32_bits(sX[(kk + tq) * 36 + cc + g]),
+                                         tf32_bits(sX[(kk + tq + 4) * 36 + cc + g])};
+                mma_tf32_16x8x8(d[q], af, bfr);
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            float *o = sT + rr * kLDL + 8 * (nb + q);
+            o[g * kLDL + 2 * tq] = -d[q][0];
+            o[g * kLDL + 2 * tq + 1] = -d[q][1];
+            o[(g + 8) * kLDL + 2 * tq] = -d[q][2];
+            o[(g + 8) * kLDL + 2 * tq + 1] = -d[q][3];
+        }
+    }
+    named_bar(bar_id, kSolveThreads);
+
+    // Tb = T diag(b) -> bf16, rows 0..63 of the Tb|0|P tile
+    {
+        const int r = t >> 1, half = t & 1;
+        const float *Tr = sT + r * kLDL + 32 * half;
+        const float *bs = sB_s + 32 * half;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float4 t0v = *reinterpret_cast<const float4 *>(Tr + 8 * j);
+            const float4 t1v = *reinterpret_cast<const float4 *>(Tr + 8 * j + 4);
+            const float4 b0v = *reinterpret_cast<const float4 *>(bs + 8 * j);
+            const float4 b1v = *reinterpret_cast<const float4 *>(bs + 8 * j + 4);
+            sts128(tp + sw128_off(r, 4 * half + j), pack2(t0v.x * b0v.x, t0v.y * b0v.y),
+                   pack2(t0v.z * b0v.z, t0v.w * b0v.w), pack2(t1v.x * b1v.x, t1v.y * b1v.y),
+                   pack2(t1v.z * b1v.z, t1v.w * b1v.w));
+        }
+    }
+    fence_proxy_async();
+    named_bar(bar_id, kSolveThreads);
+}
+
+// ---------------------------------------------------------------------------
+// W (TMEM column tm_w, lanes 0..63, fp32) -> -W as bf16 over the Kg rows of
+// the KQ stage.  Run by the two warps owning TMEM lanes 0..63 (sw = 0, 1).
+// Ends with the proxy and tcgen05 fences; the caller then arrives.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void convert_w(int sw, int lane, uint32_t tmem, uint32_t tm_w,
+                                          uint32_t kq_stage) {
+    const int r = 32 * sw + lane;
+#pragma unroll
+    for (int blk = 0; blk < 4; ++blk) {
+        uint32_t v[32];
+        tmem_ld32(tmem_addr(tmem, 32 * sw, tm_w + 32 * blk), v);
+        tmem_wait_ld();
+        const int aa = blk >> 1;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            uint32_t o[4];
+#pragma unroll
+            for (int e2 = 0; e2 < 4; ++e2) {
+                const int c = 8 * j + 2 * e2;
+                o[e2] = pack2(-__uint_as_float(v[c]), -__uint_as_float(v[c + 1]));
+            }
+            const int chunk = 4 * (blk & 1) + j;
+            sts128(kq_stage + aa * 16384 + sw128_off(r, chunk), o[0], o[1], o[2], o[3]);
+        }
+    }
+    fence_proxy_async();
+    tc_fence_before();
+    __syncwarp();
+}
+
+}  // namespace tc
+}  // namespace kda

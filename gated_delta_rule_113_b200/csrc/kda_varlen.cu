@@ -12,10 +12,43 @@ namespace kda {
 
 __global__ void __launch_bounds__(1024) varlen_index_kernel(const int32_t *__restrict__ cu, int N,
                                                             int T, int32_t *status,
-                                                            int32_t *order) {
+                                                            int32_t *order, int32_t *chunk_off) {
     __shared__ int32_t s_len[kSortMax];
+    __shared__ int32_t s_part[1024];
     __shared__ int s_bad;
     const int tid = threadIdx.x;
+    if (chunk_off) {
+        // chunk_off[n] = sum_{i<n} ceil(len_i / 64) (malformed sequences count
+        // as empty): each thread scans a contiguous segment, then the block
+        // scans the segment totals.
+        const int seg = (N + blockDim.x - 1) / blockDim.x;
+        const int lo = tid * seg, hi = min(N, lo + seg);
+        int sum = 0;
+        for (int i = lo; i < hi; ++i) {
+            const int a = cu[i], b = cu[i + 1];
+            if (a >= 0 && b >= a && b <= T) sum += (b - a + kChunk - 1) / kChunk;
+        }
+        s_part[tid] = sum;
+        __syncthreads();
+        if (tid == 0) {
+            int run = 0;
+            for (int i = 0; i < (int)blockDim.x; ++i) {
+                const int x = s_part[i];
+                s_part[i] = run;
+                run += x;
+            }
+        }
+        __syncthreads();
+        int run = s_part[tid];
+        for (int i = lo; i < hi; ++i) {
+            chunk_off[i] = run;
+            const int a = cu[i], b = cu[i + 1];
+            if (a >= 0 && b >= a && b <= T) run += (b - a + kChunk - 1) / kChunk;
+        }
+        if (hi == N && lo < hi) chunk_off[N] = run;
+        if (N == 0 && tid == 0) chunk_off[0] = 0;
+        __syncthreads();
+    }
     if (tid == 0) {
         s_bad = (cu[0] != 0 || cu[N] != T) ? 1 : 0;
     }
@@ -46,7 +79,8 @@ __global__ void __launch_bounds__(1024) varlen_index_kernel(const int32_t *__res
 }
 
 cudaError_t launch_varlen_index(const ForwardArgs &a, cudaStream_t s) {
-    varlen_index_kernel<<<1, 1024, 0, s>>>(a.cu_seqlens, a.N, a.T, a.status, a.order);
+    varlen_index_kernel<<<1, 1024, 0, s>>>(a.cu_seqlens, a.N, a.T, a.status, a.order,
+                                           a.chunk_off);
     return cudaGetLastError();
 }
 

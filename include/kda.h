@@ -78,12 +78,22 @@ typedef struct kda_params {
 /* Evaluate a bf16 problem with the fp32 CUDA-core prefill instead of the
  * tensor-core one (slower; for cross-checking the two kernels). */
 #define KDA_FLAG_FORCE_SIMT 1
+/* Use the single-kernel tensor-core prefill even when the workspace is large
+ * enough for the two-pass one (for cross-checking the two). */
+#define KDA_FLAG_FUSED_TC 2
 
 /*
- * kda_forward_workspace_size -- bytes of device workspace kda_forward needs
- * for this problem (a status word, the per-sequence work order).  Returns 0
- * when `p` is NULL or invalid.  The workspace must be 256-byte aligned; its
- * contents need no initialisation and are overwritten by every call.
+ * kda_forward_workspace_size -- bytes of device workspace for the fastest
+ * kda_forward path of this problem.  Returns 0 when `p` is NULL or invalid.
+ * The workspace must be 256-byte aligned; its contents need no
+ * initialisation and are overwritten by every call.
+ *
+ * Every path needs a status word and the per-sequence work order (256 bytes
+ * + 4 N, rounded up to 256).  For bf16 inputs with Dk = Dv = 128 the fastest
+ * path is a two-pass tensor-core prefill that also stores, per 64-token chunk
+ * and head, a 65 KB operand packet: about (total_tokens / 64 + N) * H * 65 KB
+ * (~1 KB per token and head).  Given less than that (but at least the
+ * minimum) kda_forward runs the single-kernel tensor-core prefill instead.
  */
 size_t kda_forward_workspace_size(const kda_params *p);
 
@@ -104,7 +114,8 @@ size_t kda_forward_workspace_size(const kda_params *p);
  *   cu_seqlens [N + 1]         int32, device; 0 = c_0 <= c_1 <= ... <= c_N = T_tot
  *   out        [T_tot, H, Dv]  io_dtype, written
  *   S_final    [N, H, Dk, Dv]  fp32, written, or NULL
- *   workspace  device scratch of ws_bytes >= kda_forward_workspace_size(p)
+ *   workspace  device scratch: ws_bytes >= kda_forward_workspace_size(p) for
+ *              the fastest path, at least the minimum described above
  *
  * Aliasing: out and S_final must not overlap any input.  S_final may be the
  * same buffer as S0 (in-place continuation of a chain); any other partial

@@ -17,8 +17,14 @@ from helpers import as_np, err, head_slice, rel_fro, to_dev, tol
 pytestmark = pytest.mark.gpu
 
 
-def _run(inp, force_simt=False, **kw):
+PATHS = ["two_pass", "fused_tc", "simt"]
+
+
+def _run(inp, force_simt=False, path=None, **kw):
     d = to_dev(inp)
+    if path is not None:
+        kw["fused_tc"] = path == "fused_tc"
+        force_simt = path == "simt"
     out, sf = kda.forward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["S0"],
                           d["cu_seqlens"], force_simt=force_simt, **kw)
     torch.cuda.synchronize()
@@ -50,20 +56,21 @@ def test_workload0_fp32_full():
     _check(inp, out, sf, torch.float32)
 
 
-@pytest.mark.parametrize("force_simt", [False, True])
-def test_bf16_ragged_multi_chunk(force_simt):
+@pytest.mark.parametrize("path", PATHS)
+def test_bf16_ragged_multi_chunk(path):
     w = WORKLOADS[1]
     inp = forward_inputs(w, lengths=[300, 201], H=4)
-    out, sf = _run(inp, force_simt=force_simt)
+    out, sf = _run(inp, path=path)
     _check(inp, out, sf, torch.bfloat16)
 
 
-@pytest.mark.parametrize("dtype_idx", [0, 1])
-def test_varlen_edge_lengths(dtype_idx):
+@pytest.mark.parametrize("dtype_idx,path", [(0, None), (1, "two_pass"), (1, "fused_tc"),
+                                            (1, "simt")])
+def test_varlen_edge_lengths(dtype_idx, path):
     w = WORKLOADS[dtype_idx]
     lens = [1, 63, 64, 65, 0, 130, 128, 2]
     inp = forward_inputs(w, lengths=lens, H=2, s0=True)
-    out, sf = _run(inp)
+    out, sf = _run(inp, path=path)
     _check(inp, out, sf, w.torch_dtype)
     # zero-length sequence: S_final == S0 exactly
     assert torch.equal(sf[4].cpu(), inp["S0"][4])
@@ -141,12 +148,33 @@ def test_value_channel_permutation():
     assert rel_fro(as_np(sf2), as_np(sf[..., perm.cuda()])) < 1e-3
 
 
-def test_deterministic_reruns():
+@pytest.mark.parametrize("path", ["two_pass", "fused_tc"])
+def test_deterministic_reruns(path):
     w = WORKLOADS[1]
     inp = forward_inputs(w, lengths=[257, 64], H=4)
-    a = _run(inp)
-    b = _run(inp)
+    a = _run(inp, path=path)
+    b = _run(inp, path=path)
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+def test_tensor_core_paths_agree():
+    """The two-pass and the single-kernel tensor-core prefills run the same
+    arithmetic on the same bf16 operands; their results agree closely."""
+    w = WORKLOADS[1]
+    inp = forward_inputs(w, lengths=[640, 129, 1], H=3)
+    a = _run(inp, path="two_pass")
+    b = _run(inp, path="fused_tc")
+    assert rel_fro(as_np(a[0]), as_np(b[0])) < 1e-3
+    assert rel_fro(as_np(a[1]), as_np(b[1])) < 1e-3
+
+
+def test_many_heads_spread_over_the_grid():
+    """More (chunk, head) items than SMs: the persistent key-side pass strides
+    items over its CTAs."""
+    w = WORKLOADS[1]
+    inp = forward_inputs(w, lengths=[1000, 777, 64], H=24)
+    out, sf = _run(inp)
+    _check(inp, out, sf, torch.bfloat16)
 
 
 def test_malformed_seqlens_reported_not_faulting():
@@ -161,6 +189,27 @@ def test_malformed_seqlens_reported_not_faulting():
     good = d["cu_seqlens"]
     kda.forward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["S0"], good, workspace=ws)
     assert kda.workspace_status(ws) == 0
+
+
+def test_overlapping_seqlens_stay_inside_the_workspace():
+    """Offsets that describe overlapping sequences need more chunks than the
+    workspace was sized for: the kernels must flag them and write nothing out
+    of bounds (the guard bytes after the workspace stay untouched)."""
+    w = WORKLOADS[1]
+    T, H = 256, 2
+    inp = forward_inputs(w, lengths=[T], H=H)
+    d = to_dev(inp)
+    cu = torch.tensor([0, T, 0, T, 0, T, 0, T, 0, T], dtype=torch.int32, device="cuda")
+    N = cu.numel() - 1
+    n_ws = kda.forward_workspace_size(N, T, H, 128, 128)
+    buf = torch.zeros(n_ws + (1 << 20), dtype=torch.uint8, device="cuda")
+    ws = buf[:n_ws]
+    out = torch.empty((T, H, 128), dtype=torch.bfloat16, device="cuda")
+    sf = torch.empty((N, H, 128, 128), dtype=torch.float32, device="cuda")
+    kda.forward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], None, cu, out=out,
+                S_final=sf, workspace=ws)
+    assert kda.workspace_status(ws) == 7
+    assert int(buf[n_ws:].count_nonzero()) == 0
 
 
 # ------------------------------------------------------------------- decode

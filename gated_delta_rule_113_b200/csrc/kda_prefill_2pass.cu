@@ -29,6 +29,28 @@ namespace {
 using namespace sm100;
 using namespace tc;
 
+// Optional per-chunk timeline of pass 2's CTA 0 (clock64 per pipeline event),
+// compiled in only with -DKDA_TRACE for profiling builds; a no-op otherwise.
+#ifdef KDA_TRACE
+__device__ unsigned long long g_kda_trace1[64 * 16];
+#define KDA_TRACE1(n, e)                                                          \
+    do {                                                                          \
+        if (blockIdx.x == 0 && (n) < 64) g_kda_trace1[(n) * 16 + (e)] = clock64(); \
+    } while (0)
+__device__ unsigned long long g_kda_trace2[64 * 16];
+#define KDA_TRACE2(n, e)                                                          \
+    do {                                                                          \
+        if (blockIdx.x == 0 && (n) < 64) g_kda_trace2[(n) * 16 + (e)] = clock64(); \
+    } while (0)
+#else
+#define KDA_TRACE1(n, e) \
+    do {                 \
+    } while (0)
+#define KDA_TRACE2(n, e) \
+    do {                 \
+    } while (0)
+#endif
+
 // packet layout (bytes)
 constexpr uint32_t kPkKQ = 0;
 constexpr uint32_t kPkKI = 32768;
@@ -59,19 +81,20 @@ __device__ __forceinline__ Item item_of(long long m, int H, const int32_t *chunk
 }
 
 // ============================================================ pass 1
-constexpr int kKsWarps = 14;   // 0-7 prep, 8-11 solve, 12 TMA + packet store, 13 MMA
+constexpr int kKsWarps = 15;   // 0-7 prep, 8-11 solve, 12 TMA loads, 13 MMA, 14 packet stores
 constexpr int kKsThreads = kKsWarps * 32;
-enum KsRole { kKsPrep0 = 0, kKsSolve0 = 8, kKsTma = 12, kKsMma = 13 };
+enum KsRole { kKsPrep0 = 0, kKsSolve0 = 8, kKsTma = 12, kKsMma = 13, kKsStore = 14 };
 enum KsBars {
-    kbRawFull = 0,   // [2]
-    kbKqFull = 2,    // [2] count 8
-    kbApFull = 4,
-    kbApFree = 5,
-    kbTbFull = 6,    // [2]
-    kbWaccFull = 8,
-    kbWReady = 9,    // [2] count 2
-    kbDrain = 11,
-    kbNum = 12
+    kbRawFull = 0,   // [2] TMA -> prep
+    kbKqFull = 2,    // [2] count 8: prep -> MMA, stores (Qg, Ki, Gam_L final)
+    kbApFull = 4,    // [2] MMA_AP -> solve
+    kbApFree = 6,    // [2] solve read D_AP[s] -> MMA
+    kbTbFull = 8,    // [2] solve -> MMA, stores (Tb, P final)
+    kbWaccFull = 10, // MMA_W -> solve
+    kbWReady = 11,   // [2] count 2: -W written -> MMA (D_W free), stores
+    kbStored = 13,   // [2] every store of a stage has read shared memory -> TMA
+    kbDrain = 15,
+    kbNum = 16
 };
 
 struct KsLayout {
@@ -80,9 +103,8 @@ struct KsLayout {
     static constexpr uint32_t kTP = kKI + 2 * 16384;        // 2 x 24 KB
     static constexpr uint32_t kL = kTP + 2 * 24576;
     static constexpr uint32_t kT = kL + 64 * kLDL * 4;
-    static constexpr uint32_t kX = kT + 64 * kLDL * 4;
-    static constexpr uint32_t kXw = kX + 32 * 36 * 4;
-    static constexpr uint32_t kGP = kXw + 4 * 16 * 9 * 4;
+    static constexpr uint32_t kXw = kT + 64 * kLDL * 4;     // fp32 4 x [16][17]
+    static constexpr uint32_t kGP = kXw + 4 * 16 * 17 * 4;
     static constexpr uint32_t kSUF = kGP + 16 * 128 * 4;
     static constexpr uint32_t kGL = kSUF + 16 * 128 * 4;    // [2][128]
     static constexpr uint32_t kB = kGL + 2 * 128 * 4;       // [2][64]
@@ -90,7 +112,8 @@ struct KsLayout {
     static constexpr uint32_t kMisc = kBar + 16 * 8;
     static constexpr uint32_t kAlloc = kMisc + 16 + 1024;
     static_assert(kAlloc <= 232448, "shared memory budget exceeded");
-    static constexpr uint32_t kTmAP = 0, kTmW = 64, kTmCols = 256;
+    static constexpr uint32_t kTmAP = 0;     // + s * 64 (two A/P accumulators)
+    static constexpr uint32_t kTmW = 128, kTmCols = 256;
 };
 
 struct KsParams {
@@ -115,7 +138,6 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + Ly::kMisc + 4);
     float *sL = reinterpret_cast<float *>(sm + Ly::kL);
     float *sT = reinterpret_cast<float *>(sm + Ly::kT);
-    float *sX = reinterpret_cast<float *>(sm + Ly::kX);
     float *sXw = reinterpret_cast<float *>(sm + Ly::kXw);
     float *sGP = reinterpret_cast<float *>(sm + Ly::kGP);
     float *sSUF = reinterpret_cast<float *>(sm + Ly::kSUF);
@@ -164,30 +186,14 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     const uint32_t tmem = *tmem_slot;
 
     if (warp == kKsTma) {
-        // ---------------------------------------- loads and packet stores
+        // ------------------------------------------------------ TMA loads
         if (lane == 0) {
-            auto store_packet = [&](int i) {
+            for (int i = 0; i < count; ++i) {
                 const int s = i & 1;
-                unsigned char *dst = p.packets + (size_t)(first + (long long)i * stride) * kPacketBytes;
-                bulk_store(dst + kPkKQ, sm + Ly::kKQ + s * 32768, 32768);
-                bulk_store(dst + kPkKI, sm + Ly::kKI + s * 16384, 16384);
-                bulk_store(dst + kPkTb, sm + Ly::kTP + s * 24576, 8192);
-                bulk_store(dst + kPkP, sm + Ly::kTP + s * 24576 + 16384, 8192);
-                bulk_store(dst + kPkGL, sGL + s * 128, 512);
-                bulk_commit();
-            };
-            bool ok = true;
-            for (int i = 0; i < count && ok; ++i) {
-                const int s = i & 1;
-                if (i >= 2) {
-                    // the packet of item i-2 leaves stage s before item i enters it
-                    if (!wait_or_abort(&bars[kbWReady + s], ((i - 2) >> 1) & 1, abort_flag, p.status)) {
-                        ok = false;
-                        break;
-                    }
-                    store_packet(i - 2);
-                    bulk_wait_read_all();
-                }
+                // the packet of item i-2 must have left stage s
+                if (i >= 2 && !wait_or_abort(&bars[kbStored + s], ((i - 2) >> 1) & 1, abort_flag,
+                                             p.status))
+                    break;
                 const Item it = item_of(first + (long long)i * stride, p.H, p.chunk_off, p.cu, p.N);
                 uint64_t *full = &bars[kbRawFull + s];
                 mbar_arrive_expect_tx(full, 6 * 8192);
@@ -197,18 +203,51 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                                 it.c0);
                     tma_load_3d(sm + Ly::kKI + s * 16384 + a * 8192, &tm_la, full, a * 64, it.h, it.c0);
                 }
-            }
-            if (ok) {
-                for (int i = max(0, count - 2); i < count; ++i) {
-                    if (!wait_or_abort(&bars[kbWReady + (i & 1)], (i >> 1) & 1, abort_flag, p.status))
-                        break;
-                    store_packet(i);
+                KDA_TRACE1(i, 0);
+                if (i + 2 < count) {   // warm L2 with the tiles this stage takes next
+                    const Item nx = item_of(first + (long long)(i + 2) * stride, p.H, p.chunk_off,
+                                            p.cu, p.N);
+                    for (int a = 0; a < 2; ++a) {
+                        tma_prefetch_3d(&tm_k, a * 64, nx.h, nx.c0);
+                        tma_prefetch_3d(&tm_q, a * 64, nx.h, nx.c0);
+                        tma_prefetch_3d(&tm_la, a * 64, nx.h, nx.c0);
+                    }
                 }
             }
-            bulk_wait_all();
             // armed loads must land before the CTA may exit
             for (int i = max(0, count - 2); i < count; ++i)
                 mbar_wait(&bars[kbRawFull + (i & 1)], (i >> 1) & 1);
+        }
+    } else if (warp == kKsStore) {
+        // ------------------------------------------------- packet stores
+        // Each part of a packet leaves as soon as it is final: Qg, Ki and
+        // Gam_L after the prep, Tb and P after the solve, -W last.
+        if (lane == 0) {
+            for (int i = 0; i < count; ++i) {
+                const int s = i & 1;
+                unsigned char *dst = p.packets + (size_t)(first + (long long)i * stride) * kPacketBytes;
+                unsigned char *kq = sm + Ly::kKQ + s * 32768;
+                unsigned char *tp = sm + Ly::kTP + s * 24576;
+                if (!wait_or_abort(&bars[kbKqFull + s], (i >> 1) & 1, abort_flag, p.status)) break;
+                bulk_store(dst + kPkKQ + 8192, kq + 8192, 8192);            // Qg, K atom 0
+                bulk_store(dst + kPkKQ + 16384 + 8192, kq + 16384 + 8192, 8192);  // Qg, atom 1
+                bulk_store(dst + kPkKI, sm + Ly::kKI + s * 16384, 16384);
+                bulk_store(dst + kPkGL, sGL + s * 128, 512);
+                bulk_commit();
+                if (!wait_or_abort(&bars[kbTbFull + s], (i >> 1) & 1, abort_flag, p.status)) break;
+                bulk_store(dst + kPkTb, tp, 8192);
+                bulk_store(dst + kPkP, tp + 16384, 8192);
+                bulk_commit();
+                if (!wait_or_abort(&bars[kbWReady + s], (i >> 1) & 1, abort_flag, p.status)) break;
+                bulk_store(dst + kPkKQ, kq, 8192);                           // -W, atom 0
+                bulk_store(dst + kPkKQ + 16384, kq + 16384, 8192);           // -W, atom 1
+                bulk_commit();
+                KDA_TRACE1(i, 9);
+                bulk_wait_read_all();
+                KDA_TRACE1(i, 10);
+                mbar_arrive(&bars[kbStored + s]);
+            }
+            bulk_wait_all();
         }
     } else if (warp >= kKsPrep0 && warp < kKsPrep0 + kPrepThreads / 32) {
         // ----------------------------------------------------------- prep
@@ -217,8 +256,10 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             const int s = i & 1;
             if (!wait_or_abort(&bars[kbRawFull + s], (i >> 1) & 1, abort_flag, p.status)) break;
             const Item it = item_of(first + (long long)i * stride, p.H, p.chunk_off, p.cu, p.N);
+            if (t == 0) KDA_TRACE1(i, 1);
             prep_chunk(t, sbase + Ly::kKQ + s * 32768, sbase + Ly::kKI + s * 16384, sGP, sSUF,
                        sGL + s * 128, sB + s * 64, p.beta, it.c0, it.L, p.H, it.h, 1);
+            if (t == 0) KDA_TRACE1(i, 2);
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[kbKqFull + s]);
         }
@@ -228,16 +269,20 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         const int t = tid - kKsSolve0 * 32;
         for (int i = 0; i < count; ++i) {
             const int s = i & 1;
-            if (!wait_or_abort(&bars[kbApFull], i & 1, abort_flag, p.status)) break;
+            if (!wait_or_abort(&bars[kbApFull + s], (i >> 1) & 1, abort_flag, p.status)) break;
             tc_fence_after();
-            solve_chunk(sw, lane, tmem, Ly::kTmAP, sbase + Ly::kTP + s * 24576, sL, sT, sX, sXw,
-                        sB + s * 64, &bars[kbApFree], 2);
+            if (t == 0) KDA_TRACE1(i, 4);
+            solve_chunk(sw, lane, tmem, Ly::kTmAP + s * 64, sbase + Ly::kTP + s * 24576, sL, sT,
+                        sXw, sB + s * 64, &bars[kbApFree + s], 2);
             if (t == 0) mbar_arrive(&bars[kbTbFull + s]);
+            if (t == 0) KDA_TRACE1(i, 5);
             if (sw < 2) {
                 if (!wait_or_abort(&bars[kbWaccFull], i & 1, abort_flag, p.status)) break;
                 tc_fence_after();
+                if (t == 0) KDA_TRACE1(i, 7);
                 convert_w(sw, lane, tmem, Ly::kTmW, sbase + Ly::kKQ + s * 32768);
                 if (lane == 0) mbar_arrive(&bars[kbWReady + s]);
+                if (t == 0) KDA_TRACE1(i, 8);
             }
         }
     } else if (warp == kKsMma) {
@@ -253,13 +298,16 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 const uint64_t d_tp = smem_desc(sbase + Ly::kTP + s * 24576, 16, 1024, kSw128);
                 const uint64_t d_kg = smem_desc(kq, 16384, 1024, kSw128);
                 if (!wait_or_abort(&bars[kbKqFull + s], (i >> 1) & 1, abort_flag, p.status)) break;
-                if (i >= 1 && !wait_or_abort(&bars[kbApFree], (i - 1) & 1, abort_flag, p.status)) break;
+                if (i >= 2 && !wait_or_abort(&bars[kbApFree + s], ((i - 2) >> 1) & 1, abort_flag,
+                                             p.status))
+                    break;
                 tc_fence_after();
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
-                    mma_bf16(tmem + Ly::kTmAP, d_kq + kmaj_step(ks, 16384), d_ki + kmaj_step(ks, 8192),
-                             kIdAP, ks > 0);
-                mma_commit(&bars[kbApFull]);
+                    mma_bf16(tmem + Ly::kTmAP + s * 64, d_kq + kmaj_step(ks, 16384),
+                             d_ki + kmaj_step(ks, 8192), kIdAP, ks > 0);
+                mma_commit(&bars[kbApFull + s]);
+                KDA_TRACE1(i, 3);
                 if (!wait_or_abort(&bars[kbTbFull + s], (i >> 1) & 1, abort_flag, p.status)) break;
                 if (i >= 1 && !wait_or_abort(&bars[kbWReady + ((i - 1) & 1)], ((i - 1) >> 1) & 1,
                                              abort_flag, p.status))
@@ -270,6 +318,7 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                     mma_bf16(tmem + Ly::kTmW, d_tp + ((uint64_t)(ks * 32) >> 4),
                              d_kg + ((uint64_t)(ks * 2048) >> 4), kIdW, ks > 0);
                 mma_commit(&bars[kbWaccFull]);
+                KDA_TRACE1(i, 6);
             }
             mma_commit(&bars[kbDrain]);
             mbar_wait(&bars[kbDrain], 0);
@@ -408,6 +457,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
                 bulk_load(st + Ly::kTP + 16384, src + kPkP, 8192, full);
                 bulk_load(st + Ly::kGL, src + kPkGL, 512, full);
                 tma_load_3d(st + Ly::kV, &tm_v, full, vs * VS, h, t0 + j * kChunk);
+                KDA_TRACE2(j, 0);
                 if (j + 2 < nchunks) bulk_prefetch_l2(packet(j + 2), kPkGL + 512);
             }
             for (int j = max(0, nchunks - 2); j < nchunks; ++j)
@@ -433,18 +483,22 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
                 if (j >= 2 && !wait_or_abort(&bars[cbD1Free + s], ((j - 2) >> 1) & 1, abort_flag,
                                              p.status))
                     break;
+                KDA_TRACE2(j, 1);
                 tc_fence_after();
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)   // D1 = Tb V (U0; zero in rows 64..127)
                     mma_bf16(d1, d_tp + ((uint64_t)(ks * 32) >> 4), d_v + vs_step<VS>(ks), kIdV,
                              ks > 0);
                 if (!wait_or_abort(&bars[cbSbFull], j & 1, abort_flag, p.status)) break;
+                KDA_TRACE2(j, 2);
                 tc_fence_after();
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)   // D1 += [-W; Qg] S
                     mma_bf16(d1, d_kq + kmaj_step(ks, 16384), d_sb + vs_step<VS>(ks), kIdV, 1);
                 mma_commit(&bars[cbUFull]);
+                KDA_TRACE2(j, 3);
                 if (!wait_or_abort(&bars[cbUbFull], j & 1, abort_flag, p.status)) break;
+                KDA_TRACE2(j, 4);
                 tc_fence_after();
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)   // dS = Ki^T U
@@ -456,6 +510,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
                     mma_bf16(d1, d_p + ((uint64_t)(ks * 32) >> 4), d_ub + vs_step<VS>(ks), kIdV, 1);
                 mma_commit(&bars[cbOFull + s]);
                 mma_commit(&bars[cbStageFree + s]);
+                KDA_TRACE2(j, 5);
             }
             mma_commit(&bars[cbDrain]);
             mbar_wait(&bars[cbDrain], 0);
@@ -503,6 +558,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
                 // S <- Diag(Gam_L) (S + dS) for chunk j-1
                 if (!wait_or_abort(&bars[cbDsFull], (j - 1) & 1, abort_flag, p.status)) { ok = false; break; }
                 tc_fence_after();
+                if (c == 0) KDA_TRACE2(j - 1, 6);
 #pragma unroll
                 for (int jj = 0; jj < VS; jj += 32) {
                     uint32_t v[32];
@@ -524,6 +580,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
             const int s = j & 1;
             if (!wait_or_abort(&bars[cbFull + s], (j >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
             gl_cur = reinterpret_cast<const float *>(sm + s * Ly::kStage + Ly::kGL)[c];
+            if (c == 0) KDA_TRACE2(j, 7);
             {
                 const uint32_t sb = sbase + Ly::kSB;
 #pragma unroll
@@ -537,11 +594,13 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[cbSbFull]);
+            if (c == 0) KDA_TRACE2(j, 8);
 
             if (wq < 2) {
                 // U rows: D1 lanes 0..63 -> bf16 operand
                 if (!wait_or_abort(&bars[cbUFull], j & 1, abort_flag, p.status)) { ok = false; break; }
                 tc_fence_after();
+                if (c == 0) KDA_TRACE2(j, 9);
                 const uint32_t ub = sbase + Ly::kUB;
 #pragma unroll
                 for (int jj = 0; jj < VS; jj += 32) {
@@ -561,6 +620,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars[cbUbFull]);
+                if (c == 0) KDA_TRACE2(j, 10);
             } else if (j > 0) {
                 const int m = j - 1;
                 if (!wait_or_abort(&bars[cbOFull + (m & 1)], (m >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
@@ -650,3 +710,12 @@ cudaError_t launch_prefill_two_pass(const ForwardArgs &a, cudaStream_t s) {
 }
 
 }  // namespace kda
+
+#ifdef KDA_TRACE
+extern "C" int kda_trace1_read(unsigned long long *host) {
+    return (int)cudaMemcpyFromSymbol(host, kda::g_kda_trace1, sizeof(kda::g_kda_trace1));
+}
+extern "C" int kda_trace2_read(unsigned long long *host) {
+    return (int)cudaMemcpyFromSymbol(host, kda::g_kda_trace2, sizeof(kda::g_kda_trace2));
+}
+#endif

@@ -205,14 +205,16 @@ __device__ __forceinline__ void prep_chunk(int t, uint32_t kq_stage, uint32_t ki
 // synchronise on named barrier `bar_id`.  Reads D_AP from TMEM (column
 // tm_ap), writes L = strict_lower(diag(b) A) to sL and the masked bf16 P into
 // TP rows 128..191, arrives once on `ap_free` when D_AP may be overwritten,
-// then builds T = (I + L)^{-1} (16x16 diagonal blocks by substitution, 32x32
-// and 64x64 merges with mma.sync tf32) and writes Tb = T diag(b) as bf16 into
-// TP rows 0..63.  Blocks of sT above the diagonal blocks must be zero on
-// entry (they are never written).  Ends with a proxy fence and a barrier.
+// then builds T = (I + L)^{-1} (16x16 diagonal blocks by substitution, then a
+// block forward substitution per 16-column block with mma.sync tf32) and
+// writes Tb = T diag(b) as bf16 into TP rows 0..63.  Blocks of sT above the
+// diagonal blocks must be zero on entry (they are never written).  sXw is
+// 4 x [16][17] fp32 warp-private scratch.  Ends with a proxy fence and a
+// barrier.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void solve_chunk(int sw, int lane, uint32_t tmem, uint32_t tm_ap,
-                                            uint32_t tp, float *sL, float *sT, float *sX,
-                                            float *sXw, const float *sB_s, uint64_t *ap_free,
+                                            uint32_t tp, float *sL, float *sT, float *sXw,
+                                            const float *sB_s, uint64_t *ap_free,
                                             uint32_t bar_id) {
     const int t = sw * 32 + lane;
     const int g = lane >> 2, tq = lane & 3;
@@ -281,115 +283,87 @@ __device__ __forceinline__ void solve_chunk(int sw, int lane, uint32_t tmem, uin
     }
     named_bar(bar_id, kSolveThreads);
 
-    // phase 2: 32x32 blocks: T21 = -T22 (L21 T11), one 16x8 tile per warp
+    // phase 2: block forward substitution, warp sw owning the 16 columns
+    // [16 sw, 16 sw + 16) of T.  Block rows above sw are zero, block row sw is
+    // D_sw, and for i > sw:  T_i = -D_i * sum_{sw <= j < i} L_ij T_j.  Each warp
+    // only reads L, the diagonal blocks and its own columns, so no barrier is
+    // needed until the whole Tb tile is written.  X goes through a warp-private
+    // [16][17] scratch to turn accumulator fragments into B fragments.
     {
-        const int pb = sw >> 1, nt = sw & 1;
-        const int R1 = 32 * pb + 16, C0 = 32 * pb;
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        float *xw = sXw + sw * 16 * 17;
+        const int c0 = 16 * sw;
+        for (int i = sw + 1; i < 4; ++i) {
+            float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+            for (int jb = sw; jb < i; ++jb) {
 #pragma unroll
-        for (int kk = 0; kk < 16; kk += 8) {
-            const uint32_t af[4] = {tf32_bits(sL[(R1 + g) * kLDL + C0 + kk + tq]),
-                                    tf32_bits(sL[(R1 + g + 8) * kLDL + C0 + kk + tq]),
-                                    tf32_bits(sL[(R1 + g) * kLDL + C0 + kk + tq + 4]),
-                                    tf32_bits(sL[(R1 + g + 8) * kLDL + C0 + kk + tq + 4])};
-            const uint32_t bfr[2] = {tf32_bits(sT[(C0 + kk + tq) * kLDL + C0 + 8 * nt + g]),
-                                     tf32_bits(sT[(C0 + kk + tq + 4) * kLDL + C0 + 8 * nt + g])};
-            mma_tf32_16x8x8(acc, af, bfr);
-        }
-        float *xw = sXw + sw * 16 * 9;
-        xw[g * 9 + 2 * tq] = acc[0];
-        xw[g * 9 + 2 * tq + 1] = acc[1];
-        xw[(g + 8) * 9 + 2 * tq] = acc[2];
-        xw[(g + 8) * 9 + 2 * tq + 1] = acc[3];
-        __syncwarp();
-        float d[4] = {0.f, 0.f, 0.f, 0.f};
+                for (int kk = 0; kk < 16; kk += 8) {
+                    const float *Lr = sL + (16 * i + g) * kLDL + 16 * jb + kk + tq;
+                    const uint32_t af[4] = {tf32_bits(Lr[0]), tf32_bits(Lr[8 * kLDL]),
+                                            tf32_bits(Lr[4]), tf32_bits(Lr[8 * kLDL + 4])};
 #pragma unroll
-        for (int kk = 0; kk < 16; kk += 8) {
-            const uint32_t af[4] = {tf32_bits(sT[(R1 + g) * kLDL + R1 + kk + tq]),
-                                    tf32_bits(sT[(R1 + g + 8) * kLDL + R1 + kk + tq]),
-                                    tf32_bits(sT[(R1 + g) * kLDL + R1 + kk + tq + 4]),
-                                    tf32_bits(sT[(R1 + g + 8) * kLDL + R1 + kk + tq + 4])};
-            const uint32_t bfr[2] = {tf32_bits(xw[(kk + tq) * 9 + g]),
-                                     tf32_bits(xw[(kk + tq + 4) * 9 + g])};
-            mma_tf32_16x8x8(d, af, bfr);
-        }
-        float *o = sT + R1 * kLDL + C0 + 8 * nt;
-        o[g * kLDL + 2 * tq] = -d[0];
-        o[g * kLDL + 2 * tq + 1] = -d[1];
-        o[(g + 8) * kLDL + 2 * tq] = -d[2];
-        o[(g + 8) * kLDL + 2 * tq + 1] = -d[3];
-    }
-    named_bar(bar_id, kSolveThreads);
-
-    // phase 3: 64x64: T_BA = -T_B (L_BA T_A); warp = (m tile, pair of n tiles).
-    // Blocks above the diagonal blocks of T are zero.
-    {
-        const int mt = sw & 1, nb = 2 * (sw >> 1);
-        const int rr = 32 + 16 * mt;
-        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-        for (int kk = 0; kk < 32; kk += 8) {
-            const uint32_t af[4] = {tf32_bits(sL[(rr + g) * kLDL + kk + tq]),
-                                    tf32_bits(sL[(rr + g + 8) * kLDL + kk + tq]),
-                                    tf32_bits(sL[(rr + g) * kLDL + kk + tq + 4]),
-                                    tf32_bits(sL[(rr + g + 8) * kLDL + kk + tq + 4])};
+                    for (int q = 0; q < 2; ++q) {
+                        const float *Tc = sT + (16 * jb + kk + tq) * kLDL + c0 + 8 * q + g;
+                        const uint32_t bfr[2] = {tf32_bits(Tc[0]), tf32_bits(Tc[4 * kLDL])};
+                        mma_tf32_16x8x8(acc[q], af, bfr);
+                    }
+                }
+            }
 #pragma unroll
             for (int q = 0; q < 2; ++q) {
-                const int c = 8 * (nb + q) + g;
-                const uint32_t bfr[2] = {tf32_bits(sT[(kk + tq) * kLDL + c]),
-                                         tf32_bits(sT[(kk + tq + 4) * kLDL + c])};
-                mma_tf32_16x8x8(acc[q], af, bfr);
+                xw[g * 17 + 8 * q + 2 * tq] = acc[q][0];
+                xw[g * 17 + 8 * q + 2 * tq + 1] = acc[q][1];
+                xw[(g + 8) * 17 + 8 * q + 2 * tq] = acc[q][2];
+                xw[(g + 8) * 17 + 8 * q + 2 * tq + 1] = acc[q][3];
             }
-        }
+            __syncwarp();
+            float d[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
-            float *o = sX + (16 * mt) * 36 + 8 * (nb + q);
-            o[g * 36 + 2 * tq] = acc[q][0];
-            o[g * 36 + 2 * tq + 1] = acc[q][1];
-            o[(g + 8) * 36 + 2 * tq] = acc[q][2];
-            o[(g + 8) * 36 + 2 * tq + 1] = acc[q][3];
-        }
-        named_bar(bar_id, kSolveThreads);
-        float d[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+            for (int kk = 0; kk < 16; kk += 8) {
+                const float *Dr = sT + (16 * i + g) * kLDL + 16 * i + kk + tq;
+                const uint32_t af[4] = {tf32_bits(Dr[0]), tf32_bits(Dr[8 * kLDL]),
+                                        tf32_bits(Dr[4]), tf32_bits(Dr[8 * kLDL + 4])};
 #pragma unroll
-        for (int kk = 0; kk < 32; kk += 8) {
-            const uint32_t af[4] = {tf32_bits(sT[(rr + g) * kLDL + 32 + kk + tq]),
-                                    tf32_bits(sT[(rr + g + 8) * kLDL + 32 + kk + tq]),
-                                    tf32_bits(sT[(rr + g) * kLDL + 32 + kk + tq + 4]),
-                                    tf32_bits(sT[(rr + g + 8) * kLDL + 32 + kk + tq + 4])};
+                for (int q = 0; q < 2; ++q) {
+                    const uint32_t bfr[2] = {tf32_bits(xw[(kk + tq) * 17 + 8 * q + g]),
+                                             tf32_bits(xw[(kk + tq + 4) * 17 + 8 * q + g])};
+                    mma_tf32_16x8x8(d[q], af, bfr);
+                }
+            }
 #pragma unroll
             for (int q = 0; q < 2; ++q) {
-                const int cc = 8 * (nb + q);
-                const uint32_t bfr[2] = {tf32_bits(sX[(kk + tq) * 36 + cc + g]),
-                                         tf32_bits(sX[(kk + tq + 4) * 36 + cc + g])};
-                mma_tf32_16x8x8(d[q], af, bfr);
+                float *o = sT + (16 * i) * kLDL + c0 + 8 * q;
+                o[g * kLDL + 2 * tq] = -d[q][0];
+                o[g * kLDL + 2 * tq + 1] = -d[q][1];
+                o[(g + 8) * kLDL + 2 * tq] = -d[q][2];
+                o[(g + 8) * kLDL + 2 * tq + 1] = -d[q][3];
             }
-        }
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-            float *o = sT + rr * kLDL + 8 * (nb + q);
-            o[g * kLDL + 2 * tq] = -d[q][0];
-            o[g * kLDL + 2 * tq + 1] = -d[q][1];
-            o[(g + 8) * kLDL + 2 * tq] = -d[q][2];
-            o[(g + 8) * kLDL + 2 * tq + 1] = -d[q][3];
+            __syncwarp();
         }
     }
-    named_bar(bar_id, kSolveThreads);
 
-    // Tb = T diag(b) -> bf16, rows 0..63 of the Tb|0|P tile
+    // Tb = T diag(b) -> bf16 into rows 0..63 of the Tb|0|P tile; warp sw
+    // writes its own 16 columns (two 16-byte chunks of every row)
     {
-        const int r = t >> 1, half = t & 1;
-        const float *Tr = sT + r * kLDL + 32 * half;
-        const float *bs = sB_s + 32 * half;
+        const int c0 = 16 * sw;
+        const float *bs = sB_s + c0;
+        const float4 b0 = *reinterpret_cast<const float4 *>(bs);
+        const float4 b1 = *reinterpret_cast<const float4 *>(bs + 4);
+        const float4 b2 = *reinterpret_cast<const float4 *>(bs + 8);
+        const float4 b3 = *reinterpret_cast<const float4 *>(bs + 12);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const float4 t0v = *reinterpret_cast<const float4 *>(Tr + 8 * j);
-            const float4 t1v = *reinterpret_cast<const float4 *>(Tr + 8 * j + 4);
-            const float4 b0v = *reinterpret_cast<const float4 *>(bs + 8 * j);
-            const float4 b1v = *reinterpret_cast<const float4 *>(bs + 8 * j + 4);
-            sts128(tp + sw128_off(r, 4 * half + j), pack2(t0v.x * b0v.x, t0v.y * b0v.y),
-                   pack2(t0v.z * b0v.z, t0v.w * b0v.w), pack2(t1v.x * b1v.x, t1v.y * b1v.y),
-                   pack2(t1v.z * b1v.z, t1v.w * b1v.w));
+        for (int rr = 0; rr < 2; ++rr) {
+            const int r = lane + 32 * rr;
+            const float *Tr = sT + r * kLDL + c0;
+            const float4 t0 = *reinterpret_cast<const float4 *>(Tr);
+            const float4 t1 = *reinterpret_cast<const float4 *>(Tr + 4);
+            const float4 t2 = *reinterpret_cast<const float4 *>(Tr + 8);
+            const float4 t3 = *reinterpret_cast<const float4 *>(Tr + 12);
+            sts128(tp + sw128_off(r, 2 * sw), pack2(t0.x * b0.x, t0.y * b0.y),
+                   pack2(t0.z * b0.z, t0.w * b0.w), pack2(t1.x * b1.x, t1.y * b1.y),
+                   pack2(t1.z * b1.z, t1.w * b1.w));
+            sts128(tp + sw128_off(r, 2 * sw + 1), pack2(t2.x * b2.x, t2.y * b2.y),
+                   pack2(t2.z * b2.z, t2.w * b2.w), pack2(t3.x * b3.x, t3.y * b3.y),
+                   pack2(t3.z * b3.z, t3.w * b3.w));
         }
     }
     fence_proxy_async();

@@ -30,14 +30,16 @@ __global__ void __launch_bounds__(1024) varlen_index_kernel(const int32_t *__res
         }
         s_part[tid] = sum;
         __syncthreads();
-        if (tid == 0) {
-            int run = 0;
-            for (int i = 0; i < (int)blockDim.x; ++i) {
-                const int x = s_part[i];
-                s_part[i] = run;
-                run += x;
-            }
+        // exclusive scan of the segment totals (Hillis-Steele, log2(1024) steps)
+        for (int off = 1; off < (int)blockDim.x; off <<= 1) {
+            const int x = tid >= off ? s_part[tid - off] : 0;
+            __syncthreads();
+            s_part[tid] += x;
+            __syncthreads();
         }
+        const int incl = s_part[tid];
+        __syncthreads();
+        s_part[tid] = incl - sum;
         __syncthreads();
         int run = s_part[tid];
         for (int i = lo; i < hi; ++i) {

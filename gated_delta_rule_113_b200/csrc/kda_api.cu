@@ -123,6 +123,7 @@ kda_status kda_forward(const void *q, const void *k, const void *v, const void *
     a.N = p->num_seqs; a.T = p->total_tokens; a.H = p->H; a.Dk = p->Dk; a.Dv = p->Dv;
     a.io_dtype = p->io_dtype; a.gate_dtype = p->gate_dtype;
     a.status = reinterpret_cast<int32_t *>(workspace);
+    a.work_ctr = a.status + 4;   // inside the 256-byte header
     a.order = reinterpret_cast<int32_t *>(static_cast<char *>(workspace) + kWsHeader);
     a.chunk_off = nullptr;
     a.packets = nullptr;

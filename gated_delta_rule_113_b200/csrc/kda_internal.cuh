@@ -24,6 +24,7 @@ struct ForwardArgs {
     int N, T, H, Dk, Dv;
     int io_dtype, gate_dtype;
     int32_t *status;   // device status word (workspace)
+    int32_t *work_ctr; // device item counter of the key-side pass (workspace header)
     int32_t *order;    // device work order [N] (workspace)
     int32_t *chunk_off;    // device [N+1] exclusive prefix of per-sequence chunk counts, or null
     unsigned char *packets;  // device per-(chunk, head) key-side operand packets, or null
@@ -47,7 +48,7 @@ cudaError_t launch_prefill_two_pass(const ForwardArgs &a, cudaStream_t s);
 
 // Two-pass tensor-core prefill: bytes of one key-side operand packet and the
 // number of packets a problem can need (one per 64-token chunk and head).
-constexpr size_t kPacketBytes = 66560;
+constexpr size_t kPacketBytes = 66048;
 inline size_t packet_slots_bound(int64_t T, int64_t N, int64_t H) {
     return (size_t)((T + kChunk - 1) / kChunk + N) * (size_t)H;
 }

@@ -42,7 +42,20 @@ __device__ unsigned long long g_kda_trace2[64 * 16];
     do {                                                                          \
         if (blockIdx.x == 0 && (n) < 64) g_kda_trace2[(n) * 16 + (e)] = clock64(); \
     } while (0)
+// per-CTA [globaltimer start, end, clock64 start, end] of both passes
+__device__ unsigned long long g_kda_span1[1024 * 4];
+__device__ unsigned long long g_kda_span2[1024 * 4];
+#define KDA_SPAN(buf, k)                                                                   \
+    do {                                                                                   \
+        if (threadIdx.x == 0 && blockIdx.x < 1024) {                                       \
+            buf[blockIdx.x * 4 + (k)] = globaltimer_ns();                                  \
+            buf[blockIdx.x * 4 + 2 + (k)] = clock64();                                     \
+        }                                                                                  \
+    } while (0)
 #else
+#define KDA_SPAN(buf, k) \
+    do {                 \
+    } while (0)
 #define KDA_TRACE1(n, e) \
     do {                 \
     } while (0)
@@ -51,22 +64,31 @@ __device__ unsigned long long g_kda_trace2[64 * 16];
     } while (0)
 #endif
 
-// packet layout (bytes)
+// Packet layout (bytes).  Every tile is the 128-byte-swizzled K-major image
+// the chain pass hands to the tensor cores as it lands:
+//   [-W; Qe]  two 16 KB atoms (channels 0-63, 64-127) of 128 rows: rows
+//             0-63 = -W = -Tb Kg, rows 64-127 = Qe = Qg - P W
+//   Ki        two 8 KB atoms of 64 rows
+//   [Tb; PT]  128 rows x 64 positions: Tb = T diag(b), PT = P Tb
+//   Gam_L     128 fp32 channel decays of the whole chunk
+// With these the chain computes U = Tb V - W S and O = Qe S + PT V, which
+// equals Qg S + P U: the intra-chunk output needs no product after U.
 constexpr uint32_t kPkKQ = 0;
 constexpr uint32_t kPkKI = 32768;
-constexpr uint32_t kPkTb = 49152;
-constexpr uint32_t kPkP = 57344;
+constexpr uint32_t kPkTP = 49152;
 constexpr uint32_t kPkGL = 65536;
 static_assert(kPkGL + 512 <= kPacketBytes, "packet layout");
 
 // Maps item index m (= global chunk g * H + head) to its chunk.
 struct Item {
     int h, c0, L;
+    int m;   // packet index m; negative: this CTA has no further item
 };
 __device__ __forceinline__ Item item_of(long long m, int H, const int32_t *chunk_off,
                                         const int32_t *cu, int N) {
     const int g = (int)(m / H);
     Item it;
+    it.m = (int)m;
     it.h = (int)(m % H);
     int lo = 0, hi = N;   // largest n with chunk_off[n] <= g
     while (hi - lo > 1) {
@@ -80,40 +102,110 @@ __device__ __forceinline__ Item item_of(long long m, int H, const int32_t *chunk
     return it;
 }
 
+// PT = P Tb from its M = 64 accumulator (row r in TMEM lane 32 (r / 16) +
+// r % 16) to bf16 rows 64..127 of the Tb|PT tile.  Run by the eight prep
+// warps: warp w reads lane quarter w % 4 and columns 32 (w / 4) .. + 31.
+__device__ __forceinline__ void convert_pt8(int w, int lane, uint32_t tmem, uint32_t tm_pt,
+                                            uint32_t tp) {
+    const int qt = w & 3, hh = w >> 2;
+    uint32_t v[32];
+    tmem_ld32(tmem_addr(tmem, 32 * qt, tm_pt + 32 * hh), v);
+    tmem_wait_ld();
+    if (lane < 16) {
+        const int r = 64 + 16 * qt + lane;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            sts128(tp + sw128_off(r, 4 * hh + j),
+                   pack2(__uint_as_float(v[8 * j]), __uint_as_float(v[8 * j + 1])),
+                   pack2(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3])),
+                   pack2(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5])),
+                   pack2(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7])));
+    }
+    fence_proxy_async();
+    tc_fence_before();
+    __syncwarp();
+}
+
+// [W; PW] (TMEM lanes 0..127) -> -W over the Kg rows and Qe = Qg - PW over
+// the Qg rows of the key-query tile, as bf16.  Run by the eight prep warps:
+// warp w owns rows 32 (w % 4) .. + 31 and the 64 channels of atom w / 4.
+__device__ __forceinline__ void convert_wqe8(int w, int lane, uint32_t tmem, uint32_t tm_w,
+                                             uint32_t kq_stage) {
+    const int qt = w & 3, hh = w >> 2;
+    const int r = 32 * qt + lane;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        uint32_t v[32];
+        tmem_ld32(tmem_addr(tmem, 32 * qt, tm_w + 64 * hh + 32 * half), v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t addr = kq_stage + hh * 16384 + sw128_off(r, 4 * half + j);
+            uint32_t o[4];
+            if (qt < 2) {
+#pragma unroll
+                for (int e2 = 0; e2 < 4; ++e2)
+                    o[e2] = pack2(-__uint_as_float(v[8 * j + 2 * e2]),
+                                  -__uint_as_float(v[8 * j + 2 * e2 + 1]));
+            } else {
+                const uint4 qv = lds128(addr);
+                const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
+#pragma unroll
+                for (int e2 = 0; e2 < 4; ++e2)
+                    o[e2] = pack2(bf16lo(qw[e2]) - __uint_as_float(v[8 * j + 2 * e2]),
+                                  bf16hi(qw[e2]) - __uint_as_float(v[8 * j + 2 * e2 + 1]));
+            }
+            sts128(addr, o[0], o[1], o[2], o[3]);
+        }
+    }
+    fence_proxy_async();
+    tc_fence_before();
+    __syncwarp();
+}
+
 // ============================================================ pass 1
 constexpr int kKsWarps = 15;   // 0-7 prep, 8-11 solve, 12 TMA loads, 13 MMA, 14 packet stores
 constexpr int kKsThreads = kKsWarps * 32;
 enum KsRole { kKsPrep0 = 0, kKsSolve0 = 8, kKsTma = 12, kKsMma = 13, kKsStore = 14 };
+constexpr int kKsStages = 3;   // ring depth of the raw/processed key-query tiles
 enum KsBars {
-    kbRawFull = 0,   // [2] TMA -> prep
-    kbKqFull = 2,    // [2] count 8: prep -> MMA, stores (Qg, Ki, Gam_L final)
-    kbApFull = 4,    // [2] MMA_AP -> solve
-    kbApFree = 6,    // [2] solve read D_AP[s] -> MMA
-    kbTbFull = 8,    // [2] solve -> MMA, stores (Tb, P final)
-    kbWaccFull = 10, // MMA_W -> solve
-    kbWReady = 11,   // [2] count 2: -W written -> MMA (D_W free), stores
-    kbStored = 13,   // [2] every store of a stage has read shared memory -> TMA
-    kbDrain = 15,
-    kbNum = 16
+    kbRawFull = 0,   // [3] TMA -> prep
+    kbKqFull = 3,    // [3] count 8: prep -> A/P issuer, stores (Ki, Gam_L final)
+    kbApFull = 6,    // [2] A/P product -> solve (two TMEM accumulators)
+    kbApFree = 8,    // [2] solve has read D_AP[s] -> A/P issuer
+    kbTbFull = 10,   // solve -> PT issuer (Tb and P final, D_AP read)
+    kbPtAcc = 11,    // PT = P Tb product -> prep warps
+    kbPtReady = 12,  // count 8: PT written as bf16 -> W issuer
+    kbTpFree = 13,   // the Tb|PT tile has been read -> Tb write of the next chunk
+    kbWaccFull = 14, // [W; PW] product -> prep warps
+    kbWReady = 15,   // count 8: -W and Qe written -> stores (and D_W free)
+    kbStored = 16,   // [3] every store of a stage has read shared memory -> TMA
+    kbKiFree = 19,   // [3] Ki and Gam_L have been read out of the stage
+    kbDrain = 22,    // [2] A/P issuer, PT/W issuer
+    kbNum = 24
 };
 
 struct KsLayout {
-    static constexpr uint32_t kKQ = 0;                      // 2 x 32 KB
-    static constexpr uint32_t kKI = kKQ + 2 * 32768;        // 2 x 16 KB
-    static constexpr uint32_t kTP = kKI + 2 * 16384;        // 2 x 24 KB
-    static constexpr uint32_t kL = kTP + 2 * 24576;
+    static constexpr uint32_t kKQ = 0;                              // 3 x 32 KB
+    static constexpr uint32_t kKI = kKQ + kKsStages * 32768;        // 3 x 16 KB
+    static constexpr uint32_t kTP = kKI + kKsStages * 16384;        // 16 KB: Tb | PT
+    static constexpr uint32_t kP = kTP + 16384;                       // 8 KB: P
+    static constexpr uint32_t kL = kP + 8192;
     static constexpr uint32_t kT = kL + 64 * kLDL * 4;
     static constexpr uint32_t kXw = kT + 64 * kLDL * 4;     // fp32 4 x [16][17]
     static constexpr uint32_t kGP = kXw + 4 * 16 * 17 * 4;
     static constexpr uint32_t kSUF = kGP + 16 * 128 * 4;
-    static constexpr uint32_t kGL = kSUF + 16 * 128 * 4;    // [2][128]
-    static constexpr uint32_t kB = kGL + 2 * 128 * 4;       // [2][64]
-    static constexpr uint32_t kBar = kB + 2 * 64 * 4;
-    static constexpr uint32_t kMisc = kBar + 16 * 8;
-    static constexpr uint32_t kAlloc = kMisc + 16 + 1024;
+    static constexpr uint32_t kGL = kSUF + 16 * 128 * 4;    // [3][128]
+    static constexpr uint32_t kB = kGL + kKsStages * 128 * 4;       // [3][64]
+    static constexpr uint32_t kBar = kB + kKsStages * 64 * 4;
+    static constexpr uint32_t kMisc = kBar + 24 * 8;
+    static constexpr uint32_t kItem = kMisc + 16;   // [3] Item of the tile in each stage
+    static constexpr uint32_t kAlloc = kItem + kKsStages * sizeof(Item) + 1024;
     static_assert(kAlloc <= 232448, "shared memory budget exceeded");
-    static constexpr uint32_t kTmAP = 0;     // + s * 64 (two A/P accumulators)
-    static constexpr uint32_t kTmW = 128, kTmCols = 256;
+    static constexpr uint32_t kTmAP = 0;     // + (i & 1) * 64 (two A/P accumulators)
+    static constexpr uint32_t kTmW = 128;    // [W; PW], 128 columns
+    static constexpr uint32_t kTmPT = 256;   // PT (M = 64: 16 lanes per quarter), 64 columns
+    static constexpr uint32_t kTmCols = 512;
 };
 
 struct KsParams {
@@ -123,6 +215,7 @@ struct KsParams {
     unsigned char *packets;
     long long slots;          // packets the workspace holds
     int32_t *status;
+    int32_t *work_ctr;        // items past the first wave are claimed from here
     int N, H;
 };
 
@@ -150,15 +243,17 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         if (blockIdx.x == 0 && threadIdx.x == 0) set_status(p.status, KDA_ERR_SEQLENS);
         total = p.slots;
     }
-    const long long first = blockIdx.x, stride = gridDim.x;
-    const int count = first < total ? (int)((total - first + stride - 1) / stride) : 0;
-    if (count == 0) return;
+    // Each CTA starts on item blockIdx.x and claims further items from a
+    // counter as its loader frees a stage, so CTAs that run faster (SMs vary
+    // by several percent here) take more of the work.
+    if ((long long)blockIdx.x >= total) return;
+    Item *items = reinterpret_cast<Item *>(sm + Ly::kItem);
 
     if (tid == 0) {
         for (int i = 0; i < kbNum; ++i) {
             uint32_t cnt = 1;
-            if (i == kbKqFull || i == kbKqFull + 1) cnt = kPrepThreads / 32;
-            if (i == kbWReady || i == kbWReady + 1) cnt = 2;
+            if (i >= kbKqFull && i < kbKqFull + kKsStages) cnt = kPrepThreads / 32;
+            if (i == kbWReady || i == kbPtReady) cnt = kPrepThreads / 32;
             mbar_init(&bars[i], cnt);
         }
         *abort_flag = 0;
@@ -168,10 +263,6 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_k);
         prefetch_tmap(&tm_la);
-    }
-    for (int i = tid; i < 2 * 512; i += kKsThreads) {   // zero rows of both Tb|0|P tiles
-        const int s = i / 512, j = i % 512;
-        sts128(sbase + Ly::kTP + s * 24576 + 8192 + j * 16, 0, 0, 0, 0);
     }
     for (int i = tid; i < 64 * kLDL / 4; i += kKsThreads)  // T stays zero above its blocks
         sts128(sbase + Ly::kT + i * 16, 0, 0, 0, 0);
@@ -184,147 +275,287 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    KDA_SPAN(g_kda_span1, 0);
 
     if (warp == kKsTma) {
         // ------------------------------------------------------ TMA loads
-        if (lane == 0) {
-            for (int i = 0; i < count; ++i) {
-                const int s = i & 1;
-                // the packet of item i-2 must have left stage s
-                if (i >= 2 && !wait_or_abort(&bars[kbStored + s], ((i - 2) >> 1) & 1, abort_flag,
-                                             p.status))
-                    break;
-                const Item it = item_of(first + (long long)i * stride, p.H, p.chunk_off, p.cu, p.N);
-                uint64_t *full = &bars[kbRawFull + s];
-                mbar_arrive_expect_tx(full, 6 * 8192);
-                for (int a = 0; a < 2; ++a) {
-                    tma_load_3d(sm + Ly::kKQ + s * 32768 + a * 16384, &tm_k, full, a * 64, it.h, it.c0);
-                    tma_load_3d(sm + Ly::kKQ + s * 32768 + a * 16384 + 8192, &tm_q, full, a * 64, it.h,
-                                it.c0);
-                    tma_load_3d(sm + Ly::kKI + s * 16384 + a * 8192, &tm_la, full, a * 64, it.h, it.c0);
-                }
-                KDA_TRACE1(i, 0);
-                if (i + 2 < count) {   // warm L2 with the tiles this stage takes next
-                    const Item nx = item_of(first + (long long)(i + 2) * stride, p.H, p.chunk_off,
-                                            p.cu, p.N);
-                    for (int a = 0; a < 2; ++a) {
-                        tma_prefetch_3d(&tm_k, a * 64, nx.h, nx.c0);
-                        tma_prefetch_3d(&tm_q, a * 64, nx.h, nx.c0);
-                        tma_prefetch_3d(&tm_la, a * 64, nx.h, nx.c0);
-                    }
-                }
+        // Copies issued by one thread are serviced one after another, so each
+        // of the six tiles of a stage is issued by its own lane.
+        static_assert(kKsStages == 3, "the look-ahead below keeps three items");
+        // Items are claimed three ahead of their load so their tiles can be
+        // warmed in L2; lane 0 claims and looks the coordinates up (global
+        // memory) and broadcasts them.
+        bool claimed_out = false;
+        auto claim = [&](bool first_item) -> Item {
+            Item it;
+            it.h = it.c0 = it.L = 0;
+            it.m = -1;
+            if (lane == 0 && !claimed_out) {
+                const long long m = first_item ? (long long)blockIdx.x
+                                               : (long long)gridDim.x + atomicAdd(p.work_ctr, 1);
+                if (m < total) it = item_of(m, p.H, p.chunk_off, p.cu, p.N);
             }
-            // armed loads must land before the CTA may exit
-            for (int i = max(0, count - 2); i < count; ++i)
-                mbar_wait(&bars[kbRawFull + (i & 1)], (i >> 1) & 1);
+            it.h = __shfl_sync(0xffffffffu, it.h, 0);
+            it.c0 = __shfl_sync(0xffffffffu, it.c0, 0);
+            it.L = __shfl_sync(0xffffffffu, it.L, 0);
+            it.m = __shfl_sync(0xffffffffu, it.m, 0);
+            if (it.m < 0) claimed_out = true;
+            return it;
+        };
+        const int a = lane & 1, which = lane >> 1;   // lanes 0-5: atom a of k, q or log_alpha
+        const CUtensorMap *tm = which == 0 ? &tm_k : which == 1 ? &tm_q : &tm_la;
+        auto warm = [&](const Item &it) {   // L2 prefetch of an item's tiles
+            if (it.m >= 0 && lane < 6) tma_prefetch_3d(tm, a * 64, it.h, it.c0);
+        };
+        Item nx0 = claim(true);
+        Item nx1 = claim(false);
+        warm(nx1);
+        Item nx2 = claim(false);
+        warm(nx2);
+        int n_loaded = 0;
+        bool ended = false;
+        for (int i = 0;; ++i) {
+            const int s = i % kKsStages;
+            const Item it = nx0;
+            nx0 = nx1;
+            nx1 = nx2;
+            // the packet of item i-3 must have left stage s
+            bool ok = true;
+            if (lane == 0 && i >= kKsStages)
+                ok = wait_or_abort(&bars[kbStored + s], ((i / kKsStages) - 1) & 1, abort_flag, p.status);
+            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+            uint64_t *full = &bars[kbRawFull + s];
+            if (it.m < 0) {   // no more items: tell the prep, which tells the rest
+                if (lane == 0) {
+                    items[s] = it;
+                    mbar_arrive(full);
+                }
+                ended = true;
+                break;
+            }
+            if (lane == 0) {
+                items[s] = it;
+                mbar_arrive_expect_tx(full, 6 * 8192);
+            }
+            __syncwarp();
+            if (lane < 6) {
+                const uint32_t dst = which < 2 ? Ly::kKQ + s * 32768 + a * 16384 + which * 8192
+                                               : Ly::kKI + s * 16384 + a * 8192;
+                tma_load_3d(sm + dst, tm, full, a * 64, it.h, it.c0);
+            }
+            if (lane == 0) KDA_TRACE1(i, 0);
+            n_loaded = i + 1;
+            nx2 = claim(false);
+            warm(nx2);
         }
+        // Armed loads must land before the CTA may exit.  The end marker went
+        // to the stage of item n_loaded - 3, whose load the Stored wait above
+        // already saw consumed (and whose phase the marker has moved past).
+        if (lane == 0)
+            for (int i = max(0, n_loaded - kKsStages + (ended ? 1 : 0)); i < n_loaded; ++i)
+                mbar_wait(&bars[kbRawFull + i % kKsStages], (i / kKsStages) & 1);
     } else if (warp == kKsStore) {
         // ------------------------------------------------- packet stores
-        // Each part of a packet leaves as soon as it is final: Qg, Ki and
-        // Gam_L after the prep, Tb and P after the solve, -W last.
-        if (lane == 0) {
-            for (int i = 0; i < count; ++i) {
-                const int s = i & 1;
-                unsigned char *dst = p.packets + (size_t)(first + (long long)i * stride) * kPacketBytes;
-                unsigned char *kq = sm + Ly::kKQ + s * 32768;
-                unsigned char *tp = sm + Ly::kTP + s * 24576;
-                if (!wait_or_abort(&bars[kbKqFull + s], (i >> 1) & 1, abort_flag, p.status)) break;
-                bulk_store(dst + kPkKQ + 8192, kq + 8192, 8192);            // Qg, K atom 0
-                bulk_store(dst + kPkKQ + 16384 + 8192, kq + 16384 + 8192, 8192);  // Qg, atom 1
-                bulk_store(dst + kPkKI, sm + Ly::kKI + s * 16384, 16384);
-                bulk_store(dst + kPkGL, sGL + s * 128, 512);
-                bulk_commit();
-                if (!wait_or_abort(&bars[kbTbFull + s], (i >> 1) & 1, abort_flag, p.status)) break;
-                bulk_store(dst + kPkTb, tp, 8192);
-                bulk_store(dst + kPkP, tp + 16384, 8192);
-                bulk_commit();
-                if (!wait_or_abort(&bars[kbWReady + s], (i >> 1) & 1, abort_flag, p.status)) break;
-                bulk_store(dst + kPkKQ, kq, 8192);                           // -W, atom 0
-                bulk_store(dst + kPkKQ + 16384, kq + 16384, 8192);           // -W, atom 1
-                bulk_commit();
-                KDA_TRACE1(i, 9);
-                bulk_wait_read_all();
-                KDA_TRACE1(i, 10);
-                mbar_arrive(&bars[kbStored + s]);
-            }
-            bulk_wait_all();
-        }
-    } else if (warp >= kKsPrep0 && warp < kKsPrep0 + kPrepThreads / 32) {
-        // ----------------------------------------------------------- prep
-        const int t = tid - kKsPrep0 * 32;
-        for (int i = 0; i < count; ++i) {
-            const int s = i & 1;
-            if (!wait_or_abort(&bars[kbRawFull + s], (i >> 1) & 1, abort_flag, p.status)) break;
-            const Item it = item_of(first + (long long)i * stride, p.H, p.chunk_off, p.cu, p.N);
-            if (t == 0) KDA_TRACE1(i, 1);
-            prep_chunk(t, sbase + Ly::kKQ + s * 32768, sbase + Ly::kKI + s * 16384, sGP, sSUF,
-                       sGL + s * 128, sB + s * 64, p.beta, it.c0, it.L, p.H, it.h, 1);
-            if (t == 0) KDA_TRACE1(i, 2);
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[kbKqFull + s]);
-        }
-    } else if (warp >= kKsSolve0 && warp < kKsSolve0 + 4) {
-        // ---------------------------------------------------------- solve
-        const int sw = warp - kKsSolve0;
-        const int t = tid - kKsSolve0 * 32;
-        for (int i = 0; i < count; ++i) {
-            const int s = i & 1;
-            if (!wait_or_abort(&bars[kbApFull + s], (i >> 1) & 1, abort_flag, p.status)) break;
-            tc_fence_after();
-            if (t == 0) KDA_TRACE1(i, 4);
-            solve_chunk(sw, lane, tmem, Ly::kTmAP + s * 64, sbase + Ly::kTP + s * 24576, sL, sT,
-                        sXw, sB + s * 64, &bars[kbApFree + s], 2);
-            if (t == 0) mbar_arrive(&bars[kbTbFull + s]);
-            if (t == 0) KDA_TRACE1(i, 5);
-            if (sw < 2) {
-                if (!wait_or_abort(&bars[kbWaccFull], i & 1, abort_flag, p.status)) break;
+        // Lane 0 waits and issues the products that follow the solve; the
+        // copies are spread over lanes, each lane tracking its own groups.
+        for (int i = 0;; ++i) {
+            const int s = i % kKsStages;
+            unsigned char *kq = sm + Ly::kKQ + s * 32768;
+            unsigned char *tp = sm + Ly::kTP;
+            bool ok = true;
+            // The products after the solve are issued here rather than by the
+            // A/P issuer, so the next chunk's A/P product never queues behind
+            // this chunk's solve.  D_PT and D_W are free: this lane already
+            // waited for the previous chunk's conversions out of them.
+            if (lane == 0) ok = wait_or_abort(&bars[kbTbFull], i & 1, abort_flag, p.status);
+            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+            const int m = items[s].m;
+            if (m < 0) break;
+            unsigned char *dst = p.packets + (size_t)m * kPacketBytes;
+            if (lane == 0) {   // PT = P Tb  (M = 64, B = Tb read MN-major)
                 tc_fence_after();
-                if (t == 0) KDA_TRACE1(i, 7);
-                convert_w(sw, lane, tmem, Ly::kTmW, sbase + Ly::kKQ + s * 32768);
-                if (lane == 0) mbar_arrive(&bars[kbWReady + s]);
-                if (t == 0) KDA_TRACE1(i, 8);
-            }
-        }
-    } else if (warp == kKsMma) {
-        // ------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t kIdAP = idesc_bf16(128, 64, 0, 0);
-            constexpr uint32_t kIdW = idesc_bf16(128, 128, 0, 1);
-            for (int i = 0; i < count; ++i) {
-                const int s = i & 1;
-                const uint32_t kq = sbase + Ly::kKQ + s * 32768;
-                const uint64_t d_kq = smem_desc(kq, 16, 1024, kSw128);
-                const uint64_t d_ki = smem_desc(sbase + Ly::kKI + s * 16384, 16, 1024, kSw128);
-                const uint64_t d_tp = smem_desc(sbase + Ly::kTP + s * 24576, 16, 1024, kSw128);
-                const uint64_t d_kg = smem_desc(kq, 16384, 1024, kSw128);
-                if (!wait_or_abort(&bars[kbKqFull + s], (i >> 1) & 1, abort_flag, p.status)) break;
-                if (i >= 2 && !wait_or_abort(&bars[kbApFree + s], ((i - 2) >> 1) & 1, abort_flag,
-                                             p.status))
-                    break;
-                tc_fence_after();
+                constexpr uint32_t kIdPT = idesc_bf16(64, 64, 0, 1);
+                const uint64_t d_p = smem_desc(sbase + Ly::kP, 16, 1024, kSw128);
+                const uint64_t d_tb = smem_desc(sbase + Ly::kTP, 8192, 1024, kSw128);
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks)
-                    mma_bf16(tmem + Ly::kTmAP + s * 64, d_kq + kmaj_step(ks, 16384),
-                             d_ki + kmaj_step(ks, 8192), kIdAP, ks > 0);
-                mma_commit(&bars[kbApFull + s]);
-                KDA_TRACE1(i, 3);
-                if (!wait_or_abort(&bars[kbTbFull + s], (i >> 1) & 1, abort_flag, p.status)) break;
-                if (i >= 1 && !wait_or_abort(&bars[kbWReady + ((i - 1) & 1)], ((i - 1) >> 1) & 1,
-                                             abort_flag, p.status))
-                    break;
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16(tmem + Ly::kTmPT, d_p + ((uint64_t)(ks * 32) >> 4),
+                             d_tb + ((uint64_t)(ks * 2048) >> 4), kIdPT, ks > 0);
+                mma_commit(&bars[kbPtAcc]);
+                ok = wait_or_abort(&bars[kbPtReady], i & 1, abort_flag, p.status);
+            }
+            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+            if (lane == 0) {   // [W; PW] = [Tb; PT] Kg
                 tc_fence_after();
+                constexpr uint32_t kIdW = idesc_bf16(128, 128, 0, 1);
+                const uint64_t d_tp = smem_desc(sbase + Ly::kTP, 16, 1024, kSw128);
+                const uint64_t d_kg = smem_desc(smem_u32(kq), 16384, 1024, kSw128);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
                     mma_bf16(tmem + Ly::kTmW, d_tp + ((uint64_t)(ks * 32) >> 4),
                              d_kg + ((uint64_t)(ks * 2048) >> 4), kIdW, ks > 0);
                 mma_commit(&bars[kbWaccFull]);
                 KDA_TRACE1(i, 6);
+                bulk_store(dst + kPkTP, tp, 16384);
+                bulk_commit();
+                bulk_wait_read_all();
+                mma_commit(&bars[kbTpFree]);   // after both products have read the tile
+                ok = wait_or_abort(&bars[kbWReady], i & 1, abort_flag, p.status);
             }
+            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+            if (lane < 2) {   // [-W; Qe], one 16 KB atom per lane
+                bulk_store(dst + kPkKQ + lane * 16384, kq + lane * 16384, 16384);
+                bulk_commit();
+            }
+            if (lane == 0) KDA_TRACE1(i, 9);
+            bulk_wait_read_all();
+            // Ki and Gam_L leave from the A/P warp; their reads finished too
+            if (lane == 0)
+                ok = wait_or_abort(&bars[kbKiFree + s], (i / kKsStages) & 1, abort_flag, p.status);
+            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+            if (lane == 0) {
+                KDA_TRACE1(i, 10);
+                mbar_arrive(&bars[kbStored + s]);
+            }
+        }
+        if (lane == 0) {
+            mma_commit(&bars[kbDrain + 1]);   // every product of this lane done before TMEM is freed
+            mbar_wait(&bars[kbDrain + 1], 0);
+        }
+        bulk_wait_all();
+    } else if (warp >= kKsPrep0 && warp < kKsPrep0 + kPrepThreads / 32) {
+        // ----------------------------------------------------------- prep
+        const int t = tid - kKsPrep0 * 32;
+        // After preparing chunk i these warps turn chunk i-1's PT and [W; PW]
+        // products into bf16 operands, so the solve warps only solve.
+        auto convert = [&](int m) -> bool {
+            const int sm3 = m % kKsStages;
+            if (!wait_or_abort(&bars[kbPtAcc], m & 1, abort_flag, p.status)) return false;
+            tc_fence_after();
+            convert_pt8(warp, lane, tmem, Ly::kTmPT, sbase + Ly::kTP);
+            if (lane == 0) mbar_arrive(&bars[kbPtReady]);
+            if (!wait_or_abort(&bars[kbWaccFull], m & 1, abort_flag, p.status)) return false;
+            tc_fence_after();
+            if (t == 0) KDA_TRACE1(m, 7);
+            convert_wqe8(warp, lane, tmem, Ly::kTmW, sbase + Ly::kKQ + sm3 * 32768);
+            if (lane == 0) mbar_arrive(&bars[kbWReady]);
+            if (t == 0) KDA_TRACE1(m, 8);
+            return true;
+        };
+        bool ok = true;
+        int n_items = 0;
+        for (int i = 0;; ++i) {
+            const int s = i % kKsStages;
+            if (!wait_or_abort(&bars[kbRawFull + s], (i / kKsStages) & 1, abort_flag, p.status)) {
+                ok = false;
+                break;
+            }
+            const Item it = items[s];
+            if (it.m < 0) {   // pass the end on
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars[kbKqFull + s]);
+                break;
+            }
+            if (t == 0) KDA_TRACE1(i, 1);
+            prep_chunk(t, sbase + Ly::kKQ + s * 32768, sbase + Ly::kKI + s * 16384, sGP, sSUF,
+                       sGL + s * 128, sB + s * 64, p.beta, it.c0, it.L, p.H, it.h, 1);
+            if (t == 0) KDA_TRACE1(i, 2);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[kbKqFull + s]);
+            n_items = i + 1;
+            if (i >= 1 && !convert(i - 1)) {
+                ok = false;
+                break;
+            }
+        }
+        if (ok && n_items > 0) convert(n_items - 1);
+    } else if (warp >= kKsSolve0 && warp < kKsSolve0 + 4) {
+        // ---------------------------------------------------------- solve
+        const int sw = warp - kKsSolve0;
+        const int t = tid - kKsSolve0 * 32;
+        for (int i = 0;; ++i) {
+            const int s = i % kKsStages, a = i & 1;
+            if (!wait_or_abort(&bars[kbApFull + a], (i >> 1) & 1, abort_flag, p.status)) break;
+            if (items[s].m < 0) {   // pass the end on, after the store warp has taken
+                                    // TbFull's previous phase (TpFree follows it)
+                if (t == 0 && (i < 1 || wait_or_abort(&bars[kbTpFree], (i - 1) & 1, abort_flag,
+                                                      p.status)))
+                    mbar_arrive(&bars[kbTbFull]);
+                break;
+            }
+            tc_fence_after();
+            if (t == 0) KDA_TRACE1(i, 4);
+            solve_chunk<false>(sw, lane, tmem, Ly::kTmAP + a * 64, sbase + Ly::kP, sL, sT, sXw,
+                               sB + s * 64, nullptr, 2);
+            // P leaves TMEM only now: the previous chunk's PT product must be
+            // done with the P tile, which by this time it long is
+            if (i >= 1 && sw >= 2 && !wait_or_abort(&bars[kbPtAcc], (i - 1) & 1, abort_flag, p.status))
+                break;
+            write_p(sw, lane, tmem, Ly::kTmAP + a * 64, sbase + Ly::kP);
+            tc_fence_before();
+            // the previous chunk's Tb|PT tile must have been read
+            if (i >= 1 && !wait_or_abort(&bars[kbTpFree], (i - 1) & 1, abort_flag, p.status)) break;
+            write_tb(sw, lane, sbase + Ly::kTP, sT, sB + s * 64, 2);
+            if (t == 0) {
+                mbar_arrive(&bars[kbApFree + a]);
+                mbar_arrive(&bars[kbTbFull]);
+            }
+            if (t == 0) KDA_TRACE1(i, 5);
+        }
+    } else if (warp == kKsMma) {
+        // --------------------------------- A/P issuer (lane 0), Ki stores (lane 1)
+        // Ki and Gam_L are final once the prep is done.  They leave from here,
+        // not from the store warp, which works a chunk behind: the solve writes
+        // P over Ki and must not wait for the previous chunk's stores.
+        constexpr uint32_t kIdAP = idesc_bf16(128, 64, 0, 0);
+        for (int i = 0;; ++i) {
+            const int s = i % kKsStages, a = i & 1;
+            bool ok = true;
+            if (lane == 0)
+                ok = wait_or_abort(&bars[kbKqFull + s], (i / kKsStages) & 1, abort_flag, p.status);
+            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+            const int m = items[s].m;
+            if (m < 0) {   // pass the end on, after the same wait a product takes,
+                           // so the solve has consumed ApFull[a]'s previous phase
+                if (lane == 0 && (i < 2 || wait_or_abort(&bars[kbApFree + a], ((i - 2) >> 1) & 1,
+                                                         abort_flag, p.status)))
+                    mbar_arrive(&bars[kbApFull + a]);
+                break;
+            }
+            if (lane == 1) {
+                unsigned char *dst = p.packets + (size_t)m * kPacketBytes;
+                bulk_store(dst + kPkKI, sm + Ly::kKI + s * 16384, 16384);
+                bulk_store(dst + kPkGL, sGL + s * 128, 512);
+                bulk_commit();
+                bulk_wait_read_all();
+                mbar_arrive(&bars[kbKiFree + s]);
+            }
+            if (lane == 0) {
+                const uint32_t kq = sbase + Ly::kKQ + s * 32768;
+                const uint64_t d_kq = smem_desc(kq, 16, 1024, kSw128);
+                const uint64_t d_ki = smem_desc(sbase + Ly::kKI + s * 16384, 16, 1024, kSw128);
+                if (i >= 2)
+                    ok = wait_or_abort(&bars[kbApFree + a], ((i - 2) >> 1) & 1, abort_flag, p.status);
+                if (ok) {
+                    tc_fence_after();
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks)
+                        mma_bf16(tmem + Ly::kTmAP + a * 64, d_kq + kmaj_step(ks, 16384),
+                                 d_ki + kmaj_step(ks, 8192), kIdAP, ks > 0);
+                    mma_commit(&bars[kbApFull + a]);
+                    KDA_TRACE1(i, 3);
+                }
+            }
+            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+        }
+        if (lane == 0) {
             mma_commit(&bars[kbDrain]);
             mbar_wait(&bars[kbDrain], 0);
         }
+        bulk_wait_all();
     }
 
+    KDA_SPAN(g_kda_span1, 1);
     tc_fence_before();
     __syncthreads();
     if (warp == kKsMma) {
@@ -336,32 +567,35 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 // ============================================================ pass 2
 constexpr int kChWarps = 6;   // 0-3 chain, 4 loader, 5 MMA
 constexpr int kChThreads = kChWarps * 32;
+constexpr int kChStages = 3;
 enum ChRole { kChLoad = 4, kChMma = 5 };
 enum ChBars {
-    cbFull = 0,       // [2] packet + value tile landed
-    cbStageFree = 2,  // [2] every MMA of a stage done
-    cbSbFull = 4,     // count 4
-    cbUFull = 5,
-    cbUbFull = 6,     // count 2
-    cbDsFull = 7,
-    cbOFull = 8,      // [2]
-    cbD1Free = 10,    // [2] count 2
+    cbFull = 0,       // [3] packet + value tile landed
+    cbStageFree = 3,  // [3] every product reading a stage done
+    cbSbFull = 6,     // count 4: bf16 S written
+    cbUFull = 7,      // D1 = [U; O] complete
+    cbUbFull = 8,     // count 2: bf16 U written
+    cbDsFull = 9,     // dS = Ki^T U complete
+    cbD1Free = 10,    // [2] count 2: O read out of D1[d]
     cbDrain = 12,
     cbNum = 13
 };
 
 template <int VS>
 struct ChLayout {
-    static constexpr uint32_t kKQ = 0, kKI = 32768, kTP = 49152, kV = 73728;
-    static constexpr uint32_t kGL = kV + 64 * VS * 2;     // 512 B
-    static constexpr uint32_t kStage = (kGL + 512 + 1023) / 1024 * 1024;  // KQ | KI | TP | V | GL
-    static constexpr uint32_t kSB = 2 * kStage;
+    // stage: the packet exactly as stored ([-W; Qe] | Ki | [Tb; PT] | Gam_L),
+    // so one bulk copy fills it, then the V slice
+    static constexpr uint32_t kKQ = kPkKQ, kKI = kPkKI, kTP = kPkTP, kGL = kPkGL;
+    static constexpr uint32_t kV = (kPkGL + 512 + 1023) / 1024 * 1024;
+    static constexpr uint32_t kStage = (kV + 64 * VS * 2 + 1023) / 1024 * 1024;
+    static_assert(kPkGL + 512 == kPacketBytes, "the packet is one contiguous copy");
+    static constexpr uint32_t kSB = kChStages * kStage;
     static constexpr uint32_t kUB = kSB + 128 * VS * 2;
     static constexpr uint32_t kBar = kUB + 64 * VS * 2;
     static constexpr uint32_t kMisc = kBar + 16 * 8;
     static constexpr uint32_t kAlloc = kMisc + 16 + 1024;
     static_assert(kAlloc <= 232448, "shared memory budget exceeded");
-    static constexpr uint32_t kTmD1 = 0;          // + s * VS
+    static constexpr uint32_t kTmD1 = 0;          // + d * VS, d = chunk & 1
     static constexpr uint32_t kTmD2 = 2 * VS;
     static constexpr uint32_t kTmCols = 128;
 };
@@ -379,6 +613,15 @@ struct ChParams {
     int N, T, H;
 };
 
+// One CTA per (sequence, head, VS-wide slice of the value dimension) walks
+// the sequence's chunks in order.  Per chunk, with S the bf16 copy of the
+// fp32 state slice kept in the chain warps' registers:
+//   D1  = [Tb; PT] V          (rows 0-63: U0 = Tb V, rows 64-127: P U0)
+//   D1 += [-W; Qe] S          (rows 0-63: U,  rows 64-127: O)
+//   dS  = Ki^T bf16(U)
+//   S   = Diag(Gam_L) (S + dS)
+// Only the last two steps and the product of the bf16 S with [-W; Qe] lie on
+// the chain from one chunk's state to the next.
 template <int VS>
 __global__ void __launch_bounds__(kChThreads, 1)
 chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
@@ -413,27 +656,22 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
         for (int i = 0; i < cbNum; ++i) {
             uint32_t cnt = 1;
             if (i == cbSbFull) cnt = 4;
-            if (i == cbUbFull) cnt = 2;
-            if (i == cbD1Free || i == cbD1Free + 1) cnt = 2;
+            if (i == cbUbFull || i == cbD1Free || i == cbD1Free + 1) cnt = 2;
             mbar_init(&bars[i], cnt);
         }
         *abort_flag = 0;
         fence_mbar_init();
     }
     if (warp == kChLoad && lane == 0) prefetch_tmap(&tm_v);
-    for (int i = tid; i < 2 * 512; i += kChThreads) {   // zero rows of both Tb|0|P tiles
-        const int s = i / 512, j = i % 512;
-        sts128(sbase + s * Ly::kStage + Ly::kTP + 8192 + j * 16, 0, 0, 0, 0);
-    }
     if (warp == kChMma) {
         tmem_alloc(tmem_slot, Ly::kTmCols);
         tmem_relinquish();
     }
-    fence_proxy_async();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    KDA_SPAN(g_kda_span2, 0);
 
     auto packet = [&](int j) {
         return p.packets + ((size_t)(g0 + j) * p.H + h) * kPacketBytes;
@@ -441,28 +679,37 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
 
     if (warp == kChLoad) {
         // ------------------------------------------------------- loader
-        if (lane == 0) {
-            for (int j = 0; j < nchunks; ++j) {
-                const int s = j & 1;
-                if (j >= 2 && !wait_or_abort(&bars[cbStageFree + s], ((j - 2) >> 1) & 1, abort_flag,
-                                             p.status))
-                    break;
-                unsigned char *st = sm + s * Ly::kStage;
-                const unsigned char *src = packet(j);
-                uint64_t *full = &bars[cbFull + s];
-                mbar_arrive_expect_tx(full, 65536 + 512 + 64 * VS * 2);
-                bulk_load(st + Ly::kKQ, src + kPkKQ, 32768, full);
-                bulk_load(st + Ly::kKI, src + kPkKI, 16384, full);
-                bulk_load(st + Ly::kTP, src + kPkTb, 8192, full);
-                bulk_load(st + Ly::kTP + 16384, src + kPkP, 8192, full);
-                bulk_load(st + Ly::kGL, src + kPkGL, 512, full);
-                tma_load_3d(st + Ly::kV, &tm_v, full, vs * VS, h, t0 + j * kChunk);
-                KDA_TRACE2(j, 0);
-                if (j + 2 < nchunks) bulk_prefetch_l2(packet(j + 2), kPkGL + 512);
+        // One copy for the packet (lane 0) and one for the value tile (lane
+        // 1): copies from different threads are serviced concurrently.
+        for (int j = 0; j < nchunks; ++j) {
+            const int s = j % kChStages;
+            bool ok = true;
+            if (lane == 0 && j >= kChStages)
+                ok = wait_or_abort(&bars[cbStageFree + s], (j / kChStages - 1) & 1, abort_flag, p.status);
+            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+            unsigned char *st = sm + s * Ly::kStage;
+            uint64_t *full = &bars[cbFull + s];
+            if (lane == 0) mbar_arrive_expect_tx(full, (uint32_t)kPacketBytes + 64 * VS * 2);
+            __syncwarp();
+            if (lane < 4) {   // the packet in four pieces, one per lane
+                const uint32_t off = lane * 16384u;
+                const uint32_t len = lane < 3 ? 16384u : (uint32_t)kPacketBytes - 3 * 16384u;
+                bulk_load(st + off, packet(j) + off, len, full);
             }
-            for (int j = max(0, nchunks - 2); j < nchunks; ++j)
-                mbar_wait(&bars[cbFull + (j & 1)], (j >> 1) & 1);
+            if (lane == 4) tma_load_3d(st + Ly::kV, &tm_v, full, vs * VS, h, t0 + j * kChunk);
+            if (lane == 5 && j + kChStages < nchunks)
+                bulk_prefetch_l2(packet(j + kChStages), (uint32_t)kPacketBytes);
+            if (lane == 0) KDA_TRACE2(j, 0);
+#ifdef KDA_TRACE
+            if (lane == 6) {
+                mbar_wait(full, (j / kChStages) & 1);
+                KDA_TRACE2(j, 11);
+            }
+#endif
         }
+        if (lane == 0)
+            for (int j = max(0, nchunks - kChStages); j < nchunks; ++j)
+                mbar_wait(&bars[cbFull + j % kChStages], (j / kChStages) & 1);
     } else if (warp == kChMma) {
         // ------------------------------------------------------ MMA issuer
         if (lane == 0) {
@@ -470,34 +717,45 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
             constexpr uint32_t kIdS = idesc_bf16(128, VS, 1, 1);
             const uint64_t d_sb = vs_desc<VS>(sbase + Ly::kSB, 128);
             const uint64_t d_ub = vs_desc<VS>(sbase + Ly::kUB, 64);
-            for (int j = 0; j < nchunks; ++j) {
-                const int s = j & 1;
+            // D1[d] = [Tb; PT] V for chunk j: issued one chunk ahead, while the
+            // chain warps turn the previous chunk's U into bf16, so it never
+            // sits between the state and the product that consumes it.
+            auto issue_u0 = [&](int j) -> bool {
+                const int s = j % kChStages, d = j & 1;
                 const uint32_t st = sbase + s * Ly::kStage;
-                const uint32_t d1 = tmem + Ly::kTmD1 + s * VS;
-                const uint64_t d_kq = smem_desc(st + Ly::kKQ, 16, 1024, kSw128);
-                const uint64_t d_kit = smem_desc(st + Ly::kKI, 8192, 1024, kSw128);
-                const uint64_t d_tp = smem_desc(st + Ly::kTP, 16, 1024, kSw128);
-                const uint64_t d_p = smem_desc(st + Ly::kTP + 8192, 16, 1024, kSw128);
-                const uint64_t d_v = vs_desc<VS>(st + Ly::kV, 64);
-                if (!wait_or_abort(&bars[cbFull + s], (j >> 1) & 1, abort_flag, p.status)) break;
-                if (j >= 2 && !wait_or_abort(&bars[cbD1Free + s], ((j - 2) >> 1) & 1, abort_flag,
+                if (!spin_or_abort(&bars[cbFull + s], (j / kChStages) & 1, abort_flag, p.status))
+                    return false;
+                KDA_TRACE2(j, 12);
+                if (j >= 2 && !spin_or_abort(&bars[cbD1Free + d], ((j - 2) >> 1) & 1, abort_flag,
                                              p.status))
-                    break;
+                    return false;
                 KDA_TRACE2(j, 1);
                 tc_fence_after();
+                const uint64_t d_tp = smem_desc(st + Ly::kTP, 16, 1024, kSw128);
+                const uint64_t d_v = vs_desc<VS>(st + Ly::kV, 64);
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks)   // D1 = Tb V (U0; zero in rows 64..127)
-                    mma_bf16(d1, d_tp + ((uint64_t)(ks * 32) >> 4), d_v + vs_step<VS>(ks), kIdV,
-                             ks > 0);
-                if (!wait_or_abort(&bars[cbSbFull], j & 1, abort_flag, p.status)) break;
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16(tmem + Ly::kTmD1 + d * VS, d_tp + ((uint64_t)(ks * 32) >> 4),
+                             d_v + vs_step<VS>(ks), kIdV, ks > 0);
+                return true;
+            };
+            bool ok = nchunks > 0 && issue_u0(0);
+            for (int j = 0; j < nchunks && ok; ++j) {
+                const int s = j % kChStages, d = j & 1;
+                const uint32_t st = sbase + s * Ly::kStage;
+                const uint32_t d1 = tmem + Ly::kTmD1 + d * VS;
+                const uint64_t d_kq = smem_desc(st + Ly::kKQ, 16, 1024, kSw128);
+                const uint64_t d_kit = smem_desc(st + Ly::kKI, 8192, 1024, kSw128);
+                if (!spin_or_abort(&bars[cbSbFull], j & 1, abort_flag, p.status)) break;
                 KDA_TRACE2(j, 2);
                 tc_fence_after();
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks)   // D1 += [-W; Qg] S
+                for (int ks = 0; ks < 8; ++ks)   // D1 += [-W; Qe] S
                     mma_bf16(d1, d_kq + kmaj_step(ks, 16384), d_sb + vs_step<VS>(ks), kIdV, 1);
                 mma_commit(&bars[cbUFull]);
                 KDA_TRACE2(j, 3);
-                if (!wait_or_abort(&bars[cbUbFull], j & 1, abort_flag, p.status)) break;
+                if (j + 1 < nchunks && !issue_u0(j + 1)) break;
+                if (!spin_or_abort(&bars[cbUbFull], j & 1, abort_flag, p.status)) break;
                 KDA_TRACE2(j, 4);
                 tc_fence_after();
 #pragma unroll
@@ -505,10 +763,6 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
                     mma_bf16(tmem + Ly::kTmD2, d_kit + ((uint64_t)(ks * 2048) >> 4),
                              d_ub + vs_step<VS>(ks), kIdS, ks > 0);
                 mma_commit(&bars[cbDsFull]);
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)   // D1 += [0; P] U  (O)
-                    mma_bf16(d1, d_p + ((uint64_t)(ks * 32) >> 4), d_ub + vs_step<VS>(ks), kIdV, 1);
-                mma_commit(&bars[cbOFull + s]);
                 mma_commit(&bars[cbStageFree + s]);
                 KDA_TRACE2(j, 5);
             }
@@ -528,35 +782,12 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
                 S[jj] = v.x; S[jj + 1] = v.y; S[jj + 2] = v.z; S[jj + 3] = v.w;
             }
         }
-        auto store_out = [&](int m) {
-            const int sm1 = m & 1;
-            const int c0 = t0 + m * kChunk, L = min(kChunk, t1 - c0);
-            const int r = c - 64;
-#pragma unroll
-            for (int jj = 0; jj < VS; jj += 32) {
-                uint32_t v[32];
-                tmem_ld32(tmem_addr(tmem, 32 * wq, Ly::kTmD1 + sm1 * VS + jj), v);
-                tmem_wait_ld();
-                if (r < L) {
-                    __nv_bfloat16 *dst = p.out + ((size_t)(c0 + r) * p.H + h) * kDV + vs * VS + jj;
-#pragma unroll
-                    for (int e = 0; e < 32; e += 8) {
-                        uint4 w;
-                        w.x = pack2(__uint_as_float(v[e]), __uint_as_float(v[e + 1]));
-                        w.y = pack2(__uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
-                        w.z = pack2(__uint_as_float(v[e + 4]), __uint_as_float(v[e + 5]));
-                        w.w = pack2(__uint_as_float(v[e + 6]), __uint_as_float(v[e + 7]));
-                        *reinterpret_cast<uint4 *>(dst + e) = w;
-                    }
-                }
-            }
-        };
         float gl_cur = 1.f;
         bool ok = true;
         for (int j = 0; j <= nchunks && ok; ++j) {
             if (j > 0) {
                 // S <- Diag(Gam_L) (S + dS) for chunk j-1
-                if (!wait_or_abort(&bars[cbDsFull], (j - 1) & 1, abort_flag, p.status)) { ok = false; break; }
+                if (!spin_or_abort(&bars[cbDsFull], (j - 1) & 1, abort_flag, p.status)) { ok = false; break; }
                 tc_fence_after();
                 if (c == 0) KDA_TRACE2(j - 1, 6);
 #pragma unroll
@@ -568,17 +799,9 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
                     for (int e = 0; e < 32; ++e) S[jj + e] = gl_cur * (S[jj + e] + __uint_as_float(v[e]));
                 }
             }
-            if (j == nchunks) {
-                if (wq >= 2 && j > 0) {
-                    const int m = j - 1;
-                    if (!wait_or_abort(&bars[cbOFull + (m & 1)], (m >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
-                    tc_fence_after();
-                    store_out(m);
-                }
-                break;
-            }
-            const int s = j & 1;
-            if (!wait_or_abort(&bars[cbFull + s], (j >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
+            if (j == nchunks) break;
+            const int s = j % kChStages, d = j & 1;
+            if (!spin_or_abort(&bars[cbFull + s], (j / kChStages) & 1, abort_flag, p.status)) { ok = false; break; }
             gl_cur = reinterpret_cast<const float *>(sm + s * Ly::kStage + Ly::kGL)[c];
             if (c == 0) KDA_TRACE2(j, 7);
             {
@@ -596,16 +819,16 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
             if (lane == 0) mbar_arrive(&bars[cbSbFull]);
             if (c == 0) KDA_TRACE2(j, 8);
 
+            if (!spin_or_abort(&bars[cbUFull], j & 1, abort_flag, p.status)) { ok = false; break; }
+            tc_fence_after();
             if (wq < 2) {
-                // U rows: D1 lanes 0..63 -> bf16 operand
-                if (!wait_or_abort(&bars[cbUFull], j & 1, abort_flag, p.status)) { ok = false; break; }
-                tc_fence_after();
+                // U rows: D1 lanes 0..63 -> bf16 operand of dS
                 if (c == 0) KDA_TRACE2(j, 9);
                 const uint32_t ub = sbase + Ly::kUB;
 #pragma unroll
                 for (int jj = 0; jj < VS; jj += 32) {
                     uint32_t v[32];
-                    tmem_ld32(tmem_addr(tmem, 32 * wq, Ly::kTmD1 + s * VS + jj), v);
+                    tmem_ld32(tmem_addr(tmem, 32 * wq, Ly::kTmD1 + d * VS + jj), v);
                     tmem_wait_ld();
 #pragma unroll
                     for (int e = 0; e < 32; e += 8) {
@@ -621,14 +844,31 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars[cbUbFull]);
                 if (c == 0) KDA_TRACE2(j, 10);
-            } else if (j > 0) {
-                const int m = j - 1;
-                if (!wait_or_abort(&bars[cbOFull + (m & 1)], (m >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
-                tc_fence_after();
-                store_out(m);
+            } else {
+                // O rows: D1 lanes 64..127 -> bf16 output
+                const int c0 = t0 + j * kChunk, L = min(kChunk, t1 - c0);
+                const int r = c - 64;
+#pragma unroll
+                for (int jj = 0; jj < VS; jj += 32) {
+                    uint32_t v[32];
+                    tmem_ld32(tmem_addr(tmem, 32 * wq, Ly::kTmD1 + d * VS + jj), v);
+                    tmem_wait_ld();
+                    if (r < L) {
+                        __nv_bfloat16 *dst = p.out + ((size_t)(c0 + r) * p.H + h) * kDV + vs * VS + jj;
+#pragma unroll
+                        for (int e = 0; e < 32; e += 8) {
+                            uint4 w;
+                            w.x = pack2(__uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+                            w.y = pack2(__uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+                            w.z = pack2(__uint_as_float(v[e + 4]), __uint_as_float(v[e + 5]));
+                            w.w = pack2(__uint_as_float(v[e + 6]), __uint_as_float(v[e + 7]));
+                            *reinterpret_cast<uint4 *>(dst + e) = w;
+                        }
+                    }
+                }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&bars[cbD1Free + (m & 1)]);
+                if (lane == 0) mbar_arrive(&bars[cbD1Free + d]);
             }
         }
         if (ok && p.Sf) {
@@ -639,6 +879,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
         }
     }
 
+    KDA_SPAN(g_kda_span2, 1);
     tc_fence_before();
     __syncthreads();
     if (warp == kChMma) {
@@ -677,6 +918,7 @@ cudaError_t launch_prefill_two_pass(const ForwardArgs &a, cudaStream_t s) {
     kp.packets = a.packets;
     kp.slots = (long long)a.packet_slots;
     kp.status = a.status;
+    kp.work_ctr = a.work_ctr;
     kp.N = a.N;
     kp.H = a.H;
     cudaError_t e = cudaFuncSetAttribute(kside_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -714,6 +956,10 @@ cudaError_t launch_prefill_two_pass(const ForwardArgs &a, cudaStream_t s) {
 #ifdef KDA_TRACE
 extern "C" int kda_trace1_read(unsigned long long *host) {
     return (int)cudaMemcpyFromSymbol(host, kda::g_kda_trace1, sizeof(kda::g_kda_trace1));
+}
+extern "C" int kda_span_read(int which, unsigned long long *host) {
+    return (int)(which == 1 ? cudaMemcpyFromSymbol(host, kda::g_kda_span1, sizeof(kda::g_kda_span1))
+                            : cudaMemcpyFromSymbol(host, kda::g_kda_span2, sizeof(kda::g_kda_span2)));
 }
 extern "C" int kda_trace2_read(unsigned long long *host) {
     return (int)cudaMemcpyFromSymbol(host, kda::g_kda_trace2, sizeof(kda::g_kda_trace2));

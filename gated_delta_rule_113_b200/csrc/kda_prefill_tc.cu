@@ -267,8 +267,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             if (!wait_or_abort(&bars[bApFull], n & 1, abort_flag, p.status)) break;
             tc_fence_after();
             if (t == 0) KDA_TRACE_EVENT(n, 4);
-            solve_chunk(sw, lane, tmem, Ly::kTmAP, sbase + Ly::kTP + s * 24576, sL, sT, sXw,
+            solve_chunk(sw, lane, tmem, Ly::kTmAP, sbase + Ly::kTP + s * 24576 + 16384, sL, sT, sXw,
                         sB + s * 64, &bars[bApFree], kBarSolve);
+            write_tb(sw, lane, sbase + Ly::kTP + s * 24576, sT, sB + s * 64, kBarSolve);
             if (t == 0) mbar_arrive(&bars[bTbFull + s]);
             if (t == 0) KDA_TRACE_EVENT(n, 9);
 

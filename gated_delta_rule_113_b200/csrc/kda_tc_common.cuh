@@ -43,6 +43,26 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity,
     return false;
 }
 
+// Bounded wait that polls instead of suspending: for the few threads on a
+// latency-critical chain, where the wake-up of a suspended waiter costs
+// hundreds of cycles.  Same 2 s limit and abort protocol as wait_or_abort.
+__device__ __forceinline__ bool spin_or_abort(uint64_t *bar, uint32_t parity,
+                                              volatile int *abort_flag, int32_t *status) {
+    uint64_t start = 0;
+    for (uint32_t n = 1;; ++n) {
+        if (mbar_test_wait(bar, parity)) return true;
+        if ((n & 1023u) == 0) {
+            if (*abort_flag) return false;
+            const uint64_t now = globaltimer_ns();
+            if (start == 0) start = now;
+            else if (now - start > 2000000000ull) break;
+        }
+    }
+    *abort_flag = 1;
+    set_status(status, KDA_ERR_TIMEOUT);
+    return false;
+}
+
 // 16-byte shared store / load helpers
 __device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
                                        uint32_t d) {
@@ -103,6 +123,10 @@ __device__ __forceinline__ void prep_chunk(int t, uint32_t kq_stage, uint32_t ki
     const int a = cg >> 3, ch = cg & 7;
     const uint32_t kq = kq_stage + a * 16384;
     const uint32_t ki = ki_stage + a * 8192;
+    // beta comes from global memory: start its load before anything else
+    float beta_r = 0.f;
+    if (t >= 128 && t < 128 + kChunk && t - 128 < L)
+        beta_r = __bfloat162float(beta[(size_t)(c0 + t - 128) * H + h]);
     // pass 0: alpha; in-group prefix and suffix products
     float pre[4][8], suf[4][8];
 #pragma unroll
@@ -158,8 +182,7 @@ __device__ __forceinline__ void prep_chunk(int t, uint32_t kq_stage, uint32_t ki
             sx *= gv[g];
         }
     } else if (t < 128 + kChunk) {
-        const int r = t - 128;
-        sB_s[r] = r < L ? __bfloat162float(beta[(size_t)(c0 + r) * H + h]) : 0.f;
+        sB_s[t - 128] = beta_r;
     }
     named_bar(bar_id, kPrepThreads);
     // pass 1: Gam_r = pre_group * pre[i]; 1/Gam_r = (1/Gam_L) suf_group suf[i]
@@ -203,60 +226,75 @@ __device__ __forceinline__ void prep_chunk(int t, uint32_t kq_stage, uint32_t ki
 // ---------------------------------------------------------------------------
 // Solve for one chunk, run by 4 warps (sw = 0..3 owns TMEM lanes 32 sw..) that
 // synchronise on named barrier `bar_id`.  Reads D_AP from TMEM (column
-// tm_ap), writes L = strict_lower(diag(b) A) to sL and the masked bf16 P into
-// TP rows 128..191, arrives once on `ap_free` when D_AP may be overwritten,
-// then builds T = (I + L)^{-1} (16x16 diagonal blocks by substitution, then a
-// block forward substitution per 16-column block with mma.sync tf32) and
-// writes Tb = T diag(b) as bf16 into TP rows 0..63.  Blocks of sT above the
-// diagonal blocks must be zero on entry (they are never written).  sXw is
-// 4 x [16][17] fp32 warp-private scratch.  Ends with a proxy fence and a
-// barrier.
+// tm_ap), writes L = strict_lower(diag(b) A) to sL and the masked bf16 P as a
+// 64-row K-major tile at `p_tile`, arrives once on `ap_free` when D_AP may be
+// overwritten, then builds T = (I + L)^{-1} in sT (16x16 diagonal blocks by
+// substitution, then a block forward substitution by 8-column strips with
+// mma.sync tf32).  Blocks of sT above the diagonal blocks must be zero on
+// entry (they are never written).  sXw is 4 x [16][17] fp32 warp-private
+// scratch.  write_tb() then turns T into the bf16 Tb tile.
 // ---------------------------------------------------------------------------
+// P = lower_incl(Q K^T) rows (TMEM lanes 64..127 of the A/P accumulator at
+// column tm_ap) -> masked bf16 64-row K-major tile at `p_tile`.  Run by the
+// solve warps with lane quarters 2 and 3 (sw = 2, 3); a no-op for sw < 2.
+__device__ __forceinline__ void write_p(int sw, int lane, uint32_t tmem, uint32_t tm_ap,
+                                       uint32_t p_tile) {
+    if (sw < 2) return;
+    const int r = 32 * (sw & 1) + lane;
+    uint32_t v0[32], v1[32];
+    tmem_ld32(tmem_addr(tmem, 32 * sw, tm_ap), v0);
+    tmem_ld32(tmem_addr(tmem, 32 * sw, tm_ap + 32), v1);
+    tmem_wait_ld();
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        uint32_t o[4];
+#pragma unroll
+        for (int e2 = 0; e2 < 4; ++e2) {
+            const int c = 8 * j + 2 * e2;
+            const uint32_t *src = c < 32 ? &v0[c] : &v1[c - 32];
+            const float x0 = (c <= r) ? __uint_as_float(src[0]) : 0.f;
+            const float x1 = (c + 1 <= r) ? __uint_as_float(src[1]) : 0.f;
+            o[e2] = pack2(x0, x1);
+        }
+        sts128(p_tile + sw128_off(r, j), o[0], o[1], o[2], o[3]);
+    }
+}
+
+// kEarlyP: write P and release D_AP (one arrival on `ap_free`) right after
+// reading L.  Otherwise P stays in TMEM: the caller writes it with write_p()
+// and arrives on `ap_free` itself, later.
+template <bool kEarlyP = true>
 __device__ __forceinline__ void solve_chunk(int sw, int lane, uint32_t tmem, uint32_t tm_ap,
-                                            uint32_t tp, float *sL, float *sT, float *sXw,
+                                            uint32_t p_tile, float *sL, float *sT, float *sXw,
                                             const float *sB_s, uint64_t *ap_free,
                                             uint32_t bar_id) {
     const int t = sw * 32 + lane;
     const int g = lane >> 2, tq = lane & 3;
-    {
-        const int r = 32 * (sw & 1) + lane;  // row within A (sw<2) or P (sw>=2)
+    if (sw < 2) {
+        // L = strict_lower(diag(b) A)
+        const int r = 32 * sw + lane;
         uint32_t v0[32], v1[32];
         tmem_ld32(tmem_addr(tmem, 32 * sw, tm_ap), v0);
         tmem_ld32(tmem_addr(tmem, 32 * sw, tm_ap + 32), v1);
         tmem_wait_ld();
-        if (sw < 2) {
-            // L = strict_lower(diag(b) A)
-            const float br = sB_s[r];
-            float *Lr = sL + r * kLDL;
+        const float br = sB_s[r];
+        float *Lr = sL + r * kLDL;
 #pragma unroll
-            for (int c = 0; c < 64; c += 4) {
-                const uint32_t *src = c < 32 ? &v0[c] : &v1[c - 32];
-                float4 w;
-                w.x = (c + 0 < r) ? br * __uint_as_float(src[0]) : 0.f;
-                w.y = (c + 1 < r) ? br * __uint_as_float(src[1]) : 0.f;
-                w.z = (c + 2 < r) ? br * __uint_as_float(src[2]) : 0.f;
-                w.w = (c + 3 < r) ? br * __uint_as_float(src[3]) : 0.f;
-                *reinterpret_cast<float4 *>(Lr + c) = w;
-            }
-        } else {
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                uint32_t o[4];
-#pragma unroll
-                for (int e2 = 0; e2 < 4; ++e2) {
-                    const int c = 8 * j + 2 * e2;
-                    const uint32_t *src = c < 32 ? &v0[c] : &v1[c - 32];
-                    const float x0 = (c <= r) ? __uint_as_float(src[0]) : 0.f;
-                    const float x1 = (c + 1 <= r) ? __uint_as_float(src[1]) : 0.f;
-                    o[e2] = pack2(x0, x1);
-                }
-                sts128(tp + 16384 + sw128_off(r, j), o[0], o[1], o[2], o[3]);
-            }
+        for (int c = 0; c < 64; c += 4) {
+            const uint32_t *src = c < 32 ? &v0[c] : &v1[c - 32];
+            float4 w;
+            w.x = (c + 0 < r) ? br * __uint_as_float(src[0]) : 0.f;
+            w.y = (c + 1 < r) ? br * __uint_as_float(src[1]) : 0.f;
+            w.z = (c + 2 < r) ? br * __uint_as_float(src[2]) : 0.f;
+            w.w = (c + 3 < r) ? br * __uint_as_float(src[3]) : 0.f;
+            *reinterpret_cast<float4 *>(Lr + c) = w;
         }
+    } else if (kEarlyP) {
+        write_p(sw, lane, tmem, tm_ap, p_tile);
     }
     tc_fence_before();
     named_bar(bar_id, kSolveThreads);
-    if (t == 0) mbar_arrive(ap_free);
+    if (kEarlyP && t == 0) mbar_arrive(ap_free);
 
     // phase 1: invert the four 16x16 diagonal blocks, one block per warp, one
     // column per lane (lanes 0-15)
@@ -283,87 +321,86 @@ __device__ __forceinline__ void solve_chunk(int sw, int lane, uint32_t tmem, uin
     }
     named_bar(bar_id, kSolveThreads);
 
-    // phase 2: block forward substitution, warp sw owning the 16 columns
-    // [16 sw, 16 sw + 16) of T.  Block rows above sw are zero, block row sw is
-    // D_sw, and for i > sw:  T_i = -D_i * sum_{sw <= j < i} L_ij T_j.  Each warp
-    // only reads L, the diagonal blocks and its own columns, so no barrier is
-    // needed until the whole Tb tile is written.  X goes through a warp-private
+    // phase 2: block forward substitution by 8-column strips.  Block rows
+    // above a strip's block column cb are zero, block row cb is D_cb, and for
+    // i > cb:  T_i = -D_i * sum_{cb <= j < i} L_ij T_j.  Column block 0 costs
+    // the most (three block rows), so its two strips go to warps 0 and 1 and
+    // warps 2 and 3 take the strips of blocks 1 and 2; block 3 is D_3 alone.
+    // A strip only reads L, the diagonal blocks and its own columns, so no
+    // barrier is needed until Tb is written.  X goes through a warp-private
     // [16][17] scratch to turn accumulator fragments into B fragments.
     {
         float *xw = sXw + sw * 16 * 17;
-        const int c0 = 16 * sw;
-        for (int i = sw + 1; i < 4; ++i) {
-            float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-            for (int jb = sw; jb < i; ++jb) {
+        const int q = sw & 1;
+#pragma unroll 1
+        for (int pass = 0; pass < 2; ++pass) {
+            const int cb = sw < 2 ? (pass == 0 ? 0 : 4) : 1 + pass;
+            const int c0 = 16 * cb + 8 * q;
+            for (int i = cb + 1; i < 4; ++i) {
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                for (int jb = cb; jb < i; ++jb) {
 #pragma unroll
-                for (int kk = 0; kk < 16; kk += 8) {
-                    const float *Lr = sL + (16 * i + g) * kLDL + 16 * jb + kk + tq;
-                    const uint32_t af[4] = {tf32_bits(Lr[0]), tf32_bits(Lr[8 * kLDL]),
-                                            tf32_bits(Lr[4]), tf32_bits(Lr[8 * kLDL + 4])};
-#pragma unroll
-                    for (int q = 0; q < 2; ++q) {
-                        const float *Tc = sT + (16 * jb + kk + tq) * kLDL + c0 + 8 * q + g;
+                    for (int kk = 0; kk < 16; kk += 8) {
+                        const float *Lr = sL + (16 * i + g) * kLDL + 16 * jb + kk + tq;
+                        const uint32_t af[4] = {tf32_bits(Lr[0]), tf32_bits(Lr[8 * kLDL]),
+                                                tf32_bits(Lr[4]), tf32_bits(Lr[8 * kLDL + 4])};
+                        const float *Tc = sT + (16 * jb + kk + tq) * kLDL + c0 + g;
                         const uint32_t bfr[2] = {tf32_bits(Tc[0]), tf32_bits(Tc[4 * kLDL])};
-                        mma_tf32_16x8x8(acc[q], af, bfr);
+                        mma_tf32_16x8x8(acc, af, bfr);
                     }
                 }
-            }
+                xw[g * 17 + 2 * tq] = acc[0];
+                xw[g * 17 + 2 * tq + 1] = acc[1];
+                xw[(g + 8) * 17 + 2 * tq] = acc[2];
+                xw[(g + 8) * 17 + 2 * tq + 1] = acc[3];
+                __syncwarp();
+                float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int q = 0; q < 2; ++q) {
-                xw[g * 17 + 8 * q + 2 * tq] = acc[q][0];
-                xw[g * 17 + 8 * q + 2 * tq + 1] = acc[q][1];
-                xw[(g + 8) * 17 + 8 * q + 2 * tq] = acc[q][2];
-                xw[(g + 8) * 17 + 8 * q + 2 * tq + 1] = acc[q][3];
-            }
-            __syncwarp();
-            float d[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-            for (int kk = 0; kk < 16; kk += 8) {
-                const float *Dr = sT + (16 * i + g) * kLDL + 16 * i + kk + tq;
-                const uint32_t af[4] = {tf32_bits(Dr[0]), tf32_bits(Dr[8 * kLDL]),
-                                        tf32_bits(Dr[4]), tf32_bits(Dr[8 * kLDL + 4])};
-#pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    const uint32_t bfr[2] = {tf32_bits(xw[(kk + tq) * 17 + 8 * q + g]),
-                                             tf32_bits(xw[(kk + tq + 4) * 17 + 8 * q + g])};
-                    mma_tf32_16x8x8(d[q], af, bfr);
+                for (int kk = 0; kk < 16; kk += 8) {
+                    const float *Dr = sT + (16 * i + g) * kLDL + 16 * i + kk + tq;
+                    const uint32_t af[4] = {tf32_bits(Dr[0]), tf32_bits(Dr[8 * kLDL]),
+                                            tf32_bits(Dr[4]), tf32_bits(Dr[8 * kLDL + 4])};
+                    const uint32_t bfr[2] = {tf32_bits(xw[(kk + tq) * 17 + g]),
+                                             tf32_bits(xw[(kk + tq + 4) * 17 + g])};
+                    mma_tf32_16x8x8(d, af, bfr);
                 }
+                float *o = sT + (16 * i) * kLDL + c0;
+                o[g * kLDL + 2 * tq] = -d[0];
+                o[g * kLDL + 2 * tq + 1] = -d[1];
+                o[(g + 8) * kLDL + 2 * tq] = -d[2];
+                o[(g + 8) * kLDL + 2 * tq + 1] = -d[3];
+                __syncwarp();
             }
-#pragma unroll
-            for (int q = 0; q < 2; ++q) {
-                float *o = sT + (16 * i) * kLDL + c0 + 8 * q;
-                o[g * kLDL + 2 * tq] = -d[q][0];
-                o[g * kLDL + 2 * tq + 1] = -d[q][1];
-                o[(g + 8) * kLDL + 2 * tq] = -d[q][2];
-                o[(g + 8) * kLDL + 2 * tq + 1] = -d[q][3];
-            }
-            __syncwarp();
         }
     }
 
-    // Tb = T diag(b) -> bf16 into rows 0..63 of the Tb|0|P tile; warp sw
-    // writes its own 16 columns (two 16-byte chunks of every row)
+}
+
+// Tb = T diag(b) -> bf16 into rows 0..63 of the K-major tile at `tp`, one
+// 8-column chunk at a time: each warp writes the strips it computed in
+// solve_chunk, and warps 0 and 1 also the two strips of block 3 (D_3, final
+// since phase 1), so only the caller's own ordering is needed before it.
+// Ends with a proxy fence and a barrier.
+__device__ __forceinline__ void write_tb(int sw, int lane, uint32_t tp, const float *sT,
+                                         const float *sB_s, uint32_t bar_id) {
     {
-        const int c0 = 16 * sw;
-        const float *bs = sB_s + c0;
-        const float4 b0 = *reinterpret_cast<const float4 *>(bs);
-        const float4 b1 = *reinterpret_cast<const float4 *>(bs + 4);
-        const float4 b2 = *reinterpret_cast<const float4 *>(bs + 8);
-        const float4 b3 = *reinterpret_cast<const float4 *>(bs + 12);
+        const int q = sw & 1;
 #pragma unroll
-        for (int rr = 0; rr < 2; ++rr) {
-            const int r = lane + 32 * rr;
-            const float *Tr = sT + r * kLDL + c0;
-            const float4 t0 = *reinterpret_cast<const float4 *>(Tr);
-            const float4 t1 = *reinterpret_cast<const float4 *>(Tr + 4);
-            const float4 t2 = *reinterpret_cast<const float4 *>(Tr + 8);
-            const float4 t3 = *reinterpret_cast<const float4 *>(Tr + 12);
-            sts128(tp + sw128_off(r, 2 * sw), pack2(t0.x * b0.x, t0.y * b0.y),
-                   pack2(t0.z * b0.z, t0.w * b0.w), pack2(t1.x * b1.x, t1.y * b1.y),
-                   pack2(t1.z * b1.z, t1.w * b1.w));
-            sts128(tp + sw128_off(r, 2 * sw + 1), pack2(t2.x * b2.x, t2.y * b2.y),
-                   pack2(t2.z * b2.z, t2.w * b2.w), pack2(t3.x * b3.x, t3.y * b3.y),
-                   pack2(t3.z * b3.z, t3.w * b3.w));
+        for (int pass = 0; pass < 2; ++pass) {
+            const int cb = sw < 2 ? (pass == 0 ? 0 : 3) : 1 + pass;
+            const int ch = 2 * cb + q;
+            const float4 b0 = *reinterpret_cast<const float4 *>(sB_s + 8 * ch);
+            const float4 b1 = *reinterpret_cast<const float4 *>(sB_s + 8 * ch + 4);
+#pragma unroll
+            for (int rr = 0; rr < 2; ++rr) {
+                const int r = lane + 32 * rr;
+                const float *Tr = sT + r * kLDL + 8 * ch;
+                const float4 t0 = *reinterpret_cast<const float4 *>(Tr);
+                const float4 t1 = *reinterpret_cast<const float4 *>(Tr + 4);
+                sts128(tp + sw128_off(r, ch), pack2(t0.x * b0.x, t0.y * b0.y),
+                       pack2(t0.z * b0.z, t0.w * b0.w), pack2(t1.x * b1.x, t1.y * b1.y),
+                       pack2(t1.z * b1.z, t1.w * b1.w));
+            }
         }
     }
     fence_proxy_async();

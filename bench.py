@@ -93,11 +93,18 @@ def traffic_record(kernel):
     rec = recs.get(kernel)
     if not rec:
         return None
-    src = os.path.join(ROOT, rec["source"])
-    if not os.path.exists(src):
-        return None
-    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    return rec["bytes_per_launch"] if sha == rec.get("source_sha") else None
+    return rec["bytes_per_launch"] if sources_sha(rec) == rec.get("source_sha") else None
+
+
+def sources_sha(rec):
+    """Digest of every source file the recorded kernels are built from."""
+    h = hashlib.sha256()
+    for rel in rec.get("sources", [rec.get("source")]):
+        src = os.path.join(ROOT, rel)
+        if not os.path.exists(src):
+            return None
+        h.update(open(src, "rb").read())
+    return h.hexdigest()[:16]
 
 
 # --------------------------------------------------------------------------
@@ -364,7 +371,7 @@ def bench_kda(args):
     achieved = alg_bytes / (mean_ms * 1e-3) / 1e9
     roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": achieved / peaks["hbm_gbs"], "traffic": traffic_record("kda_prefill"),
-            "peak_kind": f"{peaks_kind} HBM copy", "kernel": "kda_forward (varlen index + prefill)",
+            "peak_kind": f"{peaks_kind} HBM copy", "kernel": "kda_forward (varlen_index + kside + chain kernels, one call)",
             "algorithmic_bytes": alg_bytes, "algorithmic_flops": alg_flops,
             "tensor_frac_algorithmic": alg_flops / (mean_ms * 1e-3) / 1e12 / peaks["bf16_tflops"]}
 
@@ -384,7 +391,10 @@ def bench_kda(args):
                        "parallelism": f"replicas x{world}"},
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
-            "gpu_launches": 2 * args.steps,
+            # per call: varlen index, then the key-side and chain passes
+            # (bf16, d = 128, full workspace) or the one CUDA-core kernel
+            "gpu_launches": (3 if (w.torch_dtype == torch.bfloat16 and Dk == 128 and Dv == 128)
+                             else 2) * args.steps,
             "roofline": roof,
             "cpu_baseline": cpu,
             "decode": dec,

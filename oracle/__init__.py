@@ -65,6 +65,10 @@ def bind(path: str):
     lib.kda_oracle_forward.argtypes = [
         i64, ctypes.POINTER(i64), i64, i64, i64,
         dp, dp, dp, dp, dp, dp, dp, dp, ctypes.c_int]
+    lib.kda_oracle_forward_snapshots.restype = ctypes.c_int
+    lib.kda_oracle_forward_snapshots.argtypes = [
+        i64, ctypes.POINTER(i64), i64, i64, i64,
+        dp, dp, dp, dp, dp, dp, dp, dp, i64, ctypes.POINTER(i64), dp, ctypes.c_int]
     lib.kda_oracle_decode_step.restype = ctypes.c_int
     lib.kda_oracle_decode_step.argtypes = [
         i64, i64, i64, i64, dp, dp, dp, dp, dp, dp, dp, ctypes.c_int]
@@ -99,7 +103,8 @@ def _ptr(a):
     return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
 
 
-def forward(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, threads=None, lib=None):
+def forward(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, threads=None, lib=None,
+            snapshot_every=None):
     """Token-by-token fp64 KDA over packed sequences.
 
     Shapes: q, k, log_alpha [T_tot, H, Dk]; v [T_tot, H, Dv]; beta [T_tot, H];
@@ -107,6 +112,13 @@ def forward(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, threads=None, li
     sequence of length T_tot).  Returns (out [T_tot, H, Dv], S_final
     [N, H, Dk, Dv]) as float64 arrays.  ``lib`` (tests only) substitutes
     another build of the same C source.
+
+    With ``snapshot_every`` = E > 0 it returns (out, S_final, snaps, snap_off):
+    snaps [M, H, Dk, Dv] holds the state of every chain right after each
+    E-th token of its sequence (page "Kimi K3: Open Frontier Intelligence and
+    Implementation Framework", section "Inference Serving", KDA-aware prefix
+    caching), sequence n's m-th one (m = 0, 1, ...) at index snap_off[n] + m,
+    with snap_off the exclusive prefix sum of floor(len_n / E).
     """
     q, k, v, la, b = (_f64(x) for x in (q, k, v, log_alpha, beta))
     T, H, Dk = q.shape
@@ -131,13 +143,34 @@ def forward(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, threads=None, li
             raise ValueError("S0 must be [N, H, Dk, Dv]")
     out = np.zeros((T, H, Dv), dtype=np.float64)
     sf = np.zeros((N, H, Dk, Dv), dtype=np.float64)
-    rc = (lib or _load()).kda_oracle_forward(
+    if snapshot_every is None:
+        rc = (lib or _load()).kda_oracle_forward(
+            N, cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), H, Dk, Dv,
+            _ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(b), _ptr(s0), _ptr(out),
+            _ptr(sf), int(threads or default_threads()))
+        if rc != 0:
+            raise RuntimeError(f"kda_oracle_forward failed with code {rc}")
+        return out, sf
+    E = int(snapshot_every)
+    if E <= 0:
+        raise ValueError("snapshot_every must be positive")
+    counts = np.diff(cu) // E
+    snap_off = np.ascontiguousarray(np.concatenate([[0], np.cumsum(counts)[:-1]]).astype(np.int64)
+                                    if N > 0 else np.zeros(0, dtype=np.int64))
+    # Guard slots past the end: the mutation tests run deliberately broken
+    # builds of this C source in-process, and a snapshot written one slot too
+    # far must land in memory this array owns.
+    M = int(counts.sum())
+    snaps_buf = np.zeros((M + 4, H, Dk, Dv), dtype=np.float64)
+    snaps = snaps_buf[:M]
+    rc = (lib or _load()).kda_oracle_forward_snapshots(
         N, cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), H, Dk, Dv,
         _ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(b), _ptr(s0), _ptr(out),
-        _ptr(sf), int(threads or default_threads()))
+        _ptr(sf), E, snap_off.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
+        _ptr(snaps_buf) if M else None, int(threads or default_threads()))
     if rc != 0:
-        raise RuntimeError(f"kda_oracle_forward failed with code {rc}")
-    return out, sf
+        raise RuntimeError(f"kda_oracle_forward_snapshots failed with code {rc}")
+    return out, sf, snaps, snap_off
 
 
 def decode_step(q, k, v, log_alpha, beta, S, threads=None):

@@ -44,6 +44,16 @@
  * Layouts (row-major, packed token axis of length T_tot):
  *   q, k, log_alpha : [T_tot, H, Dk]     v, out : [T_tot, H, Dv]
  *   beta            : [T_tot, H]         S0, S_final : [N, H, Dk, Dv]
+ *
+ * State snapshots.  The same page, section "Inference Serving", bullet
+ * "KDA-Aware Prefix Caching", keeps KDA recurrent states in a paged pool so
+ * that a prefix can be resumed at 512-token boundaries.  Reading taken: a
+ * snapshot is the state of a (sequence, head) chain right after token
+ * number m * every of that sequence (m = 1, 2, ...; counted from the
+ * sequence start), for every such m inside the sequence.  The oracle writes
+ * snapshot m-1 of sequence n to snap[(snap_off[n] + m - 1), h] (layout
+ * [*, H, Dk, Dv]); resuming from a snapshot is a forward pass whose S0 is
+ * that snapshot.
  */
 #include <math.h>
 #include <pthread.h>
@@ -56,6 +66,9 @@ typedef struct {
     const int64_t *cu;
     const double *q, *k, *v, *la, *beta, *S0;
     double *out, *Sf;
+    int64_t snap_every;      /* tokens between snapshots; 0: none */
+    const int64_t *snap_off; /* [N] first snapshot index of each sequence */
+    double *snap;            /* [*, H, Dk, Dv] */
     int64_t next;            /* next chain index, taken under the lock */
     pthread_mutex_t lock;
 } job_t;
@@ -106,6 +119,12 @@ static void run_chain(const job_t *J, int64_t n, int64_t h, double *S, double *e
             const double *row = S + c * Dv;
             for (int64_t j = 0; j < Dv; ++j) ot[j] = ot[j] + qc * row[j];
         }
+        /* snapshot after token number (t - t0 + 1) of the sequence */
+        const int64_t done = t - t0 + 1;
+        if (J->snap && done % J->snap_every == 0) {
+            const int64_t m = J->snap_off[n] + done / J->snap_every - 1;
+            memcpy(J->snap + (m * H + h) * Dk * Dv, S, sizeof(double) * Dk * Dv);
+        }
     }
     if (J->Sf)
         memcpy(J->Sf + (n * H + h) * Dk * Dv, S, sizeof(double) * Dk * Dv);
@@ -136,13 +155,39 @@ static void *worker(void *arg)
  * S0 slice before it writes the same slice of S_final).
  * Returns 0 on success, -1 on bad arguments, -2 on allocation/thread failure.
  */
+int kda_oracle_forward_snapshots(int64_t n_seqs, const int64_t *cu_seqlens, int64_t H,
+                                 int64_t Dk, int64_t Dv, const double *q, const double *k,
+                                 const double *v, const double *log_alpha,
+                                 const double *beta, const double *S0, double *out,
+                                 double *S_final, int64_t snap_every,
+                                 const int64_t *snap_off, double *snap, int n_threads);
+
 int kda_oracle_forward(int64_t n_seqs, const int64_t *cu_seqlens, int64_t H,
                        int64_t Dk, int64_t Dv, const double *q, const double *k,
                        const double *v, const double *log_alpha,
                        const double *beta, const double *S0, double *out,
                        double *S_final, int n_threads)
 {
+    return kda_oracle_forward_snapshots(n_seqs, cu_seqlens, H, Dk, Dv, q, k, v, log_alpha,
+                                        beta, S0, out, S_final, 0, NULL, NULL, n_threads);
+}
+
+/*
+ * kda_oracle_forward_snapshots: kda_oracle_forward that also records the
+ * state snapshots described at the top of this file.  snap_every = 0 (or
+ * snap = NULL) records none.  snap_off[n] is the index of sequence n's first
+ * snapshot; the caller sizes snap for sum_n floor(len_n / snap_every) of
+ * them.
+ */
+int kda_oracle_forward_snapshots(int64_t n_seqs, const int64_t *cu_seqlens, int64_t H,
+                                 int64_t Dk, int64_t Dv, const double *q, const double *k,
+                                 const double *v, const double *log_alpha,
+                                 const double *beta, const double *S0, double *out,
+                                 double *S_final, int64_t snap_every,
+                                 const int64_t *snap_off, double *snap, int n_threads)
+{
     if (n_seqs < 0 || H <= 0 || Dk <= 0 || Dv <= 0 || !cu_seqlens) return -1;
+    if (snap && (snap_every <= 0 || !snap_off)) return -1;
     for (int64_t n = 0; n < n_seqs; ++n)
         if (cu_seqlens[n + 1] < cu_seqlens[n]) return -1;
     if (cu_seqlens[0] != 0) return -1;
@@ -153,6 +198,7 @@ int kda_oracle_forward(int64_t n_seqs, const int64_t *cu_seqlens, int64_t H,
     J.n_seqs = n_seqs; J.H = H; J.Dk = Dk; J.Dv = Dv; J.cu = cu_seqlens;
     J.q = q; J.k = k; J.v = v; J.la = log_alpha; J.beta = beta; J.S0 = S0;
     J.out = out; J.Sf = S_final; J.next = 0;
+    J.snap_every = snap ? snap_every : 0; J.snap_off = snap_off; J.snap = snap;
     pthread_mutex_init(&J.lock, NULL);
 
     const int64_t total = n_seqs * H;

@@ -287,3 +287,63 @@ def test_bad_seqlens_rejected():
         oracle.forward(q, k, v, la, beta, cu_seqlens=[0, 3, 2, 4])
     with pytest.raises(ValueError):
         oracle.forward(q, k, v, la, beta, cu_seqlens=[0, 3])
+
+
+# --------------------------------------------------------------------------
+# state snapshots (prefix caching at fixed token boundaries)
+# --------------------------------------------------------------------------
+def _snapshot_case(seed=21, E=16):
+    rng = np.random.default_rng(seed)
+    lens = [50, 7, 32, 0, 65]   # partial, shorter than E, exact multiple, empty, one past
+    T, H, Dk, Dv = sum(lens), 2, 6, 5
+    q, k, v, la, beta, _ = _rand_chain(rng, T, H, Dk, Dv)
+    S0 = 0.1 * rng.standard_normal((len(lens), H, Dk, Dv))
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    return lens, cu, E, (q, k, v, la, beta, S0)
+
+
+def test_snapshot_counts_and_offsets():
+    lens, cu, E, (q, k, v, la, beta, S0) = _snapshot_case()
+    o, s, snaps, off = oracle.forward(q, k, v, la, beta, S0=S0, cu_seqlens=cu, snapshot_every=E)
+    counts = [n // E for n in lens]
+    assert snaps.shape[0] == sum(counts)
+    assert list(off) == list(np.concatenate([[0], np.cumsum(counts)[:-1]]))
+    # the plain call returns the same outputs and final states
+    o2, s2 = oracle.forward(q, k, v, la, beta, S0=S0, cu_seqlens=cu)
+    assert np.array_equal(o, o2) and np.array_equal(s, s2)
+
+
+def test_snapshot_equals_final_state_of_the_prefix():
+    """Snapshot m of sequence n is the final state of the same chain run on the
+    first (m + 1) E tokens only, through the plain entry point."""
+    lens, cu, E, (q, k, v, la, beta, S0) = _snapshot_case()
+    _, _, snaps, off = oracle.forward(q, k, v, la, beta, S0=S0, cu_seqlens=cu, snapshot_every=E)
+    checked = 0
+    for n, L in enumerate(lens):
+        for m in range(L // E):
+            a, b = cu[n], cu[n] + (m + 1) * E
+            _, sp = oracle.forward(q[a:b], k[a:b], v[a:b], la[a:b], beta[a:b], S0=S0[n:n + 1])
+            assert np.allclose(snaps[off[n] + m], sp[0], rtol=1e-13, atol=1e-14)
+            checked += 1
+    assert checked == sum(L // E for L in lens)
+
+
+def test_resume_from_snapshot_reproduces_the_tail():
+    """A prefill started from snapshot m (as S0) on the rest of the sequence gives
+    the same outputs and final state as the uninterrupted run."""
+    lens, cu, E, (q, k, v, la, beta, S0) = _snapshot_case()
+    o, s, snaps, off = oracle.forward(q, k, v, la, beta, S0=S0, cu_seqlens=cu, snapshot_every=E)
+    n, m = 4, 3                      # sequence of 65 tokens, resume after token 64
+    a = cu[n] + (m + 1) * E
+    b = cu[n + 1]
+    o2, s2 = oracle.forward(q[a:b], k[a:b], v[a:b], la[a:b], beta[a:b],
+                            S0=snaps[off[n] + m][None])
+    assert np.allclose(o2, o[a:b], rtol=1e-13, atol=1e-14)
+    assert np.allclose(s2[0], s[n], rtol=1e-13, atol=1e-14)
+
+
+def test_snapshot_at_sequence_end_is_the_final_state():
+    lens, cu, E, (q, k, v, la, beta, S0) = _snapshot_case()
+    _, s, snaps, off = oracle.forward(q, k, v, la, beta, S0=S0, cu_seqlens=cu, snapshot_every=E)
+    n = 2                            # 32 tokens = 2 E: its last snapshot is its final state
+    assert np.array_equal(snaps[off[n] + 1], s[n])

@@ -29,6 +29,9 @@ MUTANTS = [
      "const double *vt = J->v + (t * H + 0) * Dv;"),
     ("s0_ignored", "memcpy(S, J->S0 + (n * H + h) * Dk * Dv, sizeof(double) * Dk * Dv);",
      "memset(S, 0, sizeof(double) * Dk * Dv);"),
+    ("snapshot_one_token_early", "const int64_t done = t - t0 + 1;", "const int64_t done = t - t0 + 2;"),
+    ("snapshot_wrong_slot", "const int64_t m = J->snap_off[n] + done / J->snap_every - 1;",
+     "const int64_t m = J->snap_off[n] + done / J->snap_every - 1 + (done > J->snap_every);"),
 ]
 
 
@@ -78,8 +81,27 @@ def _exact_write_pin(lib) -> bool:
     return bool(np.allclose(out, v, atol=1e-12))
 
 
+def _snapshot_pin(lib) -> bool:
+    """Snapshots equal the final states of the prefixes (plain entry point)."""
+    rng = np.random.default_rng(3)
+    lens, E = [37, 20], 8
+    T, H, D = sum(lens), 2, 3
+    q, k, v = (rng.standard_normal((T, H, D)) for _ in range(3))
+    la = rng.uniform(-0.5, 0.0, size=(T, H, D))
+    beta = rng.uniform(0.2, 1.0, size=(T, H))
+    cu = np.array([0, lens[0], T])
+    _, _, snaps, off = oracle.forward(q, k, v, la, beta, cu_seqlens=cu, lib=lib, snapshot_every=E)
+    ok = snaps.shape[0] == sum(L // E for L in lens)
+    for n, L in enumerate(lens):
+        for m in range(L // E):
+            a, b = cu[n], cu[n] + (m + 1) * E
+            _, sp = oracle.forward(q[a:b], k[a:b], v[a:b], la[a:b], beta[a:b], lib=lib)
+            ok = ok and np.allclose(snaps[off[n] + m], sp[0], rtol=1e-12, atol=1e-12)
+    return bool(ok)
+
+
 def _pins_pass(lib) -> bool:
-    return _exact_pin(lib) and _exact_write_pin(lib)
+    return _exact_pin(lib) and _exact_write_pin(lib) and _snapshot_pin(lib)
 
 
 def test_real_source_passes(tmp_path):

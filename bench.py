@@ -358,6 +358,41 @@ def bench_kda(args):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
     e2e_value = world * T * args.steps / (e2e_ms * 1e-3)
 
+    # ---- prefix-cache snapshots: the same forward keeping the state every
+    # 512 tokens in a slot pool (bf16, d = 128 only) ------------------------
+    snap = None
+    if not args.no_snapshots and w.torch_dtype == torch.bfloat16 and Dk == 128 and Dv == 128:
+        every = 512
+        counts = [n // every for n in inp["lengths"]]
+        base = torch.tensor([sum(counts[:i]) for i in range(N)], dtype=torch.int32, device=dev)
+        pool = torch.empty((max(1, sum(counts)), H, Dk, Dv), dtype=torch.float32, device=dev)
+
+        def snap_step():
+            kda.forward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["S0"],
+                        d["cu_seqlens"], out=out, S_final=sf, workspace=ws, snapshot_pool=pool,
+                        snapshot_slot_base=base, snapshot_every=every)
+
+        for _ in range(max(3, args.warmup)):
+            flush.zero_()
+            snap_step()
+        if kda.workspace_status(ws) != 0:
+            raise RuntimeError("device status not OK with snapshots")
+        sn_ms = []
+        for _ in range(args.steps):
+            flush.zero_()
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            snap_step()
+            a1.record(stream)
+            sn_ms.append((a0, a1))
+        torch.cuda.synchronize()
+        sn_total = max_over_ranks(sum(a.elapsed_time(b) for a, b in sn_ms), world)
+        snap = {"every_tokens": every, "snapshots_per_step": sum(counts) * H,
+                "pool_bytes_written_per_step": sum(counts) * H * Dk * Dv * 4,
+                "value": world * T * args.steps / (sn_total * 1e-3), "unit": "tokens/s",
+                "ms_per_step": sn_total / args.steps,
+                "overhead_vs_plain": sn_total / total_ms - 1.0}
+
     # ---- decode workload: 64 recurrent steps ------------------------------
     dec = None
     if not args.no_decode:
@@ -398,6 +433,7 @@ def bench_kda(args):
             "roofline": roof,
             "cpu_baseline": cpu,
             "decode": dec,
+            "snapshots": snap,
             "clocks": clk.summary(),
         }
         print(json.dumps(line), flush=True)
@@ -456,6 +492,7 @@ def main(argv=None):
     ap.add_argument("--ref-tokens", type=int, default=512,
                     help="reference arm: tokens per sequence in each timed step")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-snapshots", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3:

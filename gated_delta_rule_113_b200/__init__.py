@@ -21,8 +21,9 @@ __all__ = ["forward", "decode_step", "forward_workspace_size", "workspace_status
            "KDAError", "load_library", "LIB_PATH", "EXPORTED_SYMBOLS"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkda.so")
-EXPORTED_SYMBOLS = ("kda_forward_workspace_size", "kda_forward", "kda_decode_step",
-                    "kda_workspace_status", "kda_status_string", "kda_abi_version")
+EXPORTED_SYMBOLS = ("kda_forward_workspace_size", "kda_forward", "kda_forward_snapshots",
+                    "kda_forward_noalloc", "kda_decode_step", "kda_workspace_status",
+                    "kda_status_string", "kda_abi_version")
 
 KDA_F32, KDA_BF16 = 0, 1
 FLAG_FORCE_SIMT = 1
@@ -35,6 +36,12 @@ _lib = None
 
 class KDAError(RuntimeError):
     pass
+
+
+class Snapshots(ctypes.Structure):
+    _fields_ = [("pool", ctypes.c_void_p), ("slot_base", ctypes.c_void_p),
+                ("s0_slot", ctypes.c_void_p), ("n_slots", ctypes.c_int64),
+                ("every", ctypes.c_int32)]
 
 
 class Params(ctypes.Structure):
@@ -62,6 +69,9 @@ def load_library(path: str = LIB_PATH):
         lib.kda_forward_workspace_size.argtypes = [pp]
         lib.kda_forward.restype = ctypes.c_int
         lib.kda_forward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, pp, vp, sz, vp]
+        lib.kda_forward_snapshots.restype = ctypes.c_int
+        lib.kda_forward_snapshots.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, pp,
+                                              ctypes.POINTER(Snapshots), vp, sz, vp]
         lib.kda_decode_step.restype = ctypes.c_int
         lib.kda_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, pp, vp]
         lib.kda_workspace_status.restype = ctypes.c_int
@@ -115,14 +125,21 @@ def forward_workspace_size(N: int, T: int, H: int, Dk: int, Dv: int,
 
 
 def forward(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, *, out=None, S_final=None,
-            workspace=None, output_final_state=True, force_simt=False, fused_tc=False):
-    """Chunked KDA prefill through ``kda_forward``.
+            workspace=None, output_final_state=True, force_simt=False, fused_tc=False,
+            snapshot_pool=None, snapshot_slot_base=None, snapshot_every=0, s0_slots=None):
+    """Chunked KDA prefill through ``kda_forward`` (``kda_forward_snapshots``
+    when a snapshot pool is given).
 
     q, k, log_alpha [T, H, Dk]; v [T, H, Dv]; beta [T, H]; S0 [N, H, Dk, Dv]
     fp32 or None; cu_seqlens int32 [N+1] on the device (None: one sequence).
     Returns (out [T, H, Dv] in q's dtype, S_final [N, H, Dk, Dv] fp32 or None).
     ``force_simt`` / ``fused_tc`` select the CUDA-core or the single-kernel
     tensor-core prefill instead of the default (for cross-checks).
+
+    Prefix-cache snapshots: ``snapshot_pool`` fp32 [n_slots, H, Dk, Dv];
+    every ``snapshot_every`` tokens of sequence n the state goes to slot
+    ``snapshot_slot_base[n]`` + m (int32 [N]); ``s0_slots`` (int32 [N]) starts
+    sequences from pool slots (negative: from S0).
     """
     lib = load_library()
     dev = q.device
@@ -150,11 +167,27 @@ def forward(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, *, out=None, S_f
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
     _require(dict(q=q, k=k, v=v, log_alpha=log_alpha, beta=beta, S0=S0, cu_seqlens=cu_seqlens,
-                  out=out, S_final=S_final, workspace=workspace), dev)
+                  out=out, S_final=S_final, workspace=workspace, snapshot_pool=snapshot_pool,
+                  snapshot_slot_base=snapshot_slot_base, s0_slots=s0_slots), dev)
+    if snapshot_pool is None:
+        with torch.cuda.device(dev):
+            _check(lib.kda_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+                                   _ptr(S0), _ptr(cu_seqlens), _ptr(out), _ptr(S_final),
+                                   ctypes.byref(p), _ptr(workspace), workspace.numel(),
+                                   _stream(dev)))
+        return out, S_final
+    if snapshot_pool.dtype != torch.float32 or tuple(snapshot_pool.shape[1:]) != (H, Dk, Dv):
+        raise KDAError("snapshot_pool must be float32 [n_slots, H, Dk, Dv]")
+    for name, t in (("snapshot_slot_base", snapshot_slot_base), ("s0_slots", s0_slots)):
+        if t is not None and (t.dtype != torch.int32 or t.numel() != N):
+            raise KDAError(f"{name} must be int32 [N]")
+    snap = Snapshots(_ptr(snapshot_pool), _ptr(snapshot_slot_base), _ptr(s0_slots),
+                     int(snapshot_pool.shape[0]), int(snapshot_every))
     with torch.cuda.device(dev):
-        _check(lib.kda_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0),
-                               _ptr(cu_seqlens), _ptr(out), _ptr(S_final), ctypes.byref(p),
-                               _ptr(workspace), workspace.numel(), _stream(dev)))
+        _check(lib.kda_forward_snapshots(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+                                         _ptr(S0), _ptr(cu_seqlens), _ptr(out), _ptr(S_final),
+                                         ctypes.byref(p), ctypes.byref(snap), _ptr(workspace),
+                                         workspace.numel(), _stream(dev)))
     return out, S_final
 
 

@@ -84,6 +84,7 @@ const char *kda_status_string(kda_status s) {
     case KDA_ERR_CUDA: return "KDA_ERR_CUDA: CUDA call or launch failed";
     case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT: bounded device wait gave up";
     case KDA_ERR_SEQLENS: return "KDA_ERR_SEQLENS: cu_seqlens not monotone from 0 to total_tokens";
+    case KDA_ERR_SLOT: return "KDA_ERR_SLOT: snapshot-pool slot outside the pool";
     }
     return "KDA_ERR_UNKNOWN";
 }
@@ -96,10 +97,12 @@ size_t kda_forward_workspace_size(const kda_params *p) {
     return workspace_bytes(p);
 }
 
-kda_status kda_forward(const void *q, const void *k, const void *v, const void *log_alpha,
-                       const void *beta, const float *S0, const int32_t *cu_seqlens, void *out,
-                       float *S_final, const kda_params *p, void *workspace, size_t ws_bytes,
-                       void *stream) {
+namespace {
+
+kda_status forward_impl(const void *q, const void *k, const void *v, const void *log_alpha,
+                        const void *beta, const float *S0, const int32_t *cu_seqlens, void *out,
+                        float *S_final, const kda_params *p, const kda_snapshots *snap,
+                        void *workspace, size_t ws_bytes, void *stream) {
     kda_status st = check_common(p);
     if (st != KDA_OK) return st;
     if (p->chunk != kda::kChunk || p->total_tokens < 0) return KDA_ERR_UNSUPPORTED;
@@ -107,14 +110,25 @@ kda_status kda_forward(const void *q, const void *k, const void *v, const void *
     if (!cu_seqlens) return KDA_ERR_INVALID;
     if (p->total_tokens > 0 && (!q || !k || !v || !log_alpha || !beta || !out))
         return KDA_ERR_INVALID;
-    const void *ptrs[] = {q, k, v, log_alpha, beta, S0, cu_seqlens, out, S_final, workspace};
-    for (const void *x : ptrs)
-        if (x && !aligned16(x)) return KDA_ERR_ALIGN;
+    // snapshots: `every` a multiple of the chunk; pool and slot arrays present
+    const bool use_snap = snap && (snap->every != 0 || snap->s0_slot);
+    if (use_snap) {
+        if (snap->every < 0 || snap->every % kda::kChunk) return KDA_ERR_INVALID;
+        if (!snap->pool || snap->n_slots <= 0) return KDA_ERR_INVALID;
+        if (snap->every > 0 && !snap->slot_base) return KDA_ERR_INVALID;
+        if (!aligned16(snap->pool)) return KDA_ERR_ALIGN;
+    }
+    const void *ptrs[] = {q, k, v, log_alpha, beta, S0, cu_seqlens, out, S_final, workspace,
+                          use_snap ? snap->pool : nullptr,
+                          use_snap ? snap->slot_base : nullptr,
+                          use_snap ? snap->s0_slot : nullptr};
+    for (int i = 0; i < 10; ++i)
+        if (ptrs[i] && !aligned16(ptrs[i])) return KDA_ERR_ALIGN;
     if (!workspace || ((uintptr_t)workspace & 255u) || ws_bytes < workspace_bytes(p))
         return KDA_ERR_WORKSPACE;
     // grid = N * H * (Dv / 32) CTAs must fit in gridDim.x
     if ((long long)p->num_seqs * p->H * (p->Dv / 32) > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
-    st = select_device(ptrs, 10);
+    st = select_device(ptrs, 13);
     if (st != KDA_OK) return st;
 
     kda::ForwardArgs a;
@@ -128,12 +142,18 @@ kda_status kda_forward(const void *q, const void *k, const void *v, const void *
     a.chunk_off = nullptr;
     a.packets = nullptr;
     a.packet_slots = 0;
+    a.snap_pool = use_snap ? snap->pool : nullptr;
+    a.snap_base = use_snap && snap->every > 0 ? snap->slot_base : nullptr;
+    a.s0_slot = use_snap ? snap->s0_slot : nullptr;
+    a.snap_slots = use_snap ? (long long)snap->n_slots : 0;
+    a.snap_every_chunks = use_snap ? snap->every / kda::kChunk : 0;
 
     // bf16 with Dk = Dv = 128: tensor cores, two-pass when the workspace holds
     // the operand packets, else the single fused kernel; otherwise CUDA cores.
     const bool tc = !(p->flags & KDA_FLAG_FORCE_SIMT) && kda::prefill_tc_supported(a);
     const bool two_pass =
         tc && !(p->flags & KDA_FLAG_FUSED_TC) && ws_bytes >= workspace_bytes_two_pass(p);
+    if (use_snap && !two_pass) return KDA_ERR_UNSUPPORTED;   // only the chain pass keeps them
     if (two_pass) {
         char *ws = static_cast<char *>(workspace);
         a.chunk_off = reinterpret_cast<int32_t *>(ws + chunk_off_offset(p));
@@ -148,6 +168,25 @@ kda_status kda_forward(const void *q, const void *k, const void *v, const void *
     else e = kda::launch_prefill_simt(a, s);
     if (e != cudaSuccess) return KDA_ERR_CUDA;
     return KDA_OK;
+}
+
+}  // namespace
+
+kda_status kda_forward(const void *q, const void *k, const void *v, const void *log_alpha,
+                       const void *beta, const float *S0, const int32_t *cu_seqlens, void *out,
+                       float *S_final, const kda_params *p, void *workspace, size_t ws_bytes,
+                       void *stream) {
+    return forward_impl(q, k, v, log_alpha, beta, S0, cu_seqlens, out, S_final, p, nullptr,
+                        workspace, ws_bytes, stream);
+}
+
+kda_status kda_forward_snapshots(const void *q, const void *k, const void *v,
+                                 const void *log_alpha, const void *beta, const float *S0,
+                                 const int32_t *cu_seqlens, void *out, float *S_final,
+                                 const kda_params *p, const kda_snapshots *snap, void *workspace,
+                                 size_t ws_bytes, void *stream) {
+    return forward_impl(q, k, v, log_alpha, beta, S0, cu_seqlens, out, S_final, p, snap,
+                        workspace, ws_bytes, stream);
 }
 
 kda_status kda_decode_step(const void *q, const void *k, const void *v, const void *log_alpha,

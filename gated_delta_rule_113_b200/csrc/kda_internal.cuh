@@ -29,6 +29,12 @@ struct ForwardArgs {
     int32_t *chunk_off;    // device [N+1] exclusive prefix of per-sequence chunk counts, or null
     unsigned char *packets;  // device per-(chunk, head) key-side operand packets, or null
     size_t packet_slots;     // number of packets the workspace holds
+    // state snapshots (two-pass path only): pool [n_slots, H, Dk, Dv] fp32
+    float *snap_pool;
+    const int32_t *snap_base;   // [N] first slot per sequence, negative: none
+    const int32_t *s0_slot;     // [N] start slot per sequence, negative: S0; or null
+    long long snap_slots;
+    int snap_every_chunks;      // 0: no snapshots
 };
 
 struct DecodeArgs {

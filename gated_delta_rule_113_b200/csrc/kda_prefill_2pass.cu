@@ -610,6 +610,11 @@ struct ChParams {
     float *Sf;
     const int32_t *order;
     int32_t *status;
+    float *snap_pool;            // [snap_slots, H, Dk, Dv] fp32, or null
+    const int32_t *snap_base;    // [N] first snapshot slot per sequence, or null
+    const int32_t *s0_slot;      // [N] start slot per sequence, or null
+    long long snap_slots;
+    int snap_every;              // chunks between snapshots; 0: none
     int N, T, H;
 };
 
@@ -776,6 +781,16 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
         float S[VS];
         {
             const float *src = p.S0 ? p.S0 + sbase_g + (size_t)c * kDV : nullptr;
+            if (p.s0_slot) {   // resume from a pool slot (prefix-cache hit)
+                const long long slot = p.s0_slot[seq];
+                if (slot >= p.snap_slots) {
+                    if (c == 0) set_status(p.status, KDA_ERR_SLOT);
+                    src = nullptr;
+                } else if (slot >= 0) {
+                    src = p.snap_pool + ((size_t)slot * p.H + h) * kDK * kDV + (size_t)vs * VS +
+                          (size_t)c * kDV;
+                }
+            }
 #pragma unroll
             for (int jj = 0; jj < VS; jj += 4) {
                 float4 v = src ? *reinterpret_cast<const float4 *>(src + jj) : make_float4(0, 0, 0, 0);
@@ -784,6 +799,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
         }
         float gl_cur = 1.f;
         bool ok = true;
+        const long long snap_base = (p.snap_every > 0 && p.snap_base) ? p.snap_base[seq] : -1;
         for (int j = 0; j <= nchunks && ok; ++j) {
             if (j > 0) {
                 // S <- Diag(Gam_L) (S + dS) for chunk j-1
@@ -797,6 +813,20 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
                     tmem_wait_ld();
 #pragma unroll
                     for (int e = 0; e < 32; ++e) S[jj + e] = gl_cur * (S[jj + e] + __uint_as_float(v[e]));
+                }
+                // snapshot: the state after j full chunks, every snap_every chunks
+                if (snap_base >= 0 && j % p.snap_every == 0 && j * kChunk <= t1 - t0) {
+                    const long long slot = snap_base + j / p.snap_every - 1;
+                    if (slot < p.snap_slots) {
+                        float *dst = p.snap_pool + ((size_t)slot * p.H + h) * kDK * kDV +
+                                     (size_t)c * kDV + (size_t)vs * VS;
+#pragma unroll
+                        for (int jj = 0; jj < VS; jj += 4)
+                            *reinterpret_cast<float4 *>(dst + jj) =
+                                make_float4(S[jj], S[jj + 1], S[jj + 2], S[jj + 3]);
+                    } else if (c == 0) {
+                        set_status(p.status, KDA_ERR_SLOT);
+                    }
                 }
             }
             if (j == nchunks) break;
@@ -939,6 +969,11 @@ cudaError_t launch_prefill_two_pass(const ForwardArgs &a, cudaStream_t s) {
     cp.Sf = a.S_final;
     cp.order = a.order;
     cp.status = a.status;
+    cp.snap_pool = a.snap_pool;
+    cp.snap_base = a.snap_base;
+    cp.s0_slot = a.s0_slot;
+    cp.snap_slots = a.snap_slots;
+    cp.snap_every = a.snap_every_chunks;
     cp.N = a.N;
     cp.T = a.T;
     cp.H = a.H;

@@ -44,7 +44,7 @@
 extern "C" {
 #endif
 
-#define KDA_ABI_VERSION 1
+#define KDA_ABI_VERSION 2
 
 typedef enum kda_status {
     KDA_OK = 0,
@@ -54,7 +54,8 @@ typedef enum kda_status {
     KDA_ERR_WORKSPACE = 4,    /* workspace NULL, misaligned or too small          */
     KDA_ERR_CUDA = 5,         /* a CUDA runtime call or kernel launch failed      */
     KDA_ERR_TIMEOUT = 6,      /* a bounded device-side wait gave up               */
-    KDA_ERR_SEQLENS = 7       /* device saw cu_seqlens not 0..total_tokens monotone */
+    KDA_ERR_SEQLENS = 7,      /* device saw cu_seqlens not 0..total_tokens monotone */
+    KDA_ERR_SLOT = 8          /* device saw a snapshot-pool slot outside the pool */
 } kda_status;
 
 typedef enum kda_dtype {
@@ -165,6 +166,55 @@ kda_status kda_forward_noalloc(const void *q, const void *k, const void *v,
                                const float *S0, const int32_t *cu_seqlens,
                                void *out, float *S_final, const kda_params *p,
                                void *stream);
+
+/*
+ * kda_forward_snapshots -- kda_forward that also keeps the recurrent state in
+ * a paged pool for prefix caching, and may start sequences from it.
+ *
+ * The page "Kimi K3: Open Frontier Intelligence and Implementation Framework",
+ * section "Inference Serving", bullet "KDA-Aware Prefix Caching", keeps KDA
+ * recurrent states in one paged pool so that a cached prefix can be resumed
+ * at 512-token boundaries.  Here a snapshot is the fp32 state of a (sequence,
+ * head) chain right after token number m * every of its sequence
+ * (m = 1 .. floor(len / every)), the same state a call on just that prefix
+ * would return as S_final.
+ *
+ *   pool       [n_slots, H, Dk, Dv] fp32, device.  Snapshot m-1 of sequence
+ *              n (all heads) is written to slot slot_base[n] + m - 1.
+ *   slot_base  [N] int32, device: first slot of each sequence's snapshots;
+ *              negative = record none for that sequence.  May be NULL when
+ *              every == 0.
+ *   s0_slot    [N] int32, device, or NULL: sequence n starts from the state
+ *              in slot s0_slot[n] instead of S0[n] (negative = use S0[n], or
+ *              zero when S0 is NULL).
+ *   every      tokens between snapshots: 0 (none) or a positive multiple of
+ *              the chunk (64); the page's granularity is 512.
+ *
+ * Slots read through s0_slot must not be written by the same call.  A slot
+ * outside [0, n_slots) is skipped on the device (nothing read or written;
+ * a start slot out of range starts from zero) and KDA_ERR_SLOT is recorded
+ * in the workspace status word.
+ *
+ * Only the two-pass tensor-core prefill keeps snapshots: bf16 q/k/v and
+ * gates with Dk = Dv = 128 and ws_bytes >= kda_forward_workspace_size(p).
+ * Other problems return KDA_ERR_UNSUPPORTED before anything is enqueued
+ * (snap == NULL, or every == 0 with s0_slot == NULL, is plain kda_forward).
+ * Other arguments and errors are those of kda_forward.
+ */
+typedef struct kda_snapshots {
+    float *pool;
+    const int32_t *slot_base;
+    const int32_t *s0_slot;
+    int64_t n_slots;
+    int32_t every;
+} kda_snapshots;
+
+kda_status kda_forward_snapshots(const void *q, const void *k, const void *v,
+                                 const void *log_alpha, const void *beta,
+                                 const float *S0, const int32_t *cu_seqlens,
+                                 void *out, float *S_final, const kda_params *p,
+                                 const kda_snapshots *snap,
+                                 void *workspace, size_t ws_bytes, void *stream);
 
 /*
  * kda_decode_step -- one recurrent token for N independent sequences.

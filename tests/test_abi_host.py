@@ -29,12 +29,12 @@ def test_library_loads_and_exports_every_declared_symbol():
     for name in declared:
         assert hasattr(lib, name), f"{name} declared in include/ but not exported"
     assert set(kda.EXPORTED_SYMBOLS) <= set(declared)
-    assert lib.kda_abi_version() == 1
+    assert lib.kda_abi_version() == 2
 
 
 def test_status_strings():
     lib = kda.load_library()
-    for code in range(0, 8):
+    for code in range(0, 9):
         assert lib.kda_status_string(code).startswith(b"KDA_")
     assert lib.kda_status_string(1234) == b"KDA_ERR_UNKNOWN"
 
@@ -111,3 +111,31 @@ def test_workspace_status_null_args():
     lib = kda.load_library()
     st = ctypes.c_int32(0)
     assert lib.kda_workspace_status(None, ctypes.byref(st), None) == 1
+
+
+def _fwd_snap(lib, p, every=512, pool=FAKE, base=FAKE, s0=None, n_slots=8, **over):
+    args = dict(q=FAKE, k=FAKE, v=FAKE, la=FAKE, beta=FAKE, S0=None, cu=FAKE, out=FAKE,
+                Sf=None, ws=0x20000, ws_bytes=1 << 20)
+    args.update(over)
+    vp = ctypes.c_void_p
+    snap = kda.Snapshots(vp(pool) if pool else None, vp(base) if base else None,
+                         vp(s0) if s0 else None, n_slots, every)
+    return lib.kda_forward_snapshots(vp(args["q"]), vp(args["k"]), vp(args["v"]), vp(args["la"]),
+                                     vp(args["beta"]), vp(args["S0"]), vp(args["cu"]),
+                                     vp(args["out"]), vp(args["Sf"]), ctypes.byref(p),
+                                     ctypes.byref(snap), vp(args["ws"]), args["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(every=100), 1),            # not a multiple of the chunk
+    (dict(every=-64), 1),
+    (dict(pool=None), 1),
+    (dict(base=None), 1),            # snapshots requested without slot bases
+    (dict(n_slots=0), 1),
+    (dict(every=0, s0=FAKE, pool=None), 1),
+    (dict(pool=FAKE + 4), 3),        # pool not 16-byte aligned
+    (dict(q=None), 1),               # the forward's own checks still apply
+])
+def test_forward_snapshots_host_validation(kw, code):
+    lib = kda.load_library()
+    assert _fwd_snap(lib, _params(), **kw) == code

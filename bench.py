@@ -477,7 +477,42 @@ def bench_decode(kda, dev, stream, world, args):
                          "frac": gbs / peaks["hbm_gbs"], "frac_of_8TBs_nominal": gbs / 8000.0,
                          "traffic": traffic_record("kda_decode"), "algorithmic_bytes": b,
                          "peak_kind": f"{kind} HBM copy"},
-            "state": "512 MiB fp32, larger than L2: no flush needed"}
+            "state": "512 MiB fp32, larger than L2: no flush needed",
+            "multi_token": bench_decode_multi(kda, dev, stream, world, x, S, w, peaks, kind)}
+
+
+def bench_decode_multi(kda, dev, stream, world, x, S, w, peaks, kind, n=4):
+    """Verify step of speculative decoding: n draft tokens per sequence in one
+    pass over the state, the state after every token kept (kda_decode_multi)."""
+    N, H, Dk, Dv = S.shape
+    m = {k: x[k][:n].transpose(0, 1).contiguous() for k in ("q", "k", "v", "log_alpha", "beta")}
+    out = torch.empty((N, n, H, Dv), dtype=w.torch_dtype, device=dev)
+    S_tok = torch.empty((N, n, H, Dk, Dv), dtype=torch.float32, device=dev)
+
+    def call():
+        kda.decode_multi(m["q"], m["k"], m["v"], m["log_alpha"], m["beta"], S, S_tokens=S_tok,
+                         out=out)
+
+    for _ in range(3):
+        call()
+    barrier(world)
+    reps = 20
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        call()
+    e1.record(stream)
+    barrier(world)
+    ms = max_over_ranks(e0.elapsed_time(e1), world) / reps
+    esz = 2 if w.torch_dtype == torch.bfloat16 else 4
+    # state read once, n states written, n tokens of q, k, v, log_alpha, beta, out
+    b = N * H * (Dk * Dv * 4 * (1 + n) + n * esz * (3 * Dk + 2 * Dv + 1))
+    gbs = b / (ms * 1e-3) / 1e9
+    return {"draft_tokens": n, "value": world * N * n / (ms * 1e-3), "unit": "tokens/s",
+            "us_per_call": ms * 1e3, "algorithmic_bytes": b,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm_gbs"], "peak_kind": f"{kind} HBM copy"},
+            "state": "S read once, the state after each draft token written (2.5 GiB per call)"}
 
 
 def main(argv=None):

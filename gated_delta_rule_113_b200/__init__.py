@@ -17,12 +17,13 @@ import threading
 
 import torch
 
-__all__ = ["forward", "decode_step", "forward_workspace_size", "workspace_status",
+__all__ = ["decode_multi", "forward", "decode_step", "forward_workspace_size", "workspace_status",
            "KDAError", "load_library", "LIB_PATH", "EXPORTED_SYMBOLS"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkda.so")
 EXPORTED_SYMBOLS = ("kda_forward_workspace_size", "kda_forward", "kda_forward_snapshots",
-                    "kda_forward_noalloc", "kda_decode_step", "kda_workspace_status",
+                    "kda_forward_noalloc", "kda_decode_step", "kda_decode_multi",
+                    "kda_workspace_status",
                     "kda_status_string", "kda_abi_version")
 
 KDA_F32, KDA_BF16 = 0, 1
@@ -74,6 +75,8 @@ def load_library(path: str = LIB_PATH):
                                               ctypes.POINTER(Snapshots), vp, sz, vp]
         lib.kda_decode_step.restype = ctypes.c_int
         lib.kda_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, pp, vp]
+        lib.kda_decode_multi.restype = ctypes.c_int
+        lib.kda_decode_multi.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, pp, ctypes.c_int32, vp]
         lib.kda_workspace_status.restype = ctypes.c_int
         lib.kda_workspace_status.argtypes = [vp, i32p, vp]
         lib.kda_status_string.restype = ctypes.c_char_p
@@ -224,3 +227,35 @@ def decode_step(q, k, v, log_alpha, beta, S, *, out=None):
         _check(lib.kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
                                    _ptr(S), _ptr(out), ctypes.byref(p), _stream(dev)))
     return out
+
+
+def decode_multi(q, k, v, log_alpha, beta, S, *, S_tokens=None, out=None):
+    """Several consecutive KDA tokens per sequence through ``kda_decode_multi``.
+
+    q, k, log_alpha [N, n, H, Dk]; v [N, n, H, Dv]; beta [N, n, H];
+    S [N, H, Dk, Dv] fp32 (read only).  Returns (out [N, n, H, Dv] in q's
+    dtype, S_tokens [N, n, H, Dk, Dv] fp32: the state after every token).
+    """
+    lib = load_library()
+    dev = q.device
+    N, n, H, Dk = q.shape
+    Dv = v.shape[-1]
+    if S.dtype != torch.float32 or S.shape != (N, H, Dk, Dv):
+        raise KDAError("S must be float32 [N, H, Dk, Dv]")
+    if k.shape != q.shape or log_alpha.shape != q.shape or v.shape[:3] != (N, n, H) \
+            or beta.shape != (N, n, H):
+        raise KDAError("shape mismatch among q, k, v, log_alpha, beta")
+    if k.dtype != q.dtype or v.dtype != q.dtype or beta.dtype != log_alpha.dtype:
+        raise KDAError("q, k, v must share a dtype; log_alpha and beta must share a dtype")
+    if out is None:
+        out = torch.empty((N, n, H, Dv), dtype=q.dtype, device=dev)
+    if S_tokens is None:
+        S_tokens = torch.empty((N, n, H, Dk, Dv), dtype=torch.float32, device=dev)
+    _require(dict(q=q, k=k, v=v, log_alpha=log_alpha, beta=beta, S=S, S_tokens=S_tokens,
+                  out=out), dev)
+    p = Params(N, 0, H, Dk, Dv, CHUNK, _dt(q), _dt(log_alpha), 0)
+    with torch.cuda.device(dev):
+        _check(lib.kda_decode_multi(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+                                    _ptr(S), _ptr(S_tokens), _ptr(out), ctypes.byref(p), int(n),
+                                    _stream(dev)))
+    return out, S_tokens

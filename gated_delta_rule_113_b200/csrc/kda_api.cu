@@ -205,6 +205,37 @@ kda_status kda_decode_step(const void *q, const void *k, const void *v, const vo
 
     kda::DecodeArgs a;
     a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta; a.S = S; a.out = out;
+    a.S_tokens = nullptr;
+    a.n_tokens = 1;
+    a.N = p->num_seqs; a.H = p->H; a.Dk = p->Dk; a.Dv = p->Dv;
+    a.io_dtype = p->io_dtype; a.gate_dtype = p->gate_dtype;
+    if (kda::launch_decode(a, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    return KDA_OK;
+}
+
+kda_status kda_decode_multi(const void *q, const void *k, const void *v, const void *log_alpha,
+                            const void *beta, const float *S, float *S_tokens, void *out,
+                            const kda_params *p, int32_t n_tokens, void *stream) {
+    kda_status st = check_common(p);
+    if (st != KDA_OK) return st;
+    if (n_tokens < 1) return KDA_ERR_INVALID;
+    if (p->num_seqs == 0) return KDA_OK;
+    if (!q || !k || !v || !log_alpha || !beta || !S || !S_tokens || !out) return KDA_ERR_INVALID;
+    const void *ptrs[] = {q, k, v, log_alpha, beta, S, S_tokens, out};
+    for (const void *x : ptrs)
+        if (!aligned16(x)) return KDA_ERR_ALIGN;
+    if ((long long)p->num_seqs * p->H * (p->Dv / 64) > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+    if ((long long)p->num_seqs * n_tokens > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+    st = select_device(ptrs, 8);
+    if (st != KDA_OK) return st;
+
+    kda::DecodeArgs a;
+    a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta;
+    a.S = const_cast<float *>(S);   // only read when S_tokens is set
+    a.S_tokens = S_tokens;
+    a.n_tokens = n_tokens;
+    a.out = out;
     a.N = p->num_seqs; a.H = p->H; a.Dk = p->Dk; a.Dv = p->Dv;
     a.io_dtype = p->io_dtype; a.gate_dtype = p->gate_dtype;
     if (kda::launch_decode(a, static_cast<cudaStream_t>(stream)) != cudaSuccess)

@@ -1,4 +1,7 @@
-// kda_decode.cu -- one recurrent KDA token for N independent sequences.
+// kda_decode.cu -- recurrent KDA tokens for N independent sequences: one
+// token per call (state updated in place), or several consecutive tokens per
+// sequence with the state read once and the state after every token kept
+// (for a verify step of speculative decoding that may roll back).
 //
 // Per (sequence, head) the step of the page "Kimi K3: Open Frontier
 // Intelligence and Implementation Framework" (section "Hybrid Attention
@@ -29,7 +32,7 @@ template <typename TIO, typename TG, int DK>
 __global__ void __launch_bounds__(kThreads)
 decode_kernel(const TIO *__restrict__ q, const TIO *__restrict__ k, const TIO *__restrict__ v,
               const TG *__restrict__ la, const TG *__restrict__ beta, float *__restrict__ S,
-              TIO *__restrict__ out, int H, int Dv) {
+              float *__restrict__ S_tokens, TIO *__restrict__ out, int H, int Dv, int n_tokens) {
     constexpr int RPT = DK / kRowGroups;  // rows per thread
     __shared__ float s_a[DK], s_ka[DK], s_qa[DK], s_k[DK];
     __shared__ float s_red[2][kRowGroups][kCols];
@@ -37,6 +40,7 @@ decode_kernel(const TIO *__restrict__ q, const TIO *__restrict__ k, const TIO *_
 
     const int slices = Dv / kCols;
     const int nh = blockIdx.x / slices;        // n * H + h
+    const int n = nh / H, h = nh % H;
     const int col0 = (blockIdx.x % slices) * kCols;
     const int tid = threadIdx.x;
     const int cg = tid % 16, rg = tid / 16;
@@ -48,72 +52,83 @@ decode_kernel(const TIO *__restrict__ q, const TIO *__restrict__ k, const TIO *_
     for (int i = 0; i < RPT; ++i)
         st[i] = *reinterpret_cast<const float4 *>(Sp + (size_t)(rg * RPT + i) * Dv);
 
-    const size_t vbase = (size_t)nh * DK;
-    for (int c = tid; c < DK; c += kThreads) {
-        const float a = expf(to_f32(la[vbase + c]));
-        const float kc = to_f32(k[vbase + c]);
-        s_a[c] = a;
-        s_k[c] = kc;
-        s_ka[c] = kc * a;
-        s_qa[c] = to_f32(q[vbase + c]) * a;
-    }
-    if (tid < 32) {
-        float p = 0.f;
-        for (int c = tid; c < DK; c += 32) p = fmaf(to_f32(q[vbase + c]), to_f32(k[vbase + c]), p);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
-        if (tid == 0) s_qk = p;
-    }
-    __syncthreads();
-
-    float yk[4] = {0.f, 0.f, 0.f, 0.f}, yq[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int i = 0; i < RPT; ++i) {
-        const int c = rg * RPT + i;
-        const float ka = s_ka[c], qa = s_qa[c];
-        yk[0] = fmaf(ka, st[i].x, yk[0]); yq[0] = fmaf(qa, st[i].x, yq[0]);
-        yk[1] = fmaf(ka, st[i].y, yk[1]); yq[1] = fmaf(qa, st[i].y, yq[1]);
-        yk[2] = fmaf(ka, st[i].z, yk[2]); yq[2] = fmaf(qa, st[i].z, yq[2]);
-        yk[3] = fmaf(ka, st[i].w, yk[3]); yq[3] = fmaf(qa, st[i].w, yq[3]);
-    }
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        s_red[0][rg][cg * 4 + j] = yk[j];
-        s_red[1][rg][cg * 4 + j] = yq[j];
-    }
-    __syncthreads();
-
-    const float b = to_f32(beta[nh]);
-    const float qk = s_qk;
-    float u[4], o[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        float sk = 0.f, sq = 0.f;
-#pragma unroll
-        for (int g = 0; g < kRowGroups; ++g) {
-            sk += s_red[0][g][cg * 4 + j];
-            sq += s_red[1][g][cg * 4 + j];
+    // Tokens of one sequence are consecutive rows of the token-major inputs;
+    // the state stays in registers from one token to the next.
+    for (int t = 0; t < n_tokens; ++t) {
+        const size_t row = ((size_t)n * n_tokens + t) * H + h;   // (n, t, h)
+        const size_t vbase = row * DK;
+        if (t > 0) __syncthreads();   // everyone is done with the previous token's vectors
+        for (int c = tid; c < DK; c += kThreads) {
+            const float a = expf(to_f32(la[vbase + c]));
+            const float kc = to_f32(k[vbase + c]);
+            s_a[c] = a;
+            s_k[c] = kc;
+            s_ka[c] = kc * a;
+            s_qa[c] = to_f32(q[vbase + c]) * a;
         }
-        const float vj = to_f32(v[(size_t)nh * Dv + col0 + cg * 4 + j]);
-        u[j] = b * (vj - sk);
-        o[j] = fmaf(qk, u[j], sq);
-    }
+        if (tid < 32) {
+            float p = 0.f;
+            for (int c = tid; c < DK; c += 32) p = fmaf(to_f32(q[vbase + c]), to_f32(k[vbase + c]), p);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
+            if (tid == 0) s_qk = p;
+        }
+        __syncthreads();
 
+        float yk[4] = {0.f, 0.f, 0.f, 0.f}, yq[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int i = 0; i < RPT; ++i) {
-        const int c = rg * RPT + i;
-        const float a = s_a[c], kc = s_k[c];
-        float4 w;
-        w.x = fmaf(a, st[i].x, kc * u[0]);
-        w.y = fmaf(a, st[i].y, kc * u[1]);
-        w.z = fmaf(a, st[i].z, kc * u[2]);
-        w.w = fmaf(a, st[i].w, kc * u[3]);
-        *reinterpret_cast<float4 *>(Sp + (size_t)c * Dv) = w;
-    }
-    if (rg == 0) {
-        TIO *op = out + (size_t)nh * Dv + col0 + cg * 4;
+        for (int i = 0; i < RPT; ++i) {
+            const int c = rg * RPT + i;
+            const float ka = s_ka[c], qa = s_qa[c];
+            yk[0] = fmaf(ka, st[i].x, yk[0]); yq[0] = fmaf(qa, st[i].x, yq[0]);
+            yk[1] = fmaf(ka, st[i].y, yk[1]); yq[1] = fmaf(qa, st[i].y, yq[1]);
+            yk[2] = fmaf(ka, st[i].z, yk[2]); yq[2] = fmaf(qa, st[i].z, yq[2]);
+            yk[3] = fmaf(ka, st[i].w, yk[3]); yq[3] = fmaf(qa, st[i].w, yq[3]);
+        }
 #pragma unroll
-        for (int j = 0; j < 4; ++j) op[j] = from_f32<TIO>(o[j]);
+        for (int j = 0; j < 4; ++j) {
+            s_red[0][rg][cg * 4 + j] = yk[j];
+            s_red[1][rg][cg * 4 + j] = yq[j];
+        }
+        __syncthreads();
+
+        const float b = to_f32(beta[row]);
+        const float qk = s_qk;
+        float u[4], o[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            float sk = 0.f, sq = 0.f;
+#pragma unroll
+            for (int g = 0; g < kRowGroups; ++g) {
+                sk += s_red[0][g][cg * 4 + j];
+                sq += s_red[1][g][cg * 4 + j];
+            }
+            const float vj = to_f32(v[row * Dv + col0 + cg * 4 + j]);
+            u[j] = b * (vj - sk);
+            o[j] = fmaf(qk, u[j], sq);
+        }
+
+        // the state after this token: in place for a single step, else into
+        // its own slot of S_tokens [N, n_tokens, H, Dk, Dv]
+        float *Sw = S_tokens ? S_tokens + row * DK * Dv + col0 + cg * 4 : Sp;
+#pragma unroll
+        for (int i = 0; i < RPT; ++i) {
+            const int c = rg * RPT + i;
+            const float a = s_a[c], kc = s_k[c];
+            float4 w;
+            w.x = fmaf(a, st[i].x, kc * u[0]);
+            w.y = fmaf(a, st[i].y, kc * u[1]);
+            w.z = fmaf(a, st[i].z, kc * u[2]);
+            w.w = fmaf(a, st[i].w, kc * u[3]);
+            st[i] = w;
+            if (S_tokens || t == n_tokens - 1)
+                *reinterpret_cast<float4 *>(Sw + (size_t)c * Dv) = w;
+        }
+        if (rg == 0) {
+            TIO *op = out + row * Dv + col0 + cg * 4;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) op[j] = from_f32<TIO>(o[j]);
+        }
     }
 }
 
@@ -122,7 +137,7 @@ cudaError_t launch_typed(const DecodeArgs &a, cudaStream_t s) {
     const unsigned grid = (unsigned)((size_t)a.N * a.H * (a.Dv / kCols));
     decode_kernel<TIO, TG, DK><<<grid, kThreads, 0, s>>>(
         (const TIO *)a.q, (const TIO *)a.k, (const TIO *)a.v, (const TG *)a.log_alpha,
-        (const TG *)a.beta, a.S, (TIO *)a.out, a.H, a.Dv);
+        (const TG *)a.beta, a.S, a.S_tokens, (TIO *)a.out, a.H, a.Dv, a.n_tokens);
     return cudaGetLastError();
 }
 

@@ -39,7 +39,9 @@ struct ForwardArgs {
 
 struct DecodeArgs {
     const void *q, *k, *v, *log_alpha, *beta;
-    float *S;
+    float *S;          // read; written in place when S_tokens is null
+    float *S_tokens;   // [N, n_tokens, H, Dk, Dv] state after every token, or null
+    int n_tokens;      // consecutive tokens per sequence (1 for a plain step)
     void *out;
     int N, H, Dk, Dv;
     int io_dtype, gate_dtype;

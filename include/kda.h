@@ -236,6 +236,32 @@ kda_status kda_decode_step(const void *q, const void *k, const void *v,
                            void *out, const kda_params *p, void *stream);
 
 /*
+ * kda_decode_multi -- n_tokens consecutive recurrent tokens per sequence in
+ * one pass over the state, keeping the state after every token: the verify
+ * step of speculative decoding, which accepts a prefix of draft tokens and
+ * resumes from the state after the last accepted one.  (The page "Kimi K3:
+ * Open Frontier Intelligence and Implementation Framework", section
+ * "Inference Serving", serves K3 with an EAGLE-3-style draft model.)
+ *
+ *   q, k, log_alpha [N, n_tokens, H, Dk]  (io_dtype for q/k, gate_dtype)
+ *   v               [N, n_tokens, H, Dv]  io_dtype
+ *   beta            [N, n_tokens, H]      gate_dtype
+ *   S               [N, H, Dk, Dv] fp32, read only (read once)
+ *   S_tokens        [N, n_tokens, H, Dk, Dv] fp32, written: S_tokens[n, t]
+ *                   is the state after token t of sequence n
+ *   out             [N, n_tokens, H, Dv] io_dtype, written
+ *
+ * Every token applies exactly the arithmetic of kda_decode_step, so the
+ * outputs and S_tokens[n, t] equal those of t + 1 successive single steps.
+ * S_tokens must not overlap S.  p->total_tokens and p->chunk are ignored.
+ * Errors: as kda_decode_step; n_tokens < 1 is KDA_ERR_INVALID.
+ */
+kda_status kda_decode_multi(const void *q, const void *k, const void *v,
+                            const void *log_alpha, const void *beta, const float *S,
+                            float *S_tokens, void *out, const kda_params *p,
+                            int32_t n_tokens, void *stream);
+
+/*
  * kda_workspace_status -- synchronise `stream`, then copy the device status
  * word of a kda_forward workspace into *status (KDA_OK when the last call
  * that used this workspace saw nothing wrong).  Returns KDA_ERR_INVALID for

@@ -139,3 +139,17 @@ def _fwd_snap(lib, p, every=512, pool=FAKE, base=FAKE, s0=None, n_slots=8, **ove
 def test_forward_snapshots_host_validation(kw, code):
     lib = kda.load_library()
     assert _fwd_snap(lib, _params(), **kw) == code
+
+
+def test_decode_multi_host_validation():
+    lib = kda.load_library()
+    vp = ctypes.c_void_p
+    call = lambda p, n=4, **o: lib.kda_decode_multi(*(vp(o.get(x, FAKE)) for x in
+                                                      ("q", "k", "v", "la", "b", "S", "St", "out")),
+                                                    ctypes.byref(p), n, None)
+    assert call(_params(), n=0) == 1
+    assert call(_params(), St=None) == 1
+    assert call(_params(), S=None) == 1
+    assert call(_params(), St=FAKE + 4) == 3
+    assert call(_params(Dk=32)) == 2
+    assert call(_params(num_seqs=0)) == 0

@@ -567,10 +567,9 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 // ============================================================ pass 2
 constexpr int kChWarps = 6;   // 0-3 chain, 4 loader, 5 MMA
 constexpr int kChThreads = kChWarps * 32;
-constexpr int kChStages = 3;
 enum ChRole { kChLoad = 4, kChMma = 5 };
 enum ChBars {
-    cbFull = 0,       // [3] packet + value tile landed
+    cbFull = 0,       // [3] packet + value tile landed (two used when VS = 64)
     cbStageFree = 3,  // [3] every product reading a stage done
     cbSbFull = 6,     // count 4: bf16 S written
     cbUFull = 7,      // D1 = [U; O] complete
@@ -589,7 +588,9 @@ struct ChLayout {
     static constexpr uint32_t kV = (kPkGL + 512 + 1023) / 1024 * 1024;
     static constexpr uint32_t kStage = (kV + 64 * VS * 2 + 1023) / 1024 * 1024;
     static_assert(kPkGL + 512 == kPacketBytes, "the packet is one contiguous copy");
-    static constexpr uint32_t kSB = kChStages * kStage;
+    // three stages fit beside the 32-wide operands, two beside the 64-wide ones
+    static constexpr int kStages = VS == 32 ? 3 : 2;
+    static constexpr uint32_t kSB = kStages * kStage;
     static constexpr uint32_t kUB = kSB + 128 * VS * 2;
     static constexpr uint32_t kBar = kUB + 64 * VS * 2;
     static constexpr uint32_t kMisc = kBar + 16 * 8;
@@ -597,7 +598,7 @@ struct ChLayout {
     static_assert(kAlloc <= 232448, "shared memory budget exceeded");
     static constexpr uint32_t kTmD1 = 0;          // + d * VS, d = chunk & 1
     static constexpr uint32_t kTmD2 = 2 * VS;
-    static constexpr uint32_t kTmCols = 128;
+    static constexpr uint32_t kTmCols = 4 * VS;   // D1[2], D2, rounded to a power of two
 };
 
 struct ChParams {
@@ -610,6 +611,7 @@ struct ChParams {
     float *Sf;
     const int32_t *order;
     int32_t *status;
+    const void *v_base;          // v [T, H, Dv], for the value tile map
     float *snap_pool;            // [snap_slots, H, Dk, Dv] fp32, or null
     const int32_t *snap_base;    // [N] first snapshot slot per sequence, or null
     const int32_t *s0_slot;      // [N] start slot per sequence, or null
@@ -687,10 +689,10 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
         // One copy for the packet (lane 0) and one for the value tile (lane
         // 1): copies from different threads are serviced concurrently.
         for (int j = 0; j < nchunks; ++j) {
-            const int s = j % kChStages;
+            const int s = j % Ly::kStages;
             bool ok = true;
-            if (lane == 0 && j >= kChStages)
-                ok = wait_or_abort(&bars[cbStageFree + s], (j / kChStages - 1) & 1, abort_flag, p.status);
+            if (lane == 0 && j >= Ly::kStages)
+                ok = wait_or_abort(&bars[cbStageFree + s], (j / Ly::kStages - 1) & 1, abort_flag, p.status);
             if (!__shfl_sync(0xffffffffu, ok, 0)) break;
             unsigned char *st = sm + s * Ly::kStage;
             uint64_t *full = &bars[cbFull + s];
@@ -702,19 +704,19 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
                 bulk_load(st + off, packet(j) + off, len, full);
             }
             if (lane == 4) tma_load_3d(st + Ly::kV, &tm_v, full, vs * VS, h, t0 + j * kChunk);
-            if (lane == 5 && j + kChStages < nchunks)
-                bulk_prefetch_l2(packet(j + kChStages), (uint32_t)kPacketBytes);
+            if (lane == 5 && j + Ly::kStages < nchunks)
+                bulk_prefetch_l2(packet(j + Ly::kStages), (uint32_t)kPacketBytes);
             if (lane == 0) KDA_TRACE2(j, 0);
 #ifdef KDA_TRACE
             if (lane == 6) {
-                mbar_wait(full, (j / kChStages) & 1);
+                mbar_wait(full, (j / Ly::kStages) & 1);
                 KDA_TRACE2(j, 11);
             }
 #endif
         }
         if (lane == 0)
-            for (int j = max(0, nchunks - kChStages); j < nchunks; ++j)
-                mbar_wait(&bars[cbFull + j % kChStages], (j / kChStages) & 1);
+            for (int j = max(0, nchunks - Ly::kStages); j < nchunks; ++j)
+                mbar_wait(&bars[cbFull + j % Ly::kStages], (j / Ly::kStages) & 1);
     } else if (warp == kChMma) {
         // ------------------------------------------------------ MMA issuer
         if (lane == 0) {
@@ -726,9 +728,9 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
             // chain warps turn the previous chunk's U into bf16, so it never
             // sits between the state and the product that consumes it.
             auto issue_u0 = [&](int j) -> bool {
-                const int s = j % kChStages, d = j & 1;
+                const int s = j % Ly::kStages, d = j & 1;
                 const uint32_t st = sbase + s * Ly::kStage;
-                if (!spin_or_abort(&bars[cbFull + s], (j / kChStages) & 1, abort_flag, p.status))
+                if (!spin_or_abort(&bars[cbFull + s], (j / Ly::kStages) & 1, abort_flag, p.status))
                     return false;
                 KDA_TRACE2(j, 12);
                 if (j >= 2 && !spin_or_abort(&bars[cbD1Free + d], ((j - 2) >> 1) & 1, abort_flag,
@@ -746,7 +748,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
             };
             bool ok = nchunks > 0 && issue_u0(0);
             for (int j = 0; j < nchunks && ok; ++j) {
-                const int s = j % kChStages, d = j & 1;
+                const int s = j % Ly::kStages, d = j & 1;
                 const uint32_t st = sbase + s * Ly::kStage;
                 const uint32_t d1 = tmem + Ly::kTmD1 + d * VS;
                 const uint64_t d_kq = smem_desc(st + Ly::kKQ, 16, 1024, kSw128);
@@ -830,8 +832,8 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
                 }
             }
             if (j == nchunks) break;
-            const int s = j % kChStages, d = j & 1;
-            if (!spin_or_abort(&bars[cbFull + s], (j / kChStages) & 1, abort_flag, p.status)) { ok = false; break; }
+            const int s = j % Ly::kStages, d = j & 1;
+            if (!spin_or_abort(&bars[cbFull + s], (j / Ly::kStages) & 1, abort_flag, p.status)) { ok = false; break; }
             gl_cur = reinterpret_cast<const float *>(sm + s * Ly::kStage + Ly::kGL)[c];
             if (c == 0) KDA_TRACE2(j, 7);
             {
@@ -931,16 +933,31 @@ int sm_count() {
 
 }  // namespace
 
+namespace {
+
+template <int VS>
+cudaError_t launch_chain(const ChParams &cp, int T, cudaStream_t s) {
+    CUtensorMap mv;
+    if (!make_tmap_bf16_3d(&mv, cp.v_base, T, cp.H, kDV, VS, VS * 2)) return cudaErrorInvalidValue;
+    auto kern = chain_kernel<VS>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)ChLayout<VS>::kAlloc);
+    if (e != cudaSuccess) return e;
+    const unsigned grid2 = (unsigned)cp.N * cp.H * (kDV / VS);
+    kern<<<grid2, kChThreads, ChLayout<VS>::kAlloc, s>>>(mv, cp);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
 cudaError_t launch_prefill_two_pass(const ForwardArgs &a, cudaStream_t s) {
-    constexpr int VS = 32;
     const int T = a.T > 0 ? a.T : 1;
-    CUtensorMap mq, mk, mla, mv;
+    CUtensorMap mq, mk, mla;
     if (!make_tmap_bf16_3d(&mq, a.q, T, a.H, kDK, 64, 128) ||
         !make_tmap_bf16_3d(&mk, a.k, T, a.H, kDK, 64, 128) ||
-        !make_tmap_bf16_3d(&mla, a.log_alpha, T, a.H, kDK, 64, 128) ||
-        !make_tmap_bf16_3d(&mv, a.v, T, a.H, kDV, VS, VS * 2))
+        !make_tmap_bf16_3d(&mla, a.log_alpha, T, a.H, kDK, 64, 128))
         return cudaErrorInvalidValue;
-    // pass 1: persistent, at most one CTA per SM, items strided over the grid
+    // pass 1: persistent, at most one CTA per SM, items claimed from a counter
     KsParams kp;
     kp.beta = static_cast<const __nv_bfloat16 *>(a.beta);
     kp.cu = a.cu_seqlens;
@@ -958,7 +975,6 @@ cudaError_t launch_prefill_two_pass(const ForwardArgs &a, cudaStream_t s) {
     const unsigned grid1 = (unsigned)(items < (size_t)sm_count() ? items : (size_t)sm_count());
     kside_kernel<<<grid1, kKsThreads, KsLayout::kAlloc, s>>>(mq, mk, mla, kp);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    // pass 2: one CTA per (sequence, head, value slice), longest sequences first
     ChParams cp;
     cp.S0 = a.S0;
     cp.cu = a.cu_seqlens;
@@ -977,13 +993,13 @@ cudaError_t launch_prefill_two_pass(const ForwardArgs &a, cudaStream_t s) {
     cp.N = a.N;
     cp.T = a.T;
     cp.H = a.H;
-    auto kern = chain_kernel<VS>;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)ChLayout<VS>::kAlloc);
-    if (e != cudaSuccess) return e;
-    const unsigned grid2 = (unsigned)a.N * a.H * (kDV / VS);
-    kern<<<grid2, kChThreads, ChLayout<VS>::kAlloc, s>>>(mv, cp);
-    return cudaGetLastError();
+    cp.v_base = a.v;
+    // pass 2: one CTA per (sequence, head, value slice), longest sequences
+    // first.  32-wide slices give
+    // the most parallel chains; once they would not fit on the GPU in one
+    // wave, 64-wide slices do twice the work per MMA instruction instead.
+    if ((long long)a.N * a.H * (kDV / 32) > sm_count()) return launch_chain<64>(cp, T, s);
+    return launch_chain<32>(cp, T, s);
 }
 
 }  // namespace kda

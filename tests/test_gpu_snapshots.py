@@ -44,11 +44,13 @@ def _workspace(inp):
                        dtype=torch.uint8, device="cuda")
 
 
-@pytest.mark.parametrize("every", [512, 128])
-def test_snapshots_match_oracle(every):
-    lengths = [1100, 600, 100, 1536, 0, 513]
-    inp = _inputs(lengths)
-    H = inp["q"].shape[1]
+@pytest.mark.parametrize("every,lengths,H", [
+    (512, [1100, 600, 100, 1536, 0, 513], 3),
+    (128, [1100, 600, 100, 1536, 0, 513], 3),
+    (512, [1100, 600], 80),          # enough chains for the 64-wide chain slices
+])
+def test_snapshots_match_oracle(every, lengths, H):
+    inp = _inputs(lengths, H=H)
     ro, rs, rsn, roff = _oracle_snaps(inp, every)
     n_snap = rsn.shape[0]
     shift = 3                               # slots need not start at 0

@@ -19,7 +19,8 @@ kda_status check_common(const kda_params *p) {
     if (p->num_seqs < 0 || p->H <= 0) return KDA_ERR_INVALID;
     if (!dtype_ok(p->io_dtype) || !dtype_ok(p->gate_dtype)) return KDA_ERR_UNSUPPORTED;
     if (!width_ok(p->Dk) || !width_ok(p->Dv)) return KDA_ERR_UNSUPPORTED;
-    if (p->flags & ~(KDA_FLAG_FORCE_SIMT | KDA_FLAG_FUSED_TC)) return KDA_ERR_INVALID;
+    if (p->flags & ~(KDA_FLAG_FORCE_SIMT | KDA_FLAG_FUSED_TC | KDA_FLAG_TEST_STALL))
+        return KDA_ERR_INVALID;
     return KDA_OK;
 }
 
@@ -147,6 +148,7 @@ kda_status forward_impl(const void *q, const void *k, const void *v, const void 
     a.s0_slot = use_snap ? snap->s0_slot : nullptr;
     a.snap_slots = use_snap ? (long long)snap->n_slots : 0;
     a.snap_every_chunks = use_snap ? snap->every / kda::kChunk : 0;
+    a.test_stall = (p->flags & KDA_FLAG_TEST_STALL) != 0;
 
     // bf16 with Dk = Dv = 128: tensor cores, two-pass when the workspace holds
     // the operand packets, else the single fused kernel; otherwise CUDA cores.

@@ -35,6 +35,7 @@ struct ForwardArgs {
     const int32_t *s0_slot;     // [N] start slot per sequence, negative: S0; or null
     long long snap_slots;
     int snap_every_chunks;      // 0: no snapshots
+    bool test_stall;            // chain pass waits on a barrier nobody arrives on
 };
 
 struct DecodeArgs {

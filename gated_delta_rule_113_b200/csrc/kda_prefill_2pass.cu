@@ -577,7 +577,8 @@ enum ChBars {
     cbDsFull = 9,     // dS = Ki^T U complete
     cbD1Free = 10,    // [2] count 2: O read out of D1[d]
     cbDrain = 12,
-    cbNum = 13
+    cbNever = 13,     // nothing arrives on it (failure-path check)
+    cbNum = 14
 };
 
 template <int VS>
@@ -617,6 +618,7 @@ struct ChParams {
     const int32_t *s0_slot;      // [N] start slot per sequence, or null
     long long snap_slots;
     int snap_every;              // chunks between snapshots; 0: none
+    int test_stall;              // MMA issuer first waits on cbNever
     int N, T, H;
 };
 
@@ -688,6 +690,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
         // ------------------------------------------------------- loader
         // One copy for the packet (lane 0) and one for the value tile (lane
         // 1): copies from different threads are serviced concurrently.
+        int n_issued = 0;
         for (int j = 0; j < nchunks; ++j) {
             const int s = j % Ly::kStages;
             bool ok = true;
@@ -706,6 +709,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
             if (lane == 4) tma_load_3d(st + Ly::kV, &tm_v, full, vs * VS, h, t0 + j * kChunk);
             if (lane == 5 && j + Ly::kStages < nchunks)
                 bulk_prefetch_l2(packet(j + Ly::kStages), (uint32_t)kPacketBytes);
+            n_issued = j + 1;
             if (lane == 0) KDA_TRACE2(j, 0);
 #ifdef KDA_TRACE
             if (lane == 6) {
@@ -714,8 +718,9 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
             }
 #endif
         }
+        // copies in flight must land before the CTA may exit
         if (lane == 0)
-            for (int j = max(0, nchunks - Ly::kStages); j < nchunks; ++j)
+            for (int j = max(0, n_issued - Ly::kStages); j < n_issued; ++j)
                 mbar_wait(&bars[cbFull + j % Ly::kStages], (j / Ly::kStages) & 1);
     } else if (warp == kChMma) {
         // ------------------------------------------------------ MMA issuer
@@ -746,7 +751,9 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
                              d_v + vs_step<VS>(ks), kIdV, ks > 0);
                 return true;
             };
-            bool ok = nchunks > 0 && issue_u0(0);
+            // failure-path check: a wait that can only run out of time
+            bool ok = !p.test_stall || spin_or_abort(&bars[cbNever], 0, abort_flag, p.status);
+            ok = ok && nchunks > 0 && issue_u0(0);
             for (int j = 0; j < nchunks && ok; ++j) {
                 const int s = j % Ly::kStages, d = j & 1;
                 const uint32_t st = sbase + s * Ly::kStage;
@@ -990,6 +997,7 @@ cudaError_t launch_prefill_two_pass(const ForwardArgs &a, cudaStream_t s) {
     cp.s0_slot = a.s0_slot;
     cp.snap_slots = a.snap_slots;
     cp.snap_every = a.snap_every_chunks;
+    cp.test_stall = a.test_stall ? 1 : 0;
     cp.N = a.N;
     cp.T = a.T;
     cp.H = a.H;

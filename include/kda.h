@@ -82,6 +82,13 @@ typedef struct kda_params {
 /* Use the single-kernel tensor-core prefill even when the workspace is large
  * enough for the two-pass one (for cross-checking the two). */
 #define KDA_FLAG_FUSED_TC 2
+/* Failure-path check: on the two-pass path the chain pass's MMA issuer waits
+ * on a barrier nothing arrives on.  The bounded wait gives up after about
+ * 2 s, every role of the CTA winds down (MMAs and copies drained, tensor
+ * memory freed), outputs are left incomplete and KDA_ERR_TIMEOUT is recorded
+ * in the workspace status; the CUDA context stays usable.  No fault, trap or
+ * unbounded wait is involved. */
+#define KDA_FLAG_TEST_STALL 4
 
 /*
  * kda_forward_workspace_size -- bytes of device workspace for the fastest

@@ -3,6 +3,7 @@ same seeded inputs.  Small cases compare every element; full-size workloads
 compare every output of sampled (sequence, head) chains, which the oracle
 computes exactly as it would inside the full problem (chains are
 independent)."""
+import ctypes
 import math
 
 import numpy as np
@@ -262,3 +263,30 @@ def test_decode_equals_prefill():
     torch.cuda.synchronize()
     assert rel_fro(as_np(dec_out.reshape(N * steps, H, -1)), as_np(p_out)) < 1e-2
     assert rel_fro(as_np(S), as_np(p_s)) < 1e-2
+
+
+def test_bounded_wait_times_out_and_the_context_stays_usable():
+    """KDA_FLAG_TEST_STALL makes the chain pass wait on a barrier nothing
+    arrives on: the wait gives up after its 2 s bound, the call records
+    KDA_ERR_TIMEOUT, and the next call on the same context is correct."""
+    import time
+    w = WORKLOADS[1]
+    inp = forward_inputs(w, lengths=[300, 129], H=2)
+    d = to_dev(inp)
+    ws = torch.empty(kda.forward_workspace_size(2, 429, 2, 128, 128), dtype=torch.uint8,
+                     device="cuda")
+    lib = kda.load_library()
+    out = torch.empty((429, 2, 128), dtype=torch.bfloat16, device="cuda")
+    sf = torch.empty((2, 2, 128, 128), dtype=torch.float32, device="cuda")
+    p = kda.Params(2, 429, 2, 128, 128, 64, 1, 1, 4)   # KDA_FLAG_TEST_STALL
+    t0 = time.time()
+    rc = lib.kda_forward(*(kda._ptr(x) for x in (d["q"], d["k"], d["v"], d["log_alpha"],
+                                                 d["beta"], d["S0"], d["cu_seqlens"], out, sf)),
+                         ctypes.byref(p), kda._ptr(ws), ws.numel(), kda._stream(out.device))
+    assert rc == 0
+    assert kda.workspace_status(ws) == 6             # KDA_ERR_TIMEOUT
+    assert time.time() - t0 < 20
+    out2, sf2 = kda.forward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["S0"],
+                            d["cu_seqlens"], workspace=ws)
+    assert kda.workspace_status(ws) == 0
+    _check(inp, out2, sf2, torch.bfloat16)

@@ -238,6 +238,11 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     float *sB = reinterpret_cast<float *>(sm + Ly::kB);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // Launched as a programmatic dependent of the varlen index: the chain
+    // pass may be scheduled onto SMs as this pass's CTAs finish, and the
+    // chunk offsets and item counter are read only after the index is done.
+    grid_launch_dependents();
+    grid_dependency_wait();
     long long total = (long long)p.chunk_off[p.N] * p.H;
     if (total > p.slots) {   // overlapping (malformed) sequences: never write past the workspace
         if (blockIdx.x == 0 && threadIdx.x == 0) set_status(p.status, KDA_ERR_SEQLENS);
@@ -643,6 +648,9 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + Ly::kMisc + 4);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // Launched as a programmatic dependent of the key-side pass: every
+    // packet (and the work order) is read only after that pass is done.
+    grid_dependency_wait();
     const int n_slices = kDV / VS;
     const int per_seq = p.H * n_slices;
     const int seq = p.order[blockIdx.x / per_seq];
@@ -942,6 +950,25 @@ int sm_count() {
 
 namespace {
 
+// Launch with programmatic stream serialisation: the kernel may start while
+// the previous kernel in the stream finishes (it waits for that kernel's
+// results itself, see grid_dependency_wait).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kern)(KArgs...), unsigned grid, unsigned block, size_t smem,
+                             cudaStream_t s, Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 template <int VS>
 cudaError_t launch_chain(const ChParams &cp, int T, cudaStream_t s) {
     CUtensorMap mv;
@@ -951,8 +978,7 @@ cudaError_t launch_chain(const ChParams &cp, int T, cudaStream_t s) {
                                          (int)ChLayout<VS>::kAlloc);
     if (e != cudaSuccess) return e;
     const unsigned grid2 = (unsigned)cp.N * cp.H * (kDV / VS);
-    kern<<<grid2, kChThreads, ChLayout<VS>::kAlloc, s>>>(mv, cp);
-    return cudaGetLastError();
+    return launch_dependent(kern, grid2, kChThreads, ChLayout<VS>::kAlloc, s, mv, cp);
 }
 
 }  // namespace
@@ -980,8 +1006,9 @@ cudaError_t launch_prefill_two_pass(const ForwardArgs &a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     const size_t items = a.packet_slots;
     const unsigned grid1 = (unsigned)(items < (size_t)sm_count() ? items : (size_t)sm_count());
-    kside_kernel<<<grid1, kKsThreads, KsLayout::kAlloc, s>>>(mq, mk, mla, kp);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_dependent(kside_kernel, grid1, kKsThreads, KsLayout::kAlloc, s, mq, mk, mla,
+                              kp)) != cudaSuccess)
+        return e;
     ChParams cp;
     cp.S0 = a.S0;
     cp.cu = a.cu_seqlens;

@@ -7,6 +7,7 @@
 // first so the chain kernels start the longest sequential chains earliest.
 // Running on the device keeps the whole call free of host synchronisation.
 #include "kda_internal.cuh"
+#include "sm100.cuh"
 
 namespace kda {
 
@@ -18,6 +19,7 @@ __global__ void __launch_bounds__(1024) varlen_index_kernel(const int32_t *__res
     __shared__ int32_t s_part[1024];
     __shared__ int s_bad;
     const int tid = threadIdx.x;
+    sm100::grid_launch_dependents();   // the key-side pass may start its set-up now
     if (chunk_off) {
         // chunk_off[n] = sum_{i<n} ceil(len_i / 64) (malformed sequences count
         // as empty): each thread scans a contiguous segment, then the block

@@ -98,6 +98,19 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
     return false;
 }
 
+// ------------------------------------------- programmatic dependent launch
+// A kernel launched with programmatic stream serialisation may start while
+// the kernel before it in the stream is still running; it must wait here
+// before it reads anything that kernel writes.  Without that launch
+// attribute both are no-ops.
+__device__ __forceinline__ void grid_dependency_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+// Lets the next kernel in the stream (if launched as above) start launching.
+__device__ __forceinline__ void grid_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- fences
 // Generic-proxy shared-memory writes -> visible to the async proxy
 // (tcgen05.mma operand reads, TMA).

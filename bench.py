@@ -224,19 +224,29 @@ def dist_setup():
 
 
 def barrier(world):
+    """All ranks meet, then this rank's GPU work is finished (CPU-only runs of
+    the host logic, e.g. the gloo tests, skip the device sync)."""
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
-    torch.cuda.synchronize()
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
 
 
 def max_over_ranks(x, world):
+    """Largest value over the ranks (device times are reported as the max)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(units_per_rank, world, max_ms):
+    """Whole-job rate: the units every rank processed over the slowest rank's time."""
+    return world * units_per_rank / (max_ms * 1e-3)
 
 
 # --------------------------------------------------------------------------
@@ -319,7 +329,7 @@ def bench_kda(args):
         barrier(world)
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     total_ms = max_over_ranks(sum(step_ms), world)
-    value = world * T * args.steps / (total_ms * 1e-3)
+    value = job_throughput(T * args.steps, world, total_ms)
 
     # ---- end to end through the public API from pinned host buffers -------
     names = ("q", "k", "v", "log_alpha", "beta")

@@ -305,16 +305,17 @@ __device__ __forceinline__ void solve_chunk(int sw, int lane, uint32_t tmem, uin
         for (int aa = 0; aa < 16; ++aa) col[aa] = 0.f;
 #pragma unroll
         for (int aa = 0; aa < 16; ++aa) {
-            float acc = 0.f;
+            // four independent partial sums keep the dependent chain short
+            float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
             for (int m4 = 0; m4 < aa; m4 += 4) {
                 const float4 l = *reinterpret_cast<const float4 *>(sL + (o + aa) * kLDL + o + m4);
-                acc = fmaf(l.x, col[m4], acc);
-                if (m4 + 1 < aa) acc = fmaf(l.y, col[m4 + 1], acc);
-                if (m4 + 2 < aa) acc = fmaf(l.z, col[m4 + 2], acc);
-                if (m4 + 3 < aa) acc = fmaf(l.w, col[m4 + 3], acc);
+                a0 = fmaf(l.x, col[m4], a0);
+                if (m4 + 1 < aa) a1 = fmaf(l.y, col[m4 + 1], a1);
+                if (m4 + 2 < aa) a2 = fmaf(l.z, col[m4 + 2], a2);
+                if (m4 + 3 < aa) a3 = fmaf(l.w, col[m4 + 3], a3);
             }
-            col[aa] = (aa == j) ? 1.f : -acc;
+            col[aa] = (aa == j) ? 1.f : -((a0 + a1) + (a2 + a3));
         }
 #pragma unroll
         for (int aa = 0; aa < 16; ++aa) sT[(o + aa) * kLDL + o + j] = col[aa];
@@ -337,7 +338,8 @@ __device__ __forceinline__ void solve_chunk(int sw, int lane, uint32_t tmem, uin
             const int cb = sw < 2 ? (pass == 0 ? 0 : 4) : 1 + pass;
             const int c0 = 16 * cb + 8 * q;
             for (int i = cb + 1; i < 4; ++i) {
-                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                // two accumulators (k halves of each block) halve the mma chain
+                float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
                 for (int jb = cb; jb < i; ++jb) {
 #pragma unroll
                     for (int kk = 0; kk < 16; kk += 8) {
@@ -346,13 +348,13 @@ __device__ __forceinline__ void solve_chunk(int sw, int lane, uint32_t tmem, uin
                                                 tf32_bits(Lr[4]), tf32_bits(Lr[8 * kLDL + 4])};
                         const float *Tc = sT + (16 * jb + kk + tq) * kLDL + c0 + g;
                         const uint32_t bfr[2] = {tf32_bits(Tc[0]), tf32_bits(Tc[4 * kLDL])};
-                        mma_tf32_16x8x8(acc, af, bfr);
+                        mma_tf32_16x8x8(acc[kk >> 3], af, bfr);
                     }
                 }
-                xw[g * 17 + 2 * tq] = acc[0];
-                xw[g * 17 + 2 * tq + 1] = acc[1];
-                xw[(g + 8) * 17 + 2 * tq] = acc[2];
-                xw[(g + 8) * 17 + 2 * tq + 1] = acc[3];
+                xw[g * 17 + 2 * tq] = acc[0][0] + acc[1][0];
+                xw[g * 17 + 2 * tq + 1] = acc[0][1] + acc[1][1];
+                xw[(g + 8) * 17 + 2 * tq] = acc[0][2] + acc[1][2];
+                xw[(g + 8) * 17 + 2 * tq + 1] = acc[0][3] + acc[1][3];
                 __syncwarp();
                 float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll

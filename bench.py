@@ -332,41 +332,73 @@ def bench_kda(args):
     value = job_throughput(T * args.steps, world, total_ms)
 
     # ---- end to end through the public API from pinned host buffers -------
+    # Every step copies its inputs in from pinned host memory, runs the
+    # forward and copies the outputs (out and S_final) back.  Steps are
+    # pipelined the way a serving loop would run them: step i+1's inputs copy
+    # in on one copy stream while step i computes and step i-1's outputs copy
+    # out on another; two device buffer sets alternate.
     names = ("q", "k", "v", "log_alpha", "beta")
     host = {k: inp[k].pin_memory() for k in names}
     host["S0"] = inp["S0"].pin_memory() if inp["S0"] is not None else None
     host_cu = inp["cu_seqlens"].pin_memory()
-    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    sf_h = torch.empty(sf.shape, dtype=sf.dtype).pin_memory()
-    dd = {k: torch.empty_like(d[k]) for k in names}
-    s0d = torch.empty_like(d["S0"]) if d["S0"] is not None else None
-    cud = torch.empty_like(d["cu_seqlens"])
+    out_h = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
+    sf_h = [torch.empty(sf.shape, dtype=sf.dtype).pin_memory() for _ in range(2)]
+    slots = []
+    for _ in range(2):
+        slots.append(dict(
+            x={k: torch.empty_like(d[k]) for k in names},
+            s0=torch.empty_like(d["S0"]) if d["S0"] is not None else None,
+            cu=torch.empty_like(d["cu_seqlens"]),
+            out=torch.empty_like(out), sf=torch.empty_like(sf),
+            ws=torch.empty_like(ws)))
     h2d = sum(host[k].numel() * host[k].element_size() for k in names) + \
         (host["S0"].numel() * 4 if host["S0"] is not None else 0) + host_cu.numel() * 4
-    d2h = out_h.numel() * out_h.element_size() + sf_h.numel() * 4
+    d2h = out_h[0].numel() * out_h[0].element_size() + sf_h[0].numel() * 4
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event()
+    inputs_free, copied_in, computed, copied_out = ([ev() for _ in range(2)] for _ in range(4))
 
-    def e2e_step():
-        for k in names:
-            dd[k].copy_(host[k], non_blocking=True)
-        if s0d is not None:
-            s0d.copy_(host["S0"], non_blocking=True)
-        cud.copy_(host_cu, non_blocking=True)
-        kda.forward(dd["q"], dd["k"], dd["v"], dd["log_alpha"], dd["beta"], s0d, cud, out=out,
-                    S_final=sf, workspace=ws)
-        out_h.copy_(out, non_blocking=True)
-        sf_h.copy_(sf, non_blocking=True)
+    def e2e_run(n_steps):
+        for i in range(n_steps):
+            b = i & 1
+            sl = slots[b]
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(inputs_free[b])
+                for k in names:
+                    sl["x"][k].copy_(host[k], non_blocking=True)
+                if sl["s0"] is not None:
+                    sl["s0"].copy_(host["S0"], non_blocking=True)
+                sl["cu"].copy_(host_cu, non_blocking=True)
+                copied_in[b].record(s_in)
+            stream.wait_event(copied_in[b])
+            if i >= 2:
+                stream.wait_event(copied_out[b])     # this set's outputs have left
+            kda.forward(sl["x"]["q"], sl["x"]["k"], sl["x"]["v"], sl["x"]["log_alpha"],
+                        sl["x"]["beta"], sl["s0"], sl["cu"], out=sl["out"], S_final=sl["sf"],
+                        workspace=sl["ws"])
+            inputs_free[b].record(stream)
+            computed[b].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(computed[b])
+                out_h[b].copy_(sl["out"], non_blocking=True)
+                sf_h[b].copy_(sl["sf"], non_blocking=True)
+                copied_out[b].record(s_out)
 
-    for _ in range(max(1, args.warmup)):
-        e2e_step()
+    e2e_run(max(2, args.warmup))
+    torch.cuda.synchronize()
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
+    s_in.wait_stream(stream)
+    e2e_run(args.steps)
+    stream.wait_stream(s_out)
     e1.record(stream)
     barrier(world)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
-    e2e_value = world * T * args.steps / (e2e_ms * 1e-3)
+    e2e_value = job_throughput(T * args.steps, world, e2e_ms)
+    if not torch.equal(out_h[(args.steps - 1) & 1].to(dev), out):
+        raise RuntimeError("end-to-end output differs from the device-resident run")
 
     # ---- prefix-cache snapshots: the same forward keeping the state every
     # 512 tokens in a slot pool (bf16, d = 128 only) ------------------------
@@ -435,7 +467,10 @@ def bench_kda(args):
                        "l2": "256 MiB flush between steps, outside the timed spans",
                        "parallelism": f"replicas x{world}"},
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h},
+                    "d2h_bytes_per_step": d2h,
+                    "ms_per_step": e2e_ms / args.steps,
+                    "schedule": "pinned host buffers; step i+1 copies in while step i computes "
+                                "and step i-1 copies out (two device buffer sets)"},
             # per call: varlen index, then the key-side and chain passes
             # (bf16, d = 128, full workspace) or the one CUDA-core kernel
             "gpu_launches": (3 if (w.torch_dtype == torch.bfloat16 and Dk == 128 and Dv == 128)

@@ -347,3 +347,28 @@ def test_snapshot_at_sequence_end_is_the_final_state():
     _, s, snaps, off = oracle.forward(q, k, v, la, beta, S0=S0, cu_seqlens=cu, snapshot_every=E)
     n = 2                            # 32 tokens = 2 E: its last snapshot is its final state
     assert np.array_equal(snaps[off[n] + 1], s[n])
+
+
+# --------------------------------------------------------------------------
+# stored exact values (tests/golden/exact_chain.json, written by
+# tests/golden/make_exact_chain.py from oracle.exact only)
+# --------------------------------------------------------------------------
+def test_oracle_reproduces_the_stored_exact_chain():
+    import json
+    import os
+    from fractions import Fraction
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "exact_chain.json")
+    doc = json.load(open(path))
+    f = lambda M: np.array([[float(Fraction(x)) for x in row] for row in M])
+    inp = doc["inputs"]
+    T = len(inp["q"])
+    q, k, v, alpha = (f(inp[n])[:, None, :] for n in ("q", "k", "v", "alpha"))
+    beta = np.array([float(Fraction(x)) for x in inp["beta"]])[:, None]
+    S0 = f(inp["S0"])[None, None]
+    out, sf = oracle.forward(q, k, v, np.log(alpha), beta, S0=S0)
+    assert np.allclose(out[:, 0], f(doc["out"]), rtol=1e-13, atol=1e-14)
+    assert np.allclose(sf[0, 0], f(doc["states"][T - 1]), rtol=1e-13, atol=1e-14)
+    # and every intermediate state, through the snapshot entry point
+    _, _, snaps, _ = oracle.forward(q, k, v, np.log(alpha), beta, S0=S0, snapshot_every=1)
+    for t in range(T):
+        assert np.allclose(snaps[t, 0], f(doc["states"][t]), rtol=1e-13, atol=1e-14)

@@ -7,18 +7,22 @@
 // work dominates the latency of a chunk, so it runs in its own pass:
 //
 //   pass 1  (kside_kernel, persistent, one chunk x head per item, spread over
-//           every SM): gate prep, [A;P] = [Kg;Qg] Ki^T, the triangular
-//           inverse Tb, W = Tb Kg.  It writes one operand packet per item to
+//           every SM, items claimed from a counter): gate prep, [A;P] =
+//           [Kg;Qg] Ki^T, the triangular inverse Tb, PT = P Tb and
+//           [W; PW] = [Tb; PT] Kg.  It writes one operand packet per item to
 //           the workspace, in the exact shared-memory layout pass 2 consumes:
-//             [-W;Qg] 32 KB | Ki 16 KB | Tb 8 KB | P 8 KB | Gam_L 512 B
+//             [-W;Qe] 32 KB | Ki 16 KB | [Tb;PT] 16 KB | Gam_L 512 B
+//           with Qe = Qg - P W.
 //   pass 2  (chain_kernel, one CTA per (sequence, head, VS-wide value slice)):
 //           streams the packets and the value tile with bulk copies and runs
 //           only the value-side products and the fp32 state chain:
-//             D1  = Tb V ; D1 += [-W;Qg] S  (U | Qg S) ; dS = Ki^T U ;
-//             D1 += [0;P] U  (O) ;  S <- Diag(Gam_L) (S + dS)
+//             D1  = [Tb;PT] V ; D1 += [-W;Qe] S   (rows: U | O = Qg S + P U)
+//             dS  = Ki^T U ;  S <- Diag(Gam_L) (S + dS)
 //
-// The packets cost ~1 KB of extra HBM traffic per token-head (written once,
-// read once; the value slices of a chain share each packet through L2).
+// The packets cost ~1 KB of extra HBM traffic per token-head each way
+// (written once, read once; the value slices of a chain share each packet
+// through L2).  Pass 1 and pass 2 are launched as programmatic dependents of
+// the kernel before them.
 #include "kda_internal.cuh"
 #include "kda_tc_common.cuh"
 #include "sm100.cuh"

@@ -514,8 +514,8 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     } else if (warp == kKsMma) {
         // --------------------------------- A/P issuer (lane 0), Ki stores (lane 1)
         // Ki and Gam_L are final once the prep is done.  They leave from here,
-        // not from the store warp, which works a chunk behind: the solve writes
-        // P over Ki and must not wait for the previous chunk's stores.
+        // as soon as they are, rather than from the store warp, which works on
+        // the products that follow the solve.
         constexpr uint32_t kIdAP = idesc_bf16(128, 64, 0, 0);
         for (int i = 0;; ++i) {
             const int s = i % kKsStages, a = i & 1;

@@ -821,6 +821,21 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
         float gl_cur = 1.f;
         bool ok = true;
         const long long snap_base = (p.snap_every > 0 && p.snap_base) ? p.snap_base[seq] : -1;
+        // snapshot: the state after j full chunks, every snap_every chunks
+        auto store_snapshot = [&](int j) {
+            if (snap_base < 0 || j % p.snap_every != 0 || j * kChunk > t1 - t0) return;
+            const long long slot = snap_base + j / p.snap_every - 1;
+            if (slot < p.snap_slots) {
+                float *dst = p.snap_pool + ((size_t)slot * p.H + h) * kDK * kDV + (size_t)c * kDV +
+                             (size_t)vs * VS;
+#pragma unroll
+                for (int jj = 0; jj < VS; jj += 4)
+                    *reinterpret_cast<float4 *>(dst + jj) =
+                        make_float4(S[jj], S[jj + 1], S[jj + 2], S[jj + 3]);
+            } else if (c == 0) {
+                set_status(p.status, KDA_ERR_SLOT);
+            }
+        };
         for (int j = 0; j <= nchunks && ok; ++j) {
             if (j > 0) {
                 // S <- Diag(Gam_L) (S + dS) for chunk j-1
@@ -835,22 +850,11 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
 #pragma unroll
                     for (int e = 0; e < 32; ++e) S[jj + e] = gl_cur * (S[jj + e] + __uint_as_float(v[e]));
                 }
-                // snapshot: the state after j full chunks, every snap_every chunks
-                if (snap_base >= 0 && j % p.snap_every == 0 && j * kChunk <= t1 - t0) {
-                    const long long slot = snap_base + j / p.snap_every - 1;
-                    if (slot < p.snap_slots) {
-                        float *dst = p.snap_pool + ((size_t)slot * p.H + h) * kDK * kDV +
-                                     (size_t)c * kDV + (size_t)vs * VS;
-#pragma unroll
-                        for (int jj = 0; jj < VS; jj += 4)
-                            *reinterpret_cast<float4 *>(dst + jj) =
-                                make_float4(S[jj], S[jj + 1], S[jj + 2], S[jj + 3]);
-                    } else if (c == 0) {
-                        set_status(p.status, KDA_ERR_SLOT);
-                    }
-                }
             }
-            if (j == nchunks) break;
+            if (j == nchunks) {
+                store_snapshot(j);
+                break;
+            }
             const int s = j % Ly::kStages, d = j & 1;
             if (!spin_or_abort(&bars[cbFull + s], (j / Ly::kStages) & 1, abort_flag, p.status)) { ok = false; break; }
             gl_cur = reinterpret_cast<const float *>(sm + s * Ly::kStage + Ly::kGL)[c];
@@ -869,6 +873,11 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[cbSbFull]);
             if (c == 0) KDA_TRACE2(j, 8);
+            // Snapshot stores go after a proxy fence, never just before one: the
+            // fence would wait for them to complete.  Rows 64-127 next fence a
+            // chunk later; rows 0-63 fence the U operand below, so they store
+            // after that.
+            if (j > 0 && wq >= 2) store_snapshot(j);
 
             if (!spin_or_abort(&bars[cbUFull], j & 1, abort_flag, p.status)) { ok = false; break; }
             tc_fence_after();
@@ -895,6 +904,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars[cbUbFull]);
                 if (c == 0) KDA_TRACE2(j, 10);
+                if (j > 0) store_snapshot(j);
             } else {
                 // O rows: D1 lanes 64..127 -> bf16 output
                 const int c0 = t0 + j * kChunk, L = min(kChunk, t1 - c0);

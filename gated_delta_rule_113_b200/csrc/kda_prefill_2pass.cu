@@ -821,9 +821,9 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
         float gl_cur = 1.f;
         bool ok = true;
         const long long snap_base = (p.snap_every > 0 && p.snap_base) ? p.snap_base[seq] : -1;
-        // snapshot: the state after j full chunks, every snap_every chunks
+        // snapshot: the state after j >= 1 full chunks, every snap_every chunks
         auto store_snapshot = [&](int j) {
-            if (snap_base < 0 || j % p.snap_every != 0 || j * kChunk > t1 - t0) return;
+            if (j <= 0 || snap_base < 0 || j % p.snap_every != 0 || j * kChunk > t1 - t0) return;
             const long long slot = snap_base + j / p.snap_every - 1;
             if (slot < p.snap_slots) {
                 float *dst = p.snap_pool + ((size_t)slot * p.H + h) * kDK * kDV + (size_t)c * kDV +

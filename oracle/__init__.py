@@ -9,6 +9,8 @@ Contents
   * ``forward`` / ``decode_step`` -- the token-by-token recurrence in plain C
     (``kda_oracle.c``), fp64, no FMA contraction, threaded over independent
     (sequence, head) chains.
+  * ``backward`` -- the gradients of a loss through that recurrence, the
+    forward steps differentiated in reverse order (``kda_oracle_bwd.c``).
   * ``chunked.forward_chunked`` -- an fp64 numpy restatement of the same
     recurrence in chunk form, used only to pin the chunk algebra that the
     GPU kernels rely on (tests compare it with ``forward``).
@@ -34,6 +36,7 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "kda_oracle.c")
+_SRC_BWD = os.path.join(_HERE, "kda_oracle_bwd.c")
 _BUILD_DIR = os.path.join(_HERE, "_build")
 _LIB_PATH = os.path.join(_BUILD_DIR, "libkda_oracle.so")
 _lock = threading.Lock()
@@ -45,13 +48,15 @@ CFLAGS = ["-O2", "-std=c11", "-fPIC", "-shared", "-pthread",
 
 
 def build(force: bool = False) -> str:
-    """Compile ``kda_oracle.c`` with gcc into ``oracle/_build``; return the path."""
+    """Compile ``kda_oracle.c`` and ``kda_oracle_bwd.c`` with gcc into one
+    library under ``oracle/_build``; return its path."""
     os.makedirs(_BUILD_DIR, exist_ok=True)
     stale = (not os.path.exists(_LIB_PATH)
-             or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC))
+             or os.path.getmtime(_LIB_PATH) < max(os.path.getmtime(_SRC),
+                                                  os.path.getmtime(_SRC_BWD)))
     if force or stale:
         tmp = _LIB_PATH + f".tmp{os.getpid()}"
-        subprocess.run(["gcc", *CFLAGS, "-o", tmp, _SRC, "-lm"], check=True)
+        subprocess.run(["gcc", *CFLAGS, "-o", tmp, _SRC, _SRC_BWD, "-lm"], check=True)
         os.replace(tmp, _LIB_PATH)
     return _LIB_PATH
 
@@ -72,6 +77,21 @@ def bind(path: str):
     lib.kda_oracle_decode_step.restype = ctypes.c_int
     lib.kda_oracle_decode_step.argtypes = [
         i64, i64, i64, i64, dp, dp, dp, dp, dp, dp, dp, ctypes.c_int]
+    if hasattr(lib, "kda_oracle_backward"):   # builds of the forward source alone lack it
+        bind_backward(lib)
+    return lib
+
+
+def bind_backward(lib):
+    """Declare the backward entry point on a loaded library (ctypes.CDLL or path)."""
+    if isinstance(lib, str):
+        lib = ctypes.CDLL(lib)
+    dp = ctypes.POINTER(ctypes.c_double)
+    i64 = ctypes.c_int64
+    lib.kda_oracle_backward.restype = ctypes.c_int
+    lib.kda_oracle_backward.argtypes = [
+        i64, ctypes.POINTER(i64), i64, i64, i64,
+        dp, dp, dp, dp, dp, dp, dp, dp, dp, dp, dp, dp, dp, dp, ctypes.c_int]
     return lib
 
 
@@ -188,3 +208,47 @@ def decode_step(q, k, v, log_alpha, beta, S, threads=None):
     if rc != 0:
         raise RuntimeError(f"kda_oracle_decode_step failed with code {rc}")
     return out, s
+
+
+def backward(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, d_out=None, dS_final=None,
+             threads=None, lib=None):
+    """fp64 gradients of a loss L through the recurrence (``kda_oracle_bwd.c``).
+
+    Inputs as ``forward``; d_out [T_tot, H, Dv] = dL/d out; dS_final
+    [N, H, Dk, Dv] = dL/dS_final or None (zero).  Returns a dict with dq, dk,
+    dlog_alpha [T_tot, H, Dk], dv [T_tot, H, Dv], dbeta [T_tot, H] and dS0
+    [N, H, Dk, Dv], all float64.  ``lib`` (tests only) substitutes another
+    build of the backward source.
+    """
+    q, k, v, la, b, do = (_f64(x) for x in (q, k, v, log_alpha, beta, d_out))
+    T, H, Dk = q.shape
+    Dv = v.shape[2]
+    if k.shape != (T, H, Dk) or la.shape != (T, H, Dk):
+        raise ValueError("q, k, log_alpha must share the shape [T, H, Dk]")
+    if v.shape[:2] != (T, H) or b.shape != (T, H) or do.shape != (T, H, Dv):
+        raise ValueError("v and d_out must be [T, H, Dv] and beta [T, H]")
+    if cu_seqlens is None:
+        cu = np.array([0, T], dtype=np.int64)
+    else:
+        if hasattr(cu_seqlens, "detach"):
+            cu_seqlens = cu_seqlens.detach().cpu().numpy()
+        cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int64))
+    N = cu.shape[0] - 1
+    if N < 0 or cu[0] != 0 or cu[-1] != T or np.any(np.diff(cu) < 0):
+        raise ValueError("cu_seqlens must start at 0, be non-decreasing and end at T")
+    s0 = None if S0 is None else _f64(S0)
+    dsf = None if dS_final is None else _f64(dS_final)
+    for name, x in (("S0", s0), ("dS_final", dsf)):
+        if x is not None and x.shape != (N, H, Dk, Dv):
+            raise ValueError(f"{name} must be [N, H, Dk, Dv]")
+    g = {"dq": np.zeros((T, H, Dk)), "dk": np.zeros((T, H, Dk)), "dv": np.zeros((T, H, Dv)),
+         "dlog_alpha": np.zeros((T, H, Dk)), "dbeta": np.zeros((T, H)),
+         "dS0": np.zeros((N, H, Dk, Dv))}
+    rc = (lib or _load()).kda_oracle_backward(
+        N, cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), H, Dk, Dv,
+        _ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(b), _ptr(s0), _ptr(do), _ptr(dsf),
+        _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["dlog_alpha"]), _ptr(g["dbeta"]),
+        _ptr(g["dS0"]), int(threads or default_threads()))
+    if rc != 0:
+        raise RuntimeError(f"kda_oracle_backward failed with code {rc}")
+    return g

@@ -241,3 +241,4 @@ int kda_oracle_decode_step(int64_t n_seqs, int64_t H, int64_t Dk, int64_t Dv,
     free(cu);
     return rc;
 }
+

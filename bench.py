@@ -440,6 +440,11 @@ def bench_kda(args):
     if not args.no_decode:
         dec = bench_decode(kda, dev, stream, world, args)
 
+    # ---- backward (gradients) on the prefill workload ---------------------
+    bwd = None
+    if not args.no_backward:
+        bwd = bench_backward(kda, dev, stream, world, w, d, T, N, H, Dk, Dv)
+
     # ---- roofline of the dominant kernel (prefill) -------------------------
     peaks, peaks_kind = load_peaks()
     alg_bytes = prefill_bytes(T, N, H, Dk, Dv, w.torch_dtype, w.torch_dtype, inp["S0"] is not None)
@@ -478,6 +483,7 @@ def bench_kda(args):
             "roofline": roof,
             "cpu_baseline": cpu,
             "decode": dec,
+            "backward": bwd,
             "snapshots": snap,
             "clocks": clk.summary(),
         }
@@ -486,6 +492,55 @@ def bench_kda(args):
         import torch.distributed as dist
         dist.destroy_process_group()
     return 0
+
+
+def bench_backward(kda, dev, stream, world, w, d, T, N, H, Dk, Dv, steps=3):
+    """kda_backward on the prefill workload: dL/d out random, dL/dS_final and
+    dL/dS0 included.  One call = the varlen index and the backward kernel.
+
+    Algorithmic flops per token-head, counted once (no recomputation): the
+    forward step 5 Dk Dv (decay, P^T k, rank-one write) and the reverse step
+    16 Dk Dv (dq, the read-out outer product, G u, G^T k, P du, dP, the decay
+    row sums and the decayed G).  The kernel runs on CUDA cores in fp32, so its
+    roof is the fp32 FMA rate: 148 SMs x 128 lanes x 2 flop x the SM clock."""
+    g = torch.Generator(device=dev).manual_seed(5)
+    d_out = torch.randn((T, H, Dv), generator=g, device=dev).to(w.torch_dtype)
+    dSf = torch.randn((N, H, Dk, Dv), generator=g, device=dev)
+    ws = torch.empty(kda.backward_workspace_size(N, T, H, Dk, Dv, w.torch_dtype),
+                     dtype=torch.uint8, device=dev)
+
+    def call():
+        return kda.backward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["S0"],
+                            d["cu_seqlens"], d_out=d_out, dS_final=dSf, workspace=ws)
+
+    for _ in range(2):
+        call()
+    if kda.workspace_status(ws) != 0:
+        raise RuntimeError("device status not OK after the backward warm-up")
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        call()
+    e1.record(stream)
+    barrier(world)
+    ms = max_over_ranks(e0.elapsed_time(e1), world) / steps
+    flops = 21.0 * Dk * Dv * T * H
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    peaks, _ = load_peaks()
+    alu_tflops = sms * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+    achieved = flops / (ms * 1e-3) / 1e12
+    io = _es(w.torch_dtype)
+    moved = T * H * (3 * Dk * io + Dv * io + 2 + Dv * io + 3 * Dk * 4 + Dv * 4 + 4) + \
+        2 * N * H * Dk * Dv * 4
+    return {"workload": w.name, "value": world * T / (ms * 1e-3), "unit": "tokens/s",
+            "ms_per_call": ms, "gpu_launches": 2 * steps,
+            "grads": "dq, dk, dv, dlog_alpha, dbeta, dS0 (fp32); dS_final given",
+            "roofline": {"bound": "alu", "achieved": achieved, "peak": alu_tflops,
+                         "unit": "TFLOP/s", "frac": achieved / alu_tflops, "traffic": None,
+                         "peak_kind": "derived: fp32 FMA, SMs x 128 x 2 x max SM clock",
+                         "algorithmic_flops": flops, "algorithmic_bytes": moved,
+                         "hbm_frac_algorithmic": moved / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}}
 
 
 def bench_decode(kda, dev, stream, world, args):
@@ -573,6 +628,7 @@ def main(argv=None):
                     help="reference arm: tokens per sequence in each timed step")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-snapshots", action="store_true")
+    ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3:

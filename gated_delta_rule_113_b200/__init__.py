@@ -17,13 +17,13 @@ import threading
 
 import torch
 
-__all__ = ["decode_multi", "forward", "decode_step", "forward_workspace_size", "workspace_status",
+__all__ = ["backward", "backward_workspace_size", "decode_multi", "forward", "decode_step", "forward_workspace_size", "workspace_status",
            "KDAError", "load_library", "LIB_PATH", "EXPORTED_SYMBOLS"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkda.so")
 EXPORTED_SYMBOLS = ("kda_forward_workspace_size", "kda_forward", "kda_forward_snapshots",
                     "kda_forward_noalloc", "kda_decode_step", "kda_decode_multi",
-                    "kda_workspace_status",
+                    "kda_backward_workspace_size", "kda_backward", "kda_workspace_status",
                     "kda_status_string", "kda_abi_version")
 
 KDA_F32, KDA_BF16 = 0, 1
@@ -77,6 +77,10 @@ def load_library(path: str = LIB_PATH):
         lib.kda_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, pp, vp]
         lib.kda_decode_multi.restype = ctypes.c_int
         lib.kda_decode_multi.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, pp, ctypes.c_int32, vp]
+        lib.kda_backward_workspace_size.restype = sz
+        lib.kda_backward_workspace_size.argtypes = [pp]
+        lib.kda_backward.restype = ctypes.c_int
+        lib.kda_backward.argtypes = [vp] * 15 + [pp, vp, sz, vp]
         lib.kda_workspace_status.restype = ctypes.c_int
         lib.kda_workspace_status.argtypes = [vp, i32p, vp]
         lib.kda_status_string.restype = ctypes.c_char_p
@@ -259,3 +263,59 @@ def decode_multi(q, k, v, log_alpha, beta, S, *, S_tokens=None, out=None):
                                     _ptr(S), _ptr(S_tokens), _ptr(out), ctypes.byref(p), int(n),
                                     _stream(dev)))
     return out, S_tokens
+
+
+def backward_workspace_size(N: int, T: int, H: int, Dk: int, Dv: int,
+                            dtype=torch.bfloat16) -> int:
+    """Bytes of device workspace ``kda_backward`` needs for this problem."""
+    d = KDA_BF16 if dtype == torch.bfloat16 else KDA_F32
+    p = Params(N, T, H, Dk, Dv, CHUNK, d, d, 0)
+    return int(load_library().kda_backward_workspace_size(ctypes.byref(p)))
+
+
+def backward(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, *, d_out, dS_final=None,
+             need_dS0=True, workspace=None):
+    """Gradients through ``kda_backward`` of a loss with dL/d out = ``d_out``
+    (and dL/dS_final = ``dS_final``, None: zero).
+
+    Inputs as ``forward``.  Returns a dict of fp32 tensors: dq, dk, dlog_alpha
+    [T, H, Dk], dv [T, H, Dv], dbeta [T, H] and dS0 [N, H, Dk, Dv] (None when
+    ``need_dS0`` is false).
+    """
+    lib = load_library()
+    dev = q.device
+    T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    if cu_seqlens is None:
+        cu_seqlens = torch.tensor([0, T], dtype=torch.int32, device=dev)
+    if cu_seqlens.dtype != torch.int32:
+        raise KDAError("cu_seqlens must be int32")
+    N = cu_seqlens.numel() - 1
+    if k.shape != q.shape or log_alpha.shape != q.shape or v.shape[:2] != (T, H) \
+            or beta.shape != (T, H) or d_out.shape != v.shape:
+        raise KDAError("shape mismatch among q, k, v, log_alpha, beta, d_out")
+    if k.dtype != q.dtype or v.dtype != q.dtype or d_out.dtype != q.dtype \
+            or beta.dtype != log_alpha.dtype:
+        raise KDAError("q, k, v, d_out must share a dtype; log_alpha and beta must share a dtype")
+    for name, x in (("S0", S0), ("dS_final", dS_final)):
+        if x is not None and (x.dtype != torch.float32 or x.shape != (N, H, Dk, Dv)):
+            raise KDAError(f"{name} must be float32 [N, H, Dk, Dv]")
+    f32 = dict(dtype=torch.float32, device=dev)
+    g = {"dq": torch.empty((T, H, Dk), **f32), "dk": torch.empty((T, H, Dk), **f32),
+         "dv": torch.empty((T, H, Dv), **f32), "dlog_alpha": torch.empty((T, H, Dk), **f32),
+         "dbeta": torch.empty((T, H), **f32),
+         "dS0": torch.empty((N, H, Dk, Dv), **f32) if need_dS0 else None}
+    p = Params(N, T, H, Dk, Dv, CHUNK, _dt(q), _dt(log_alpha), 0)
+    ws_bytes = int(lib.kda_backward_workspace_size(ctypes.byref(p)))
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    _require(dict(q=q, k=k, v=v, log_alpha=log_alpha, beta=beta, S0=S0, cu_seqlens=cu_seqlens,
+                  d_out=d_out, dS_final=dS_final, workspace=workspace, **g), dev)
+    with torch.cuda.device(dev):
+        _check(lib.kda_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+                                _ptr(S0), _ptr(cu_seqlens), _ptr(d_out), _ptr(dS_final),
+                                _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]),
+                                _ptr(g["dlog_alpha"]), _ptr(g["dbeta"]), _ptr(g["dS0"]),
+                                ctypes.byref(p), _ptr(workspace), workspace.numel(),
+                                _stream(dev)))
+    return g

@@ -245,6 +245,81 @@ kda_status kda_decode_multi(const void *q, const void *k, const void *v, const v
     return KDA_OK;
 }
 
+// Backward workspace: [status header][order: N int32][chunk_off: N+1 int32]
+// [chunk-start states: ceil(T/64) + N chunks x H x Dk x Dv fp32]
+// [per-CTA scratch: N x H x Dv/32 CTAs].
+namespace {
+size_t bw_ckpt_chunks(const kda_params *p) {
+    return (size_t)((p->total_tokens + kda::kChunk - 1) / kda::kChunk) + (size_t)p->num_seqs;
+}
+size_t bw_ckpt_offset(const kda_params *p) {
+    return kWsHeader + round_up(sizeof(int32_t) * (size_t)p->num_seqs, 256) +
+           round_up(sizeof(int32_t) * ((size_t)p->num_seqs + 1), 256);
+}
+size_t bw_scratch_offset(const kda_params *p) {
+    return bw_ckpt_offset(p) +
+           round_up(bw_ckpt_chunks(p) * p->H * p->Dk * p->Dv * sizeof(float), 256);
+}
+size_t bw_workspace_bytes(const kda_params *p) {
+    const size_t ctas = (size_t)p->num_seqs * p->H * (p->Dv / 32);
+    return bw_scratch_offset(p) + ctas * kda::backward_scratch_floats(p->Dk) * sizeof(float);
+}
+}  // namespace
+
+size_t kda_backward_workspace_size(const kda_params *p) {
+    if (check_common(p) != KDA_OK || p->total_tokens < 0) return 0;
+    return bw_workspace_bytes(p);
+}
+
+kda_status kda_backward(const void *q, const void *k, const void *v, const void *log_alpha,
+                        const void *beta, const float *S0, const int32_t *cu_seqlens,
+                        const void *d_out, const float *dS_final, float *dq, float *dk,
+                        float *dv, float *dlog_alpha, float *dbeta, float *dS0,
+                        const kda_params *p, void *workspace, size_t ws_bytes, void *stream) {
+    kda_status st = check_common(p);
+    if (st != KDA_OK) return st;
+    if (p->chunk != kda::kChunk || p->total_tokens < 0) return KDA_ERR_UNSUPPORTED;
+    if (p->num_seqs == 0) return p->total_tokens == 0 ? KDA_OK : KDA_ERR_INVALID;
+    if (!cu_seqlens) return KDA_ERR_INVALID;
+    if (p->total_tokens > 0 && (!q || !k || !v || !log_alpha || !beta || !d_out || !dq || !dk ||
+                                !dv || !dlog_alpha || !dbeta))
+        return KDA_ERR_INVALID;
+    const void *ptrs[] = {q, k, v, log_alpha, beta, S0, cu_seqlens, d_out, dS_final, dq, dk,
+                          dv, dlog_alpha, dbeta, dS0, workspace};
+    for (const void *x : ptrs)
+        if (x && !aligned16(x)) return KDA_ERR_ALIGN;
+    if (!workspace || ((uintptr_t)workspace & 255u) || ws_bytes < bw_workspace_bytes(p))
+        return KDA_ERR_WORKSPACE;
+    if ((long long)p->num_seqs * p->H * (p->Dv / 32) > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+    st = select_device(ptrs, 16);
+    if (st != KDA_OK) return st;
+
+    char *ws = static_cast<char *>(workspace);
+    kda::ForwardArgs ix;   // the varlen index: validation, order, chunk offsets
+    memset(&ix, 0, sizeof(ix));
+    ix.cu_seqlens = cu_seqlens;
+    ix.N = p->num_seqs; ix.T = p->total_tokens; ix.H = p->H;
+    ix.status = reinterpret_cast<int32_t *>(ws);
+    ix.order = reinterpret_cast<int32_t *>(ws + kWsHeader);
+    ix.chunk_off = reinterpret_cast<int32_t *>(
+        ws + kWsHeader + round_up(sizeof(int32_t) * (size_t)p->num_seqs, 256));
+    ix.work_ctr = nullptr;
+    kda::BackwardArgs a;
+    a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta; a.d_out = d_out;
+    a.S0 = S0; a.dS_final = dS_final; a.cu_seqlens = cu_seqlens;
+    a.dq = dq; a.dk = dk; a.dv = dv; a.dla = dlog_alpha; a.dbeta = dbeta; a.dS0 = dS0;
+    a.N = p->num_seqs; a.T = p->total_tokens; a.H = p->H; a.Dk = p->Dk; a.Dv = p->Dv;
+    a.io_dtype = p->io_dtype; a.gate_dtype = p->gate_dtype;
+    a.status = ix.status; a.order = ix.order; a.chunk_off = ix.chunk_off;
+    a.ckpt = reinterpret_cast<float *>(ws + bw_ckpt_offset(p));
+    a.ckpt_chunks = bw_ckpt_chunks(p);
+    a.scratch = reinterpret_cast<float *>(ws + bw_scratch_offset(p));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (kda::launch_varlen_index(ix, s) != cudaSuccess) return KDA_ERR_CUDA;
+    if (kda::launch_backward(a, s) != cudaSuccess) return KDA_ERR_CUDA;
+    return KDA_OK;
+}
+
 kda_status kda_workspace_status(const void *workspace, int32_t *status, void *stream) {
     if (!workspace || !status) return KDA_ERR_INVALID;
     const void *ptrs[] = {workspace};

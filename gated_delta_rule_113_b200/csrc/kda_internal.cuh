@@ -48,7 +48,25 @@ struct DecodeArgs {
     int io_dtype, gate_dtype;
 };
 
+// Gradients (kda_backward), already validated on the host.
+struct BackwardArgs {
+    const void *q, *k, *v, *log_alpha, *beta, *d_out;
+    const float *S0, *dS_final;       // either may be null
+    const int32_t *cu_seqlens;
+    float *dq, *dk, *dv, *dla, *dbeta;
+    float *dS0;                       // or null
+    int N, T, H, Dk, Dv;
+    int io_dtype, gate_dtype;
+    int32_t *status, *order, *chunk_off;   // workspace, as the forward's
+    float *ckpt;                      // [ckpt_chunks, H, Dv / 32, Dk, 32] chunk-start states
+    size_t ckpt_chunks;
+    float *scratch;                   // per CTA: 64 states of a slice and 64 u rows
+};
+// fp32 elements of one backward CTA's scratch (CTA = sequence, head, 32-wide value slice)
+inline size_t backward_scratch_floats(int Dk) { return (size_t)kChunk * Dk * 32 + kChunk * 32; }
+
 cudaError_t launch_varlen_index(const ForwardArgs &a, cudaStream_t s);
+cudaError_t launch_backward(const BackwardArgs &a, cudaStream_t s);
 cudaError_t launch_prefill_simt(const ForwardArgs &a, cudaStream_t s);
 bool prefill_tc_supported(const ForwardArgs &a);
 cudaError_t launch_prefill_tc(const ForwardArgs &a, cudaStream_t s);

@@ -44,7 +44,7 @@
 extern "C" {
 #endif
 
-#define KDA_ABI_VERSION 2
+#define KDA_ABI_VERSION 3
 
 typedef enum kda_status {
     KDA_OK = 0,
@@ -267,6 +267,52 @@ kda_status kda_decode_multi(const void *q, const void *k, const void *v,
                             const void *log_alpha, const void *beta, const float *S,
                             float *S_tokens, void *out, const kda_params *p,
                             int32_t n_tokens, void *stream);
+
+/*
+ * kda_backward_workspace_size -- bytes of device workspace kda_backward needs
+ * for this problem; 0 when `p` is NULL or invalid.  Must be 256-byte
+ * aligned; needs no initialisation.  About
+ * (total_tokens / 64 + N) * H * Dk * Dv * 4 bytes of chunk-start states plus
+ * N * H * (Dv / 32) * (64 * Dk * 32 + 2048) * 4 bytes of per-CTA scratch.
+ */
+size_t kda_backward_workspace_size(const kda_params *p);
+
+/*
+ * kda_backward -- gradients of a scalar loss L through kda_forward's
+ * recurrence (page "Kimi K3: Open Frontier Intelligence and Implementation
+ * Framework", section "Hybrid Attention Mechanism", KDA bullet; the same
+ * page trains the model built on it).  Given dL/d out and optionally
+ * dL/dS_final it writes dL/d of every input:
+ *
+ *   q, k, v, log_alpha, beta, S0, cu_seqlens   as kda_forward (S0 may be NULL)
+ *   d_out      [T_tot, H, Dv]  io_dtype, dL/d out
+ *   dS_final   [N, H, Dk, Dv]  fp32, dL/dS_final, or NULL (zero)
+ *   dq, dk     [T_tot, H, Dk]  fp32, written
+ *   dv         [T_tot, H, Dv]  fp32, written
+ *   dlog_alpha [T_tot, H, Dk]  fp32, written (gradient w.r.t. log_alpha)
+ *   dbeta      [T_tot, H]      fp32, written
+ *   dS0        [N, H, Dk, Dv]  fp32, written, or NULL (not computed); the
+ *              gradient w.r.t. the initial state also when S0 is NULL
+ *   workspace  ws_bytes >= kda_backward_workspace_size(p), 256-byte aligned
+ *
+ * All gradients are fp32 whatever io_dtype and gate_dtype; the arithmetic is
+ * fp32 on CUDA cores.  dq, dk, dlog_alpha and dbeta sum partial results of
+ * the 32-wide value slices with atomic adds, so their last bits can differ
+ * from one call to the next; dv and dS0 are written once.  The states are recomputed (the forward runs twice: once
+ * to keep the state at every chunk start, once per chunk in reverse order),
+ * so no state from kda_forward is needed.  `flags` is ignored.  Outputs may
+ * not overlap inputs or each other.  Errors as kda_forward: host validation
+ * codes, KDA_ERR_CUDA if a launch fails, KDA_ERR_SEQLENS recorded in the
+ * workspace status word for malformed cu_seqlens (those sequences' gradients
+ * are left as zero or unwritten).
+ */
+kda_status kda_backward(const void *q, const void *k, const void *v,
+                        const void *log_alpha, const void *beta,
+                        const float *S0, const int32_t *cu_seqlens,
+                        const void *d_out, const float *dS_final,
+                        float *dq, float *dk, float *dv, float *dlog_alpha,
+                        float *dbeta, float *dS0, const kda_params *p,
+                        void *workspace, size_t ws_bytes, void *stream);
 
 /*
  * kda_workspace_status -- synchronise `stream`, then copy the device status

@@ -29,7 +29,9 @@ def test_library_loads_and_exports_every_declared_symbol():
     for name in declared:
         assert hasattr(lib, name), f"{name} declared in include/ but not exported"
     assert set(kda.EXPORTED_SYMBOLS) <= set(declared)
-    assert lib.kda_abi_version() == 2
+    text = open(os.path.join(HEADER, "kda.h")).read()
+    assert lib.kda_abi_version() == int(re.search(r"#define KDA_ABI_VERSION (\d+)", text).group(1))
+    assert lib.kda_abi_version() == 3
 
 
 def test_status_strings():
@@ -153,3 +155,46 @@ def test_decode_multi_host_validation():
     assert call(_params(), St=FAKE + 4) == 3
     assert call(_params(Dk=32)) == 2
     assert call(_params(num_seqs=0)) == 0
+
+
+def _bwd(lib, p, **over):
+    args = dict(q=FAKE, k=FAKE, v=FAKE, la=FAKE, beta=FAKE, S0=None, cu=FAKE, do=FAKE, dSf=None,
+                dq=FAKE, dk=FAKE, dv=FAKE, dla=FAKE, db=FAKE, dS0=None, ws=0x20000,
+                ws_bytes=1 << 40)
+    args.update(over)
+    vp = ctypes.c_void_p
+    names = ("q", "k", "v", "la", "beta", "S0", "cu", "do", "dSf", "dq", "dk", "dv", "dla", "db",
+             "dS0")
+    return lib.kda_backward(*(vp(args[n]) for n in names), ctypes.byref(p), vp(args["ws"]),
+                            args["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("over,params,code", [
+    (dict(q=None), {}, 1),
+    (dict(do=None), {}, 1),
+    (dict(db=None), {}, 1),
+    (dict(cu=None), {}, 1),
+    ({}, dict(Dk=96), 2),
+    ({}, dict(chunk=32), 2),
+    (dict(dq=FAKE + 4), {}, 3),
+    (dict(dS0=FAKE + 8), {}, 3),
+    (dict(ws=None), {}, 4),
+    (dict(ws=0x20010), {}, 4),
+    (dict(ws_bytes=16), {}, 4),
+])
+def test_backward_host_validation(over, params, code):
+    lib = kda.load_library()
+    assert _bwd(lib, _params(**params), **over) == code
+
+
+def test_backward_workspace_size():
+    lib = kda.load_library()
+    p = _params()
+    n = lib.kda_backward_workspace_size(ctypes.byref(p))
+    # chunk-start states and per-CTA scratch dominate
+    T, N, H, Dk, Dv = p.total_tokens, p.num_seqs, p.H, p.Dk, p.Dv
+    states = ((T + 63) // 64 + N) * H * Dk * Dv * 4
+    scratch = N * H * (Dv // 32) * (64 * Dk * 32 + 64 * 32) * 4
+    assert states + scratch <= n <= states + scratch + 4096 + 8 * N
+    assert lib.kda_backward_workspace_size(ctypes.byref(_params(Dk=96))) == 0
+    assert lib.kda_backward_workspace_size(None) == 0

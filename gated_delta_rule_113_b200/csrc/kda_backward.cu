@@ -93,6 +93,11 @@ __device__ __forceinline__ float lane_column_sum(float (&x)[32], int lane) {
     return x[0];
 }
 
+// Pull the 128-byte line holding `p` into L1 (and L2) ahead of its load.
+__device__ __forceinline__ void prefetch_l1(const void *p) {
+    asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
+}
+
 __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll
     for (int s = 16; s >= 1; s >>= 1) x += __shfl_xor_sync(0xffffffffu, x, s);
@@ -138,15 +143,39 @@ backward_kernel(BwParams p) {
 
     // u = v_t - (Diag(alpha) S)^T k_t for this slice, S <- Diag(alpha) S + beta k u^T.
     // Column j of u, from the round's shared sums, is the same expression
-    // wherever it is formed.
+    // (the warps' sums added in warp order) wherever it is formed.
     auto col_sum = [&](int par, int j) {
         float s = 0.f;
 #pragma unroll
         for (int w = 0; w < NW; ++w) s += red[par][w][j];
         return s;
     };
+    auto col_sums = [&](int par, float (&cs)[32]) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) cs[j] = 0.f;
+#pragma unroll
+        for (int w = 0; w < NW; ++w)
+#pragma unroll
+            for (int j4 = 0; j4 < 8; ++j4) {
+                const float4 r = reinterpret_cast<const float4 *>(&red[par][w][0])[j4];
+                cs[4 * j4] += r.x; cs[4 * j4 + 1] += r.y; cs[4 * j4 + 2] += r.z; cs[4 * j4 + 3] += r.w;
+            }
+    };
+    // the inputs of token t: this thread's key row elements and the slice's v / d_out
+    auto prefetch_token = [&](int t, bool with_q) {
+        const size_t rk = ((size_t)t * p.H + h) * DK + c;
+        prefetch_l1(k + rk);
+        prefetch_l1(la + rk);
+        if (with_q) prefetch_l1(q + rk);
+        if (c == 0) {
+            prefetch_l1(beta + (size_t)t * p.H + h);
+            prefetch_l1(v + ((size_t)t * p.H + h) * p.Dv + col0);
+            if (with_q) prefetch_l1(dout + ((size_t)t * p.H + h) * p.Dv + col0);
+        }
+    };
     auto forward_token = [&](int t, float (&S)[32], float *u_out) {
         const size_t rk = ((size_t)t * p.H + h) * DK + c;
+        if (t + 1 < t1) prefetch_token(t + 1, false);
         const float kc = to_f32(k[rk]), ac = expf(to_f32(la[rk]));
         const float bt = to_f32(beta[(size_t)t * p.H + h]);
         float vv[32], x[32];
@@ -160,8 +189,10 @@ backward_kernel(BwParams p) {
         red[par][warp][lane] = lane_column_sum(x, lane);
         __syncthreads();
         const float bk = bt * kc;
+        float cs[32];
+        col_sums(par, cs);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) S[j] = fmaf(bk, vv[j] - col_sum(par, j), S[j]);
+        for (int j = 0; j < 32; ++j) S[j] = fmaf(bk, vv[j] - cs[j], S[j]);
         if (u_out && c < 32) {
             const float vj = to_f32(v[((size_t)t * p.H + h) * p.Dv + col0 + c]);
             u_out[c] = vj - col_sum(par, c);
@@ -203,6 +234,11 @@ backward_kernel(BwParams p) {
         for (int i = L - 1; i >= 0; --i) {
             const int t = c0 + i;
             const size_t rk = ((size_t)t * p.H + h) * DK + c;
+            if (i > 0) {   // the next (earlier) token's inputs, state row and u
+                prefetch_token(t - 1, true);
+                prefetch_l1(scr + ((size_t)(i - 1) * DK + c) * kBwVs);
+                if (c == 0) prefetch_l1(scr_u + (i - 1) * kBwVs);
+            }
             const float qc = to_f32(q[rk]), kc = to_f32(k[rk]), ac = expf(to_f32(la[rk]));
             const float bt = to_f32(beta[(size_t)t * p.H + h]);
             float Sp[32], x[32], u[32];
@@ -229,8 +265,9 @@ backward_kernel(BwParams p) {
             if (lane == 0) redb[par][warp] = kb;
             __syncthreads();
             float du[32];
+            col_sums(par, du);
 #pragma unroll
-            for (int jj = 0; jj < 32; ++jj) du[jj] = bt * col_sum(par, jj);
+            for (int jj = 0; jj < 32; ++jj) du[jj] *= bt;
             if (c < 32) p.dv[((size_t)t * p.H + h) * p.Dv + col0 + c] = bt * col_sum(par, c);
             if (c == 0) {
                 float db = 0.f;

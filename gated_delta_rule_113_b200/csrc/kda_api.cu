@@ -246,11 +246,11 @@ kda_status kda_decode_multi(const void *q, const void *k, const void *v, const v
 }
 
 // Backward workspace: [status header][order: N int32][chunk_off: N+1 int32]
-// [chunk-start states: ceil(T/64) + N chunks x H x Dk x Dv fp32]
+// [states every 32 tokens: 2 (ceil(T/64) + N) x H x Dk x Dv fp32]
 // [per-CTA scratch: N x H x Dv/32 CTAs].
 namespace {
-size_t bw_ckpt_chunks(const kda_params *p) {
-    return (size_t)((p->total_tokens + kda::kChunk - 1) / kda::kChunk) + (size_t)p->num_seqs;
+size_t bw_ckpt_steps(const kda_params *p) {
+    return 2 * ((size_t)((p->total_tokens + kda::kChunk - 1) / kda::kChunk) + (size_t)p->num_seqs);
 }
 size_t bw_ckpt_offset(const kda_params *p) {
     return kWsHeader + round_up(sizeof(int32_t) * (size_t)p->num_seqs, 256) +
@@ -258,7 +258,7 @@ size_t bw_ckpt_offset(const kda_params *p) {
 }
 size_t bw_scratch_offset(const kda_params *p) {
     return bw_ckpt_offset(p) +
-           round_up(bw_ckpt_chunks(p) * p->H * p->Dk * p->Dv * sizeof(float), 256);
+           round_up(bw_ckpt_steps(p) * p->H * p->Dk * p->Dv * sizeof(float), 256);
 }
 size_t bw_workspace_bytes(const kda_params *p) {
     const size_t ctas = (size_t)p->num_seqs * p->H * (p->Dv / 32);
@@ -312,7 +312,7 @@ kda_status kda_backward(const void *q, const void *k, const void *v, const void 
     a.io_dtype = p->io_dtype; a.gate_dtype = p->gate_dtype;
     a.status = ix.status; a.order = ix.order; a.chunk_off = ix.chunk_off;
     a.ckpt = reinterpret_cast<float *>(ws + bw_ckpt_offset(p));
-    a.ckpt_chunks = bw_ckpt_chunks(p);
+    a.ckpt_steps = bw_ckpt_steps(p);
     a.scratch = reinterpret_cast<float *>(ws + bw_scratch_offset(p));
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (kda::launch_varlen_index(ix, s) != cudaSuccess) return KDA_ERR_CUDA;

@@ -25,12 +25,13 @@
 // shared memory; the per-row sums over the columns (dq, dk, dlog_alpha) and
 // dbeta add the slices' partial sums into fp32 outputs zeroed beforehand.
 //
-// States: pass A runs the chain forward and stores the state at every chunk
-// start (every 64 tokens).  Pass B walks the chunks backward; for each it
-// recomputes the chunk's 64 states from its checkpoint into a per-CTA scratch
-// (with u of every token), then runs the reverse steps over the chunk.  The
+// States: pass A runs the chain forward and stores the state every kBwStep =
+// 32 tokens (a "step").  Pass B walks the steps backward; for each it
+// recomputes the step's 32 states from its checkpoint into a per-CTA scratch
+// (with u of every token), then runs the reverse steps over them.  The
 // forward is thus evaluated twice and every state is exact fp32 recomputation,
-// not an inverse of the recurrence.
+// not an inverse of the recurrence.  32 tokens keep the scratch of all CTAs
+// (512 KB each at d = 128) inside L2.
 #include "kda_internal.cuh"
 
 namespace kda {
@@ -43,9 +44,9 @@ struct BwParams {
     const float *S0, *dSf;
     const int32_t *cu, *order, *chunk_off;
     float *dq, *dk, *dv, *dla, *dbeta, *dS0;
-    float *ckpt;             // [ckpt_chunks, H, n_slices, DK, 32]
-    float *scratch;          // per CTA: [64, DK, 32] states, then [64, 32] u
-    long long ckpt_chunks;   // chunk checkpoints the workspace holds (per head and slice)
+    float *ckpt;             // [ckpt_steps, H, n_slices, DK, 32]
+    float *scratch;          // per CTA: [kBwStep, DK, 32] states, then [kBwStep, 32] u
+    long long ckpt_steps;    // checkpoints the workspace holds (per head and slice)
     int32_t *status;
     int N, T, H, Dv;
 };
@@ -126,9 +127,11 @@ backward_kernel(BwParams p) {
         if (c == 0) set_status(p.status, KDA_ERR_SEQLENS);
         return;
     }
-    const int nc = (t1 - t0 + kChunk - 1) / kChunk;
-    const long long g0 = p.chunk_off[n];
-    if (g0 + nc > p.ckpt_chunks) {   // overlapping (malformed) sequences
+    // sequence n's steps take checkpoint slots 2 chunk_off[n] .. + ceil(len / 32)
+    // (at most two per 64-token chunk)
+    const int nc = (t1 - t0 + kBwStep - 1) / kBwStep;
+    const long long g0 = 2LL * p.chunk_off[n];
+    if (g0 + nc > p.ckpt_steps) {   // overlapping (malformed) sequences
         if (c == 0) set_status(p.status, KDA_ERR_SEQLENS);
         return;
     }
@@ -137,8 +140,8 @@ backward_kernel(BwParams p) {
         return p.ckpt + ((((size_t)g0 + j) * p.H + h) * n_slices + vs) * DK * kBwVs +
                (size_t)c * kBwVs;
     };
-    float *scr = p.scratch + (size_t)blockIdx.x * (kChunk * DK * kBwVs + kChunk * kBwVs);
-    float *scr_u = scr + kChunk * DK * kBwVs;
+    float *scr = p.scratch + (size_t)blockIdx.x * (kBwStep * DK * kBwVs + kBwStep * kBwVs);
+    float *scr_u = scr + kBwStep * DK * kBwVs;
     int round = 0;
 
     // u = v_t - (Diag(alpha) S)^T k_t for this slice, S <- Diag(alpha) S + beta k u^T.
@@ -150,16 +153,11 @@ backward_kernel(BwParams p) {
         for (int w = 0; w < NW; ++w) s += red[par][w][j];
         return s;
     };
+    // all 32 column sums: lane l forms column l's, then the warp shares them
     auto col_sums = [&](int par, float (&cs)[32]) {
+        const float mine = col_sum(par, lane);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) cs[j] = 0.f;
-#pragma unroll
-        for (int w = 0; w < NW; ++w)
-#pragma unroll
-            for (int j4 = 0; j4 < 8; ++j4) {
-                const float4 r = reinterpret_cast<const float4 *>(&red[par][w][0])[j4];
-                cs[4 * j4] += r.x; cs[4 * j4 + 1] += r.y; cs[4 * j4 + 2] += r.z; cs[4 * j4 + 3] += r.w;
-            }
+        for (int j = 0; j < 32; ++j) cs[j] = __shfl_sync(0xffffffffu, mine, j);
     };
     // the inputs of token t: this thread's key row elements and the slice's v / d_out
     auto prefetch_token = [&](int t, bool with_q) {
@@ -199,7 +197,7 @@ backward_kernel(BwParams p) {
         }
     };
 
-    // ---------------------------------------------- pass A: chunk checkpoints
+    // ---------------------------------------------- pass A: checkpoints every kBwStep tokens
     float S[32];
     {
         const float *src = p.S0 ? p.S0 + (((size_t)n * p.H + h) * DK + c) * p.Dv + col0 : nullptr;
@@ -210,11 +208,11 @@ backward_kernel(BwParams p) {
     }
     for (int j = 0; j < nc; ++j) {
         store32(ckpt_row(j), S);
-        const int c0 = t0 + j * kChunk, c1 = min(t1, c0 + kChunk);
+        const int c0 = t0 + j * kBwStep, c1 = min(t1, c0 + kBwStep);
         for (int t = c0; t < c1; ++t) forward_token(t, S, nullptr);
     }
 
-    // ---------------------------------------------- pass B: reverse, chunk by chunk
+    // ---------------------------------------------- pass B: reverse, step by step
     float G[32];
     {
         const float *src = p.dSf ? p.dSf + (((size_t)n * p.H + h) * DK + c) * p.Dv + col0 : nullptr;
@@ -224,7 +222,7 @@ backward_kernel(BwParams p) {
             for (int j = 0; j < 32; ++j) G[j] = 0.f;
     }
     for (int j = nc - 1; j >= 0; --j) {
-        const int c0 = t0 + j * kChunk, L = min(kChunk, t1 - c0);
+        const int c0 = t0 + j * kBwStep, L = min(kBwStep, t1 - c0);
         load32(ckpt_row(j), S);
         for (int i = 0; i < L; ++i) {   // states S_{t-1} and u of the chunk's tokens
             store32(scr + ((size_t)i * DK + c) * kBwVs, S);
@@ -324,7 +322,7 @@ cudaError_t launch_backward(const BackwardArgs &a, cudaStream_t s) {
     bp.cu = a.cu_seqlens; bp.order = a.order; bp.chunk_off = a.chunk_off;
     bp.dq = a.dq; bp.dk = a.dk; bp.dv = a.dv; bp.dla = a.dla; bp.dbeta = a.dbeta;
     bp.dS0 = a.dS0; bp.ckpt = a.ckpt; bp.scratch = a.scratch;
-    bp.ckpt_chunks = (long long)a.ckpt_chunks; bp.status = a.status;
+    bp.ckpt_steps = (long long)a.ckpt_steps; bp.status = a.status;
     bp.N = a.N; bp.T = a.T; bp.H = a.H; bp.Dv = a.Dv;
     const bool io_bf16 = a.io_dtype == KDA_BF16, g_bf16 = a.gate_dtype == KDA_BF16;
     if (io_bf16 && g_bf16) return launch_bw_dk<__nv_bfloat16, __nv_bfloat16>(bp, a.Dk, s);

@@ -58,12 +58,14 @@ struct BackwardArgs {
     int N, T, H, Dk, Dv;
     int io_dtype, gate_dtype;
     int32_t *status, *order, *chunk_off;   // workspace, as the forward's
-    float *ckpt;                      // [ckpt_chunks, H, Dv / 32, Dk, 32] chunk-start states
-    size_t ckpt_chunks;
-    float *scratch;                   // per CTA: 64 states of a slice and 64 u rows
+    float *ckpt;                      // [ckpt_steps, H, Dv / 32, Dk, 32] states every kBwStep tokens
+    size_t ckpt_steps;
+    float *scratch;                   // per CTA: kBwStep states of a slice and kBwStep u rows
 };
-// fp32 elements of one backward CTA's scratch (CTA = sequence, head, 32-wide value slice)
-inline size_t backward_scratch_floats(int Dk) { return (size_t)kChunk * Dk * 32 + kChunk * 32; }
+// The backward keeps the state every kBwStep tokens (two per chunk); one CTA
+// (sequence, head, 32-wide value slice) recomputes kBwStep states at a time.
+constexpr int kBwStep = 32;
+inline size_t backward_scratch_floats(int Dk) { return (size_t)kBwStep * Dk * 32 + kBwStep * 32; }
 
 cudaError_t launch_varlen_index(const ForwardArgs &a, cudaStream_t s);
 cudaError_t launch_backward(const BackwardArgs &a, cudaStream_t s);

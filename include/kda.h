@@ -272,8 +272,9 @@ kda_status kda_decode_multi(const void *q, const void *k, const void *v,
  * kda_backward_workspace_size -- bytes of device workspace kda_backward needs
  * for this problem; 0 when `p` is NULL or invalid.  Must be 256-byte
  * aligned; needs no initialisation.  About
- * (total_tokens / 64 + N) * H * Dk * Dv * 4 bytes of chunk-start states plus
- * N * H * (Dv / 32) * (64 * Dk * 32 + 2048) * 4 bytes of per-CTA scratch.
+ * 2 (total_tokens / 64 + N) * H * Dk * Dv * 4 bytes of states (one every 32
+ * tokens) plus N * H * (Dv / 32) * (32 * Dk * 32 + 1024) * 4 bytes of per-CTA
+ * scratch.
  */
 size_t kda_backward_workspace_size(const kda_params *p);
 
@@ -298,8 +299,9 @@ size_t kda_backward_workspace_size(const kda_params *p);
  * All gradients are fp32 whatever io_dtype and gate_dtype; the arithmetic is
  * fp32 on CUDA cores.  dq, dk, dlog_alpha and dbeta sum partial results of
  * the 32-wide value slices with atomic adds, so their last bits can differ
- * from one call to the next; dv and dS0 are written once.  The states are recomputed (the forward runs twice: once
- * to keep the state at every chunk start, once per chunk in reverse order),
+ * from one call to the next; dv and dS0 are written once.  The states are
+ * recomputed (the forward runs twice: once to keep the state every 32
+ * tokens, once per 32 tokens in reverse order),
  * so no state from kda_forward is needed.  `flags` is ignored.  Outputs may
  * not overlap inputs or each other.  Errors as kda_forward: host validation
  * codes, KDA_ERR_CUDA if a launch fails, KDA_ERR_SEQLENS recorded in the

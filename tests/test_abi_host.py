@@ -191,10 +191,10 @@ def test_backward_workspace_size():
     lib = kda.load_library()
     p = _params()
     n = lib.kda_backward_workspace_size(ctypes.byref(p))
-    # chunk-start states and per-CTA scratch dominate
+    # the kept states and the per-CTA scratch dominate
     T, N, H, Dk, Dv = p.total_tokens, p.num_seqs, p.H, p.Dk, p.Dv
-    states = ((T + 63) // 64 + N) * H * Dk * Dv * 4
-    scratch = N * H * (Dv // 32) * (64 * Dk * 32 + 64 * 32) * 4
+    states = 2 * ((T + 63) // 64 + N) * H * Dk * Dv * 4          # one every 32 tokens
+    scratch = N * H * (Dv // 32) * (32 * Dk * 32 + 32 * 32) * 4
     assert states + scratch <= n <= states + scratch + 4096 + 8 * N
     assert lib.kda_backward_workspace_size(ctypes.byref(_params(Dk=96))) == 0
     assert lib.kda_backward_workspace_size(None) == 0

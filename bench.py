@@ -537,7 +537,8 @@ def bench_backward(kda, dev, stream, world, w, d, T, N, H, Dk, Dv, steps=3):
             "ms_per_call": ms, "gpu_launches": 2 * steps,
             "grads": "dq, dk, dv, dlog_alpha, dbeta, dS0 (fp32); dS_final given",
             "roofline": {"bound": "alu", "achieved": achieved, "peak": alu_tflops,
-                         "unit": "TFLOP/s", "frac": achieved / alu_tflops, "traffic": None,
+                         "unit": "TFLOP/s", "frac": achieved / alu_tflops,
+                         "traffic": traffic_record("kda_backward"),
                          "peak_kind": "derived: fp32 FMA, SMs x 128 x 2 x max SM clock",
                          "algorithmic_flops": flops, "algorithmic_bytes": moved,
                          "hbm_frac_algorithmic": moved / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}}

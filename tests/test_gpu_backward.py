@@ -103,3 +103,41 @@ def test_backward_malformed_seqlens_reported_not_faulting():
                  d_out=inp["d_out"].cuda(), workspace=buf[:n_ws])
     assert kda.workspace_status(buf[:n_ws]) == 7
     assert not buf[n_ws:].any()            # nothing written past the workspace
+
+
+def test_backward_fp32_io_bf16_gates():
+    w = WORKLOADS[0]
+    inp = _case(w, [150, 90], 2, True, True)
+    inp["log_alpha"] = inp["log_alpha"].to(torch.bfloat16)
+    inp["beta"] = inp["beta"].to(torch.bfloat16)
+    _check(inp, _run(inp))
+
+
+def test_backward_full_size_sampled_chains():
+    """The benchmark's workload (bf16, B=2, T=4096, H=16, d=128) in one call on
+    the GPU; the oracle recomputes two whole chains (one per sequence, heads 0
+    and 11) from the same inputs and the sampled gradients must match."""
+    w = WORKLOADS[1]
+    inp = forward_inputs(w)
+    g = torch.Generator().manual_seed(21)
+    T, H = inp["q"].shape[:2]
+    N = inp["cu_seqlens"].numel() - 1
+    inp["d_out"] = torch.randn((T, H, w.Dv), generator=g).to(inp["v"].dtype)
+    inp["dS_final"] = torch.randn((N, H, w.Dk, w.Dv), generator=g)
+    got = _run(inp)
+    cu = inp["cu_seqlens"].numpy()
+    for n, h in ((0, 0), (1, 11)):
+        a, b = int(cu[n]), int(cu[n + 1])
+        one = {k: inp[k][a:b, h:h + 1].contiguous() for k in ("q", "k", "v", "log_alpha",
+                                                               "d_out")}
+        one["beta"] = inp["beta"][a:b, h:h + 1].contiguous()
+        one["S0"] = inp["S0"][n:n + 1, h:h + 1] if inp["S0"] is not None else None
+        one["dS_final"] = inp["dS_final"][n:n + 1, h:h + 1]
+        one["cu_seqlens"] = torch.tensor([0, b - a], dtype=torch.int32)
+        ref = _oracle(one)
+        sl = {"dq": got["dq"][a:b, h], "dk": got["dk"][a:b, h], "dv": got["dv"][a:b, h],
+              "dlog_alpha": got["dlog_alpha"][a:b, h], "dbeta": got["dbeta"][a:b, h],
+              "dS0": got["dS0"][n, h]}
+        for name, x in sl.items():
+            e = rel_fro(as_np(x), ref[name].reshape(as_np(x).shape))
+            assert e <= TOL_GRAD, f"chain ({n}, {h}) {name}: relative error {e:.3e}"

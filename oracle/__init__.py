@@ -13,7 +13,9 @@ Contents
     forward steps differentiated in reverse order (``kda_oracle_bwd.c``).
   * ``chunked.forward_chunked`` -- an fp64 numpy restatement of the same
     recurrence in chunk form, used only to pin the chunk algebra that the
-    GPU kernels rely on (tests compare it with ``forward``).
+    GPU kernels rely on (tests compare it with ``forward``);
+    ``chunked.backward_chunked`` takes reverse mode through that chunk
+    algebra (tests compare it with ``backward``).
   * ``exact.unrolled_product`` -- the recurrence written as an explicit
     product of transition matrices in exact rational arithmetic, for tiny
     inputs (pins ``forward`` to the definition itself).

@@ -157,3 +157,28 @@ def test_backward_mutant_rejected(tmp_path, name, orig, mut):
     text = open(SRC_BWD).read()
     assert text.count(orig) == 1, f"mutation anchor for {name} not unique"
     assert not _fd_pin(_build_bwd(tmp_path, name, text.replace(orig, mut))), name
+
+
+@pytest.mark.parametrize("C", [1, 7, 16, 64])
+def test_chunk_form_backward_matches_token_backward(C):
+    """The chunk-form gradients (oracle.chunked.backward_chunked: reverse mode
+    through the chunk algebra of the forward, the algebra a chunked backward
+    kernel uses) equal the token-level backward, including partial last
+    chunks and an empty sequence."""
+    from oracle.chunked import backward_chunked
+    rng = np.random.default_rng(C)
+    lens = [70, 0, 33, 129]
+    T, H, Dk, Dv, N = sum(lens), 2, 8, 6, len(lens)
+    x = lambda *s: rng.standard_normal(s)
+    q, k = x(T, H, Dk), x(T, H, Dk)
+    q /= np.linalg.norm(q, axis=-1, keepdims=True)
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    v, do = x(T, H, Dv), x(T, H, Dv)
+    la = rng.uniform(math.log(0.8), 0.0, (T, H, Dk))
+    b = rng.uniform(0.1, 1.0, (T, H))
+    S0, dSf = x(N, H, Dk, Dv), x(N, H, Dk, Dv)
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    ref = oracle.backward(q, k, v, la, b, S0, cu, do, dSf)
+    got = backward_chunked(q, k, v, la, b, S0, cu, do, dSf, chunk=C)
+    for name in NAMES.values():
+        np.testing.assert_allclose(got[name], ref[name], rtol=1e-10, atol=1e-10, err_msg=name)

@@ -308,14 +308,16 @@ cudaError_t launch_bw_dk(const BwParams &bp, int Dk, cudaStream_t s) {
 
 cudaError_t launch_backward(const BackwardArgs &a, cudaStream_t s) {
     const size_t T = (size_t)a.T, H = (size_t)a.H;
-    // the slices' partial sums are added into these
+    // the slices' partial sums are added into these (absent when there are no tokens)
     cudaError_t e;
-    if ((e = cudaMemsetAsync(a.dq, 0, T * H * a.Dk * sizeof(float), s)) != cudaSuccess ||
-        (e = cudaMemsetAsync(a.dk, 0, T * H * a.Dk * sizeof(float), s)) != cudaSuccess ||
-        (e = cudaMemsetAsync(a.dla, 0, T * H * a.Dk * sizeof(float), s)) != cudaSuccess ||
-        (e = cudaMemsetAsync(a.dbeta, 0, T * H * sizeof(float), s)) != cudaSuccess)
+    if (T > 0 &&
+        ((e = cudaMemsetAsync(a.dq, 0, T * H * a.Dk * sizeof(float), s)) != cudaSuccess ||
+         (e = cudaMemsetAsync(a.dk, 0, T * H * a.Dk * sizeof(float), s)) != cudaSuccess ||
+         (e = cudaMemsetAsync(a.dla, 0, T * H * a.Dk * sizeof(float), s)) != cudaSuccess ||
+         (e = cudaMemsetAsync(a.dbeta, 0, T * H * sizeof(float), s)) != cudaSuccess))
         return e;
-    if (a.N == 0 || a.T == 0) return cudaSuccess;
+    // with no tokens at all the chains still pass dS_final (or zero) on to dS0
+    if (a.N == 0) return cudaSuccess;
     BwParams bp;
     bp.q = a.q; bp.k = a.k; bp.v = a.v; bp.la = a.log_alpha; bp.beta = a.beta;
     bp.d_out = a.d_out; bp.S0 = a.S0; bp.dSf = a.dS_final;

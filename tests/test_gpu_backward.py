@@ -141,3 +141,18 @@ def test_backward_full_size_sampled_chains():
         for name, x in sl.items():
             e = rel_fro(as_np(x), ref[name].reshape(as_np(x).shape))
             assert e <= TOL_GRAD, f"chain ({n}, {h}) {name}: relative error {e:.3e}"
+
+
+def test_backward_with_no_tokens_passes_dS_final_to_dS0():
+    H, D = 2, 128
+    cu = torch.zeros(3, dtype=torch.int32, device="cuda")
+    e = torch.empty((0, H, D), dtype=torch.bfloat16, device="cuda")
+    dSf = torch.randn((2, H, D, D), device="cuda")
+    g = kda.backward(e, e, e, e, torch.empty((0, H), dtype=torch.bfloat16, device="cuda"), None,
+                     cu, d_out=e, dS_final=dSf)
+    torch.cuda.synchronize()
+    assert torch.equal(g["dS0"], dSf)
+    g0 = kda.backward(e, e, e, e, torch.empty((0, H), dtype=torch.bfloat16, device="cuda"), None,
+                      cu, d_out=e)
+    torch.cuda.synchronize()
+    assert torch.equal(g0["dS0"], torch.zeros_like(dSf))

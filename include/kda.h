@@ -302,7 +302,9 @@ size_t kda_backward_workspace_size(const kda_params *p);
  * from one call to the next; dv and dS0 are written once.  The states are
  * recomputed (the forward runs twice: once to keep the state every 32
  * tokens, once per 32 tokens in reverse order),
- * so no state from kda_forward is needed.  `flags` is ignored.  Outputs may
+ * so no state from kda_forward is needed.  The recurrence is evaluated token by
+ * token here, so the lower bound on the in-chunk decay stated at the top of
+ * this file does not apply to this entry point.  `flags` is ignored.  Outputs may
  * not overlap inputs or each other.  Errors as kda_forward: host validation
  * codes, KDA_ERR_CUDA if a launch fails, KDA_ERR_SEQLENS recorded in the
  * workspace status word for malformed cu_seqlens (those sequences' gradients

@@ -220,3 +220,61 @@ def test_backward_through_the_packets_matches_the_oracle(C, alpha_min, seed):
     got = _two_pass_backward(q, k, v, la, beta, S0, cu, dout, dSf, C)
     for name, r in ref.items():
         assert np.max(np.abs(got[name] - r)) <= 1e-9 * max(np.max(np.abs(r)), 1.0), name
+
+
+# ------------------------------------------------------------ transfer form
+# A re-association of the chain that leaves one short product per chunk on the
+# path from one chunk to the next.  With Ks_j = Ki_j Diag(Gam_L,j) (keys decayed
+# to the chunk's end) and X_{j+1} = W_{j+1} Ks_j^T (64 x 64):
+#   U_{j+1} = U0_{j+1} - W_{j+1} (Diag(Gam_L,j) S_j) - X_{j+1} U_j
+#   S_{j+1} = Diag(Gam_L,j) S_j + Ks_j^T U_j
+# U_{j+1} needs S_j (one chunk old) and U_j through X_{j+1} only.
+
+def _transfer_form(q, k, v, la, beta, S0, cu, C):
+    T, H, Dk = q.shape
+    Dv = v.shape[2]
+    out = np.zeros((T, H, Dv))
+    Sf = np.zeros((len(cu) - 1, H, Dk, Dv))
+    for n in range(len(cu) - 1):
+        for h in range(H):
+            starts = list(range(cu[n], cu[n + 1], C))
+            S = S0[n, h].copy()
+            pks, U = [], None
+            for c0 in starts:
+                sl = slice(c0, min(c0 + C, cu[n + 1]))
+                pk = _packet(q[sl, h], k[sl, h], la[sl, h], beta[sl, h])
+                pk["U0"], pk["V"] = pk["Tb"] @ v[sl, h], v[sl, h]
+                pk["Ks"] = pk["Ki"] * pk["GL"][None, :]
+                pks.append((sl, pk))
+            for j, (sl, pk) in enumerate(pks):
+                if j == 0:
+                    U = pk["U0"] + pk["mW"] @ S
+                out[sl, h] = pk["Qe"] @ S + pk["PT"] @ pk["V"]
+                S_next = pk["GL"][:, None] * S + pk["Ks"].T @ U
+                if j + 1 < len(pks):
+                    nx = pks[j + 1][1]
+                    X = -nx["mW"] @ pk["Ks"].T
+                    U = nx["U0"] + nx["mW"] @ (pk["GL"][:, None] * S) - X @ U
+                S = S_next
+            Sf[n, h] = S
+    return out, Sf
+
+
+@pytest.mark.parametrize("C,alpha_min,seed", [(64, 0.9, 3), (16, 0.5, 4), (7, 0.95, 5)])
+def test_transfer_form_matches_the_recurrence(C, alpha_min, seed):
+    rng = np.random.default_rng(seed)
+    lens = [150, 64, 1, 0, 97]
+    T, H, Dk, Dv = sum(lens), 2, 8, 6
+    q = rng.standard_normal((T, H, Dk))
+    k = rng.standard_normal((T, H, Dk))
+    q /= np.linalg.norm(q, axis=-1, keepdims=True)
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    v = rng.standard_normal((T, H, Dv))
+    beta = 1.0 / (1.0 + np.exp(-rng.standard_normal((T, H))))
+    la = rng.uniform(math.log(alpha_min), 0.0, size=(T, H, Dk))
+    S0 = 0.1 * rng.standard_normal((len(lens), H, Dk, Dv))
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    o_ref, s_ref = oracle.forward(q, k, v, la, beta, S0=S0, cu_seqlens=cu)
+    o, s = _transfer_form(q, k, v, la, beta, S0, cu, C)
+    assert np.max(np.abs(o - o_ref)) <= 1e-10 * np.max(np.abs(o_ref))
+    assert np.max(np.abs(s - s_ref)) <= 1e-10 * np.max(np.abs(s_ref))

@@ -230,7 +230,7 @@ def test_backward_through_the_packets_matches_the_oracle(C, alpha_min, seed):
 #   S_{j+1} = Diag(Gam_L,j) S_j + Ks_j^T U_j
 # U_{j+1} needs S_j (one chunk old) and U_j through X_{j+1} only.
 
-def _transfer_form(q, k, v, la, beta, S0, cu, C):
+def _transfer_form(q, k, v, la, beta, S0, cu, C, rescaled_w=False):
     T, H, Dk = q.shape
     Dv = v.shape[2]
     out = np.zeros((T, H, Dv))
@@ -253,15 +253,25 @@ def _transfer_form(q, k, v, la, beta, S0, cu, C):
                 S_next = pk["GL"][:, None] * S + pk["Ks"].T @ U
                 if j + 1 < len(pks):
                     nx = pks[j + 1][1]
-                    X = -nx["mW"] @ pk["Ks"].T
-                    U = nx["U0"] + nx["mW"] @ (pk["GL"][:, None] * S) - X @ U
+                    if rescaled_w:
+                        # the next packet's -W rescaled by this chunk's decay, per channel
+                        mWp = nx["mW"] * pk["GL"][None, :]
+                        U = nx["U0"] + mWp @ S + (mWp @ pk["Ki"].T) @ U
+                    else:
+                        X = -nx["mW"] @ pk["Ks"].T
+                        U = nx["U0"] + nx["mW"] @ (pk["GL"][:, None] * S) - X @ U
                 S = S_next
             Sf[n, h] = S
     return out, Sf
 
 
+@pytest.mark.parametrize("rescaled_w", [False, True])
 @pytest.mark.parametrize("C,alpha_min,seed", [(64, 0.9, 3), (16, 0.5, 4), (7, 0.95, 5)])
-def test_transfer_form_matches_the_recurrence(C, alpha_min, seed):
+def test_transfer_form_matches_the_recurrence(C, alpha_min, seed, rescaled_w):
+    """Both ways of writing it: with Ks, or with the next packet's W rescaled by
+    this chunk's decay, W' = W Diag(Gam_L,j), so that X_{j+1} = W'_{j+1} Ki_j^T,
+    U_{j+1} = U0_{j+1} - W'_{j+1} S_j - X_{j+1} U_j and the state update keeps
+    its present form S_{j+1} = Diag(Gam_L,j) (S_j + Ki_j^T U_j)."""
     rng = np.random.default_rng(seed)
     lens = [150, 64, 1, 0, 97]
     T, H, Dk, Dv = sum(lens), 2, 8, 6
@@ -275,6 +285,6 @@ def test_transfer_form_matches_the_recurrence(C, alpha_min, seed):
     S0 = 0.1 * rng.standard_normal((len(lens), H, Dk, Dv))
     cu = np.concatenate([[0], np.cumsum(lens)])
     o_ref, s_ref = oracle.forward(q, k, v, la, beta, S0=S0, cu_seqlens=cu)
-    o, s = _transfer_form(q, k, v, la, beta, S0, cu, C)
+    o, s = _transfer_form(q, k, v, la, beta, S0, cu, C, rescaled_w)
     assert np.max(np.abs(o - o_ref)) <= 1e-10 * np.max(np.abs(o_ref))
     assert np.max(np.abs(s - s_ref)) <= 1e-10 * np.max(np.abs(s_ref))

@@ -182,3 +182,29 @@ def test_chunk_form_backward_matches_token_backward(C):
     got = backward_chunked(q, k, v, la, b, S0, cu, do, dSf, chunk=C)
     for name in NAMES.values():
         np.testing.assert_allclose(got[name], ref[name], rtol=1e-10, atol=1e-10, err_msg=name)
+
+
+def test_chunk_form_backward_property():
+    """Random small shapes, lengths (empty ones included) and chunk sizes: the
+    chunk-form gradients equal the token-level ones."""
+    from hypothesis import given, settings, strategies as st
+    from oracle.chunked import backward_chunked
+
+    @settings(max_examples=40, deadline=None, derandomize=True)
+    @given(lens=st.lists(st.integers(0, 23), min_size=1, max_size=3),
+           C=st.integers(1, 9), H=st.integers(1, 2), Dk=st.integers(1, 5), Dv=st.integers(1, 4),
+           seed=st.integers(0, 2**16))
+    def check(lens, C, H, Dk, Dv, seed):
+        rng = np.random.default_rng(seed)
+        T, N = sum(lens), len(lens)
+        x = lambda *s: rng.standard_normal(s)
+        la = rng.uniform(math.log(0.5), 0.0, (T, H, Dk))
+        args = (x(T, H, Dk), x(T, H, Dk), x(T, H, Dv), la, rng.uniform(0.0, 1.0, (T, H)),
+                x(N, H, Dk, Dv), np.concatenate([[0], np.cumsum(lens)]), x(T, H, Dv),
+                x(N, H, Dk, Dv))
+        ref = oracle.backward(*args)
+        got = backward_chunked(*args, chunk=C)
+        for name in NAMES.values():
+            np.testing.assert_allclose(got[name], ref[name], rtol=1e-9, atol=1e-9, err_msg=name)
+
+    check()

@@ -3,8 +3,11 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload I] [--impl reference]
 
 One step = one ``kda_forward`` call (varlen index + chunked prefill, every
-step of the hot path) over the prefill workload ``--workload`` (default 1:
-bf16, B=2, T=4096, H=16, d_k=d_v=128, chunk 64).  The timed region is K
+step of the hot path) over the prefill workload ``--workload`` (default 3,
+the largest prefill that fits one GPU: bf16, 8 packed sequences with
+lengths drawn from U[1024, 32768], H=32, d_k=d_v=128, chunk 64; the other
+two bf16 prefill workloads are timed as extra objects of the same line,
+each with its own roofline).  The timed region is K
 steps between a barrier + synchronize on both sides; each step's kernels
 are bracketed by CUDA events on the launching stream and L2 is flushed
 (256 MiB write) between steps outside those brackets.  Multi-GPU runs are
@@ -83,14 +86,15 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
-def traffic_record(kernel):
-    """DRAM bytes per launch from a committed ncu capture, if the kernel's source is unchanged."""
+def traffic_record(kernel, workload=None):
+    """DRAM bytes per launch from a committed ncu capture (keyed by kernel, and
+    workload where the traffic depends on it), if the sources are unchanged."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         recs = json.load(f)
-    rec = recs.get(kernel)
+    rec = recs.get(f"{kernel}:{workload}" if workload else kernel)
     if not rec:
         return None
     return rec["bytes_per_launch"] if sources_sha(rec) == rec.get("source_sha") else None
@@ -249,6 +253,65 @@ def job_throughput(units_per_rank, world, max_ms):
     return world * units_per_rank / (max_ms * 1e-3)
 
 
+def prefill_roofline(w, inp, mean_ms, peaks, peaks_kind):
+    """Roofline of one kda_forward call: algorithmic bytes over its CUDA-event
+    duration against the measured HBM copy peak (the prefill is HBM-bound at
+    ~109 flop/B), with the algorithmic tensor fraction beside it."""
+    N, T = len(inp["lengths"]), int(inp["cu_seqlens"][-1])
+    alg_bytes = prefill_bytes(T, N, w.H, w.Dk, w.Dv, w.torch_dtype, w.torch_dtype,
+                              inp["S0"] is not None)
+    alg_flops = prefill_flops(T, w.H, w.Dk, w.Dv)
+    achieved = alg_bytes / (mean_ms * 1e-3) / 1e9
+    return {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / peaks["hbm_gbs"],
+            "traffic": traffic_record("kda_prefill", w.name),
+            "peak_kind": f"{peaks_kind} HBM copy",
+            "kernel": "kda_forward (varlen_index + kside + chain kernels, one call)",
+            "algorithmic_bytes": alg_bytes, "algorithmic_flops": alg_flops,
+            "tensor_frac_algorithmic": alg_flops / (mean_ms * 1e-3) / 1e12 / peaks["bf16_tflops"]}
+
+
+def time_prefill(kda, d, out, sf, ws, flush, stream, steps):
+    """CUDA-event time (ms) of each of ``steps`` kda_forward calls, L2 flushed
+    between calls outside the events."""
+    def step():
+        kda.forward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["S0"], d["cu_seqlens"],
+                    out=out, S_final=sf, workspace=ws)
+    ev = []
+    for _ in range(steps):
+        flush.zero_()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        step()
+        a1.record(stream)
+        ev.append((a0, a1))
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in ev]
+
+
+def bench_extra_prefill(kda, dev, stream, world, wid, flush, steps, peaks, peaks_kind):
+    """One more prefill workload, timed like the headline (L2 flushed between
+    calls), reported with its own roofline."""
+    w = WORKLOADS[wid]
+    inp = forward_inputs(w)
+    N, T = len(inp["lengths"]), int(inp["cu_seqlens"][-1])
+    d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    out = torch.empty((T, w.H, w.Dv), dtype=w.torch_dtype, device=dev)
+    sf = torch.empty((N, w.H, w.Dk, w.Dv), dtype=torch.float32, device=dev)
+    ws = torch.empty(kda.forward_workspace_size(N, T, w.H, w.Dk, w.Dv, w.torch_dtype),
+                     dtype=torch.uint8, device=dev)
+    time_prefill(kda, d, out, sf, ws, flush, stream, 3)
+    if kda.workspace_status(ws) != 0:
+        raise RuntimeError(f"device status not OK on {w.name}")
+    barrier(world)
+    ms = time_prefill(kda, d, out, sf, ws, flush, stream, steps)
+    total = max_over_ranks(sum(ms), world)
+    return {"workload": w.name, "num_seqs": N, "total_tokens": T, "H": w.H,
+            "value": world * T * steps / (total * 1e-3), "unit": "tokens/s",
+            "ms_per_step": total / steps, "steps": steps, "gpu_launches": 3 * steps,
+            "roofline": prefill_roofline(w, inp, sum(ms) / len(ms), peaks, peaks_kind)}
+
+
 # --------------------------------------------------------------------------
 # arms
 # --------------------------------------------------------------------------
@@ -289,7 +352,10 @@ def bench_kda(args):
     torch.cuda.set_device(dev)
     kda.load_library()
     w = WORKLOADS[args.workload]
-    inp = forward_inputs(w)
+    inp = forward_inputs(w, lengths=args.lengths)
+    if args.lengths:   # a reduced case of the workload (profiling): renamed accordingly
+        import dataclasses
+        w = dataclasses.replace(w, name=f"{w.name}_lengths_{'_'.join(map(str, args.lengths))}")
     N, T, H, Dk, Dv = len(inp["lengths"]), int(inp["cu_seqlens"][-1]), w.H, w.Dk, w.Dv
     d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
     out = torch.empty((T, H, Dv), dtype=w.torch_dtype, device=dev)
@@ -440,22 +506,32 @@ def bench_kda(args):
     if not args.no_decode:
         dec = bench_decode(kda, dev, stream, world, args)
 
-    # ---- backward (gradients) on the prefill workload ---------------------
-    bwd = None
-    if not args.no_backward:
-        bwd = bench_backward(kda, dev, stream, world, w, d, T, N, H, Dk, Dv)
-
     # ---- roofline of the dominant kernel (prefill) -------------------------
     peaks, peaks_kind = load_peaks()
-    alg_bytes = prefill_bytes(T, N, H, Dk, Dv, w.torch_dtype, w.torch_dtype, inp["S0"] is not None)
-    alg_flops = prefill_flops(T, H, Dk, Dv)
-    mean_ms = sum(step_ms) / len(step_ms)
-    achieved = alg_bytes / (mean_ms * 1e-3) / 1e9
-    roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-            "frac": achieved / peaks["hbm_gbs"], "traffic": traffic_record("kda_prefill"),
-            "peak_kind": f"{peaks_kind} HBM copy", "kernel": "kda_forward (varlen_index + kside + chain kernels, one call)",
-            "algorithmic_bytes": alg_bytes, "algorithmic_flops": alg_flops,
-            "tensor_frac_algorithmic": alg_flops / (mean_ms * 1e-3) / 1e12 / peaks["bf16_tflops"]}
+    roof = prefill_roofline(w, inp, sum(step_ms) / len(step_ms), peaks, peaks_kind)
+
+    # ---- the other bf16 prefill workloads, each with its own roofline -----
+    extra = {}
+    if not args.no_extra:
+        del d, out, sf, ws
+        torch.cuda.empty_cache()
+        for wid in (1, 2, 3):
+            if wid != args.workload:
+                extra[WORKLOADS[wid].name] = bench_extra_prefill(
+                    kda, dev, stream, world, wid, flush, max(5, args.steps // 2), peaks,
+                    peaks_kind)
+                torch.cuda.empty_cache()
+
+    # ---- backward (gradients) on the B2 T4096 H16 prefill workload ---------
+    bwd = None
+    if not args.no_backward:
+        wb = WORKLOADS[1]
+        ib = forward_inputs(wb)
+        db = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in ib.items()}
+        bwd = bench_backward(kda, dev, stream, world, wb, db, int(ib["cu_seqlens"][-1]),
+                             len(ib["lengths"]), wb.H, wb.Dk, wb.Dv)
+        del db
+        torch.cuda.empty_cache()
 
     if rank == 0:
         cpu = None
@@ -482,6 +558,7 @@ def bench_kda(args):
                              else 2) * args.steps,
             "roofline": roof,
             "cpu_baseline": cpu,
+            "prefill_workloads": extra,
             "decode": dec,
             "backward": bwd,
             "snapshots": snap,
@@ -621,7 +698,7 @@ def main(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", type=int, default=1, choices=[0, 1, 2, 3])
+    ap.add_argument("--workload", type=int, default=3, choices=[0, 1, 2, 3])
     ap.add_argument("--impl", default="kda", choices=["kda", "reference"])
     ap.add_argument("--cpu-tokens", type=int, default=4096,
                     help="oracle sample: first N tokens of each sequence")
@@ -631,6 +708,10 @@ def main(argv=None):
     ap.add_argument("--no-snapshots", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--lengths", type=lambda x: [int(v) for v in x.split(",")], default=None,
+                    help="override the workload's sequence lengths (a reduced case, e.g. for ncu)")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the extra prefill workloads (time only --workload)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3

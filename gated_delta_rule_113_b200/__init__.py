@@ -22,7 +22,7 @@ __all__ = ["backward", "backward_workspace_size", "decode_multi", "forward", "de
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkda.so")
 EXPORTED_SYMBOLS = ("kda_forward_workspace_size", "kda_forward", "kda_forward_snapshots",
-                    "kda_forward_noalloc", "kda_decode_step", "kda_decode_multi",
+                    "kda_forward_noalloc", "kda_forward_noalloc_status", "kda_decode_step", "kda_decode_multi",
                     "kda_backward_workspace_size", "kda_backward", "kda_workspace_status",
                     "kda_status_string", "kda_abi_version")
 

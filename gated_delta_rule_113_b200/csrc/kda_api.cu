@@ -25,8 +25,9 @@ kda_status check_common(const kda_params *p) {
 }
 
 // Pointers must be device (or managed) memory of one device; make that
-// device current for the launches.  Host memory would fault on the GPU.
-kda_status select_device(const void *const *ptrs, int n) {
+// device current for the launches (the guard restores the caller's context
+// when the entry point returns).  Host memory would fault on the GPU.
+kda_status select_device(const void *const *ptrs, int n, kda::DeviceGuard &guard) {
     int dev = -1;
     for (int i = 0; i < n; ++i) {
         if (!ptrs[i]) continue;
@@ -41,10 +42,7 @@ kda_status select_device(const void *const *ptrs, int n) {
         else if (dev != at.device) return KDA_ERR_INVALID;
     }
     if (dev < 0) return KDA_OK;
-    int cur = -1;
-    if (cudaGetDevice(&cur) != cudaSuccess) return KDA_ERR_CUDA;
-    if (cur != dev && cudaSetDevice(dev) != cudaSuccess) return KDA_ERR_CUDA;
-    return KDA_OK;
+    return guard.use(dev) ? KDA_OK : KDA_ERR_CUDA;
 }
 
 // Workspace layout: [status header][order: N int32][chunk_off: N+1 int32]
@@ -86,6 +84,8 @@ const char *kda_status_string(kda_status s) {
     case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT: bounded device wait gave up";
     case KDA_ERR_SEQLENS: return "KDA_ERR_SEQLENS: cu_seqlens not monotone from 0 to total_tokens";
     case KDA_ERR_SLOT: return "KDA_ERR_SLOT: snapshot-pool slot outside the pool";
+    case KDA_ERR_DECAY:
+        return "KDA_ERR_DECAY: log_alpha > 0 or not finite, or in-chunk cumulative log-decay below -80";
     }
     return "KDA_ERR_UNKNOWN";
 }
@@ -129,7 +129,8 @@ kda_status forward_impl(const void *q, const void *k, const void *v, const void 
         return KDA_ERR_WORKSPACE;
     // grid = N * H * (Dv / 32) CTAs must fit in gridDim.x
     if ((long long)p->num_seqs * p->H * (p->Dv / 32) > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
-    st = select_device(ptrs, 13);
+    kda::DeviceGuard guard;
+    st = select_device(ptrs, 13, guard);
     if (st != KDA_OK) return st;
 
     kda::ForwardArgs a;
@@ -202,7 +203,8 @@ kda_status kda_decode_step(const void *q, const void *k, const void *v, const vo
     for (const void *x : ptrs)
         if (!aligned16(x)) return KDA_ERR_ALIGN;
     if ((long long)p->num_seqs * p->H * (p->Dv / 64) > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
-    st = select_device(ptrs, 7);
+    kda::DeviceGuard guard;
+    st = select_device(ptrs, 7, guard);
     if (st != KDA_OK) return st;
 
     kda::DecodeArgs a;
@@ -229,7 +231,8 @@ kda_status kda_decode_multi(const void *q, const void *k, const void *v, const v
         if (!aligned16(x)) return KDA_ERR_ALIGN;
     if ((long long)p->num_seqs * p->H * (p->Dv / 64) > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
     if ((long long)p->num_seqs * n_tokens > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
-    st = select_device(ptrs, 8);
+    kda::DeviceGuard guard;
+    st = select_device(ptrs, 8, guard);
     if (st != KDA_OK) return st;
 
     kda::DecodeArgs a;
@@ -247,7 +250,8 @@ kda_status kda_decode_multi(const void *q, const void *k, const void *v, const v
 
 // Backward workspace: [status header][order: N int32][chunk_off: N+1 int32]
 // [states every 32 tokens: 2 (ceil(T/64) + N) x H x Dk x Dv fp32]
-// [per-CTA scratch: N x H x Dv/32 CTAs].
+// [per-CTA scratch: N x H x Dv/32 CTAs]
+// [per value slice: partial dq, dk, dlog_alpha, dbeta].
 namespace {
 size_t bw_ckpt_steps(const kda_params *p) {
     return 2 * ((size_t)((p->total_tokens + kda::kChunk - 1) / kda::kChunk) + (size_t)p->num_seqs);
@@ -260,9 +264,15 @@ size_t bw_scratch_offset(const kda_params *p) {
     return bw_ckpt_offset(p) +
            round_up(bw_ckpt_steps(p) * p->H * p->Dk * p->Dv * sizeof(float), 256);
 }
-size_t bw_workspace_bytes(const kda_params *p) {
+size_t bw_part_offset(const kda_params *p) {
     const size_t ctas = (size_t)p->num_seqs * p->H * (p->Dv / 32);
-    return bw_scratch_offset(p) + ctas * kda::backward_scratch_floats(p->Dk) * sizeof(float);
+    return bw_scratch_offset(p) +
+           round_up(ctas * kda::backward_scratch_floats(p->Dk) * sizeof(float), 256);
+}
+size_t bw_workspace_bytes(const kda_params *p) {
+    return bw_part_offset(p) + (size_t)(p->Dv / 32) *
+                                   kda::backward_part_floats(p->total_tokens, p->H, p->Dk) *
+                                   sizeof(float);
 }
 }  // namespace
 
@@ -291,7 +301,8 @@ kda_status kda_backward(const void *q, const void *k, const void *v, const void 
     if (!workspace || ((uintptr_t)workspace & 255u) || ws_bytes < bw_workspace_bytes(p))
         return KDA_ERR_WORKSPACE;
     if ((long long)p->num_seqs * p->H * (p->Dv / 32) > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
-    st = select_device(ptrs, 16);
+    kda::DeviceGuard guard;
+    st = select_device(ptrs, 16, guard);
     if (st != KDA_OK) return st;
 
     char *ws = static_cast<char *>(workspace);
@@ -314,6 +325,8 @@ kda_status kda_backward(const void *q, const void *k, const void *v, const void 
     a.ckpt = reinterpret_cast<float *>(ws + bw_ckpt_offset(p));
     a.ckpt_steps = bw_ckpt_steps(p);
     a.scratch = reinterpret_cast<float *>(ws + bw_scratch_offset(p));
+    a.part = reinterpret_cast<float *>(ws + bw_part_offset(p));
+    a.part_stride = kda::backward_part_floats(p->total_tokens, p->H, p->Dk);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (kda::launch_varlen_index(ix, s) != cudaSuccess) return KDA_ERR_CUDA;
     if (kda::launch_backward(a, s) != cudaSuccess) return KDA_ERR_CUDA;
@@ -323,7 +336,8 @@ kda_status kda_backward(const void *q, const void *k, const void *v, const void 
 kda_status kda_workspace_status(const void *workspace, int32_t *status, void *stream) {
     if (!workspace || !status) return KDA_ERR_INVALID;
     const void *ptrs[] = {workspace};
-    kda_status st = select_device(ptrs, 1);
+    kda::DeviceGuard guard;
+    kda_status st = select_device(ptrs, 1, guard);
     if (st != KDA_OK) return st;
     if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return KDA_ERR_CUDA;
     if (cudaMemcpy(status, workspace, sizeof(int32_t), cudaMemcpyDeviceToHost) != cudaSuccess)

@@ -22,8 +22,11 @@
 // 32-wide value slice); thread c holds row c of the slice of S and of G (32
 // fp32 registers each).  The per-column sums over the rows (P^T k and G^T k)
 // are one butterfly reduce-scatter per warp plus a sum over the warps in
-// shared memory; the per-row sums over the columns (dq, dk, dlog_alpha) and
-// dbeta add the slices' partial sums into fp32 outputs zeroed beforehand.
+// shared memory.  The per-row sums over the columns (dq, dk, dlog_alpha) and
+// dbeta get one partial sum per slice: each slice stores its own in the
+// workspace and a second kernel adds the slices in slice order, so every
+// gradient is the same fixed sequence of fp32 operations on every call
+// (bitwise reproducible; no atomics).
 //
 // States: pass A runs the chain forward and stores the state every kBwStep =
 // 32 tokens (a "step").  Pass B walks the steps backward; for each it
@@ -46,6 +49,8 @@ struct BwParams {
     float *dq, *dk, *dv, *dla, *dbeta, *dS0;
     float *ckpt;             // [ckpt_steps, H, n_slices, DK, 32]
     float *scratch;          // per CTA: [kBwStep, DK, 32] states, then [kBwStep, 32] u
+    float *part;             // per slice: dq, dk, dlog_alpha [T, H, DK], dbeta [T, H]
+    size_t part_stride;      // floats per slice of `part`
     long long ckpt_steps;    // checkpoints the workspace holds (per head and slice)
     int32_t *status;
     int N, T, H, Dv;
@@ -141,6 +146,10 @@ backward_kernel(BwParams p) {
                (size_t)c * kBwVs;
     };
     float *scr = p.scratch + (size_t)blockIdx.x * (kBwStep * DK * kBwVs + kBwStep * kBwVs);
+    // this slice's partial row sums
+    const size_t thd = (size_t)p.T * p.H * DK;
+    float *part_dq = p.part + (size_t)vs * p.part_stride;
+    float *part_dk = part_dq + thd, *part_dla = part_dq + 2 * thd, *part_db = part_dq + 3 * thd;
     float *scr_u = scr + kBwStep * DK * kBwVs;
     int round = 0;
 
@@ -271,7 +280,7 @@ backward_kernel(BwParams p) {
                 float db = 0.f;
 #pragma unroll
                 for (int w = 0; w < NW; ++w) db += redb[par][w];
-                atomicAdd(p.dbeta + (size_t)t * p.H + h, db);
+                part_db[(size_t)t * p.H + h] = db;
             }
             // 2'. dk_t = beta G u - P du,  dP = G - k du^T
             // 1'. dlog_alpha_t = alpha rowsum(dP * S_{t-1}),  G = Diag(alpha) dP
@@ -284,18 +293,52 @@ backward_kernel(BwParams p) {
                 G[jj] = ac * dP;
                 S[jj] = Sp[jj];
             }
-            atomicAdd(p.dq + rk, dq_c);
-            atomicAdd(p.dk + rk, fmaf(bt, ge, -pdu));
-            atomicAdd(p.dla + rk, ac * dps);
+            part_dq[rk] = dq_c;
+            part_dk[rk] = fmaf(bt, ge, -pdu);
+            part_dla[rk] = ac * dps;
         }
     }
     if (p.dS0) store32(p.dS0 + (((size_t)n * p.H + h) * DK + c) * p.Dv + col0, G);
+}
+
+// dq, dk, dlog_alpha and dbeta = the slices' partial sums added in slice
+// order.  Four float elements per thread (every region is a multiple of 4
+// floats long: T H DK with DK in {64, 128}; T H padded in the workspace).
+__global__ void __launch_bounds__(256)
+slice_sum_kernel(const float *__restrict__ part, size_t part_stride, int n_slices, size_t thd,
+                 size_t th, float *dq, float *dk, float *dla, float *dbeta) {
+    const size_t n4 = (3 * thd + th + 3) / 4;
+    for (size_t i4 = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i4 < n4;
+         i4 += (size_t)gridDim.x * blockDim.x) {
+        const size_t i = 4 * i4;
+        float4 acc = reinterpret_cast<const float4 *>(part + i)[0];
+        for (int sl = 1; sl < n_slices; ++sl) {
+            const float4 x = reinterpret_cast<const float4 *>(part + (size_t)sl * part_stride + i)[0];
+            acc.x += x.x; acc.y += x.y; acc.z += x.z; acc.w += x.w;
+        }
+        if (i < 3 * thd) {
+            float *dst = i < thd ? dq + i : i < 2 * thd ? dk + (i - thd) : dla + (i - 2 * thd);
+            *reinterpret_cast<float4 *>(dst) = acc;
+        } else {
+            // dbeta is not padded: store only its T H elements
+            const size_t j = i - 3 * thd;
+            const float v4[4] = {acc.x, acc.y, acc.z, acc.w};
+            for (int e = 0; e < 4 && j + e < th; ++e) dbeta[j + e] = v4[e];
+        }
+    }
 }
 
 template <typename TIO, typename TG, int DK>
 cudaError_t launch_bw(const BwParams &bp, cudaStream_t s) {
     const unsigned grid = (unsigned)bp.N * bp.H * (bp.Dv / kBwVs);
     backward_kernel<TIO, TG, DK><<<grid, DK, 0, s>>>(bp);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess || bp.T == 0) return e;
+    const size_t thd = (size_t)bp.T * bp.H * DK, th = (size_t)bp.T * bp.H;
+    const size_t n4 = (3 * thd + th + 3) / 4;
+    const unsigned blocks = (unsigned)((n4 + 255) / 256 < 148 * 8 ? (n4 + 255) / 256 : 148 * 8);
+    slice_sum_kernel<<<blocks, 256, 0, s>>>(bp.part, bp.part_stride, bp.Dv / kBwVs, thd, th, bp.dq,
+                                            bp.dk, bp.dla, bp.dbeta);
     return cudaGetLastError();
 }
 
@@ -307,15 +350,6 @@ cudaError_t launch_bw_dk(const BwParams &bp, int Dk, cudaStream_t s) {
 }  // namespace
 
 cudaError_t launch_backward(const BackwardArgs &a, cudaStream_t s) {
-    const size_t T = (size_t)a.T, H = (size_t)a.H;
-    // the slices' partial sums are added into these (absent when there are no tokens)
-    cudaError_t e;
-    if (T > 0 &&
-        ((e = cudaMemsetAsync(a.dq, 0, T * H * a.Dk * sizeof(float), s)) != cudaSuccess ||
-         (e = cudaMemsetAsync(a.dk, 0, T * H * a.Dk * sizeof(float), s)) != cudaSuccess ||
-         (e = cudaMemsetAsync(a.dla, 0, T * H * a.Dk * sizeof(float), s)) != cudaSuccess ||
-         (e = cudaMemsetAsync(a.dbeta, 0, T * H * sizeof(float), s)) != cudaSuccess))
-        return e;
     // with no tokens at all the chains still pass dS_final (or zero) on to dS0
     if (a.N == 0) return cudaSuccess;
     BwParams bp;
@@ -324,6 +358,7 @@ cudaError_t launch_backward(const BackwardArgs &a, cudaStream_t s) {
     bp.cu = a.cu_seqlens; bp.order = a.order; bp.chunk_off = a.chunk_off;
     bp.dq = a.dq; bp.dk = a.dk; bp.dv = a.dv; bp.dla = a.dla; bp.dbeta = a.dbeta;
     bp.dS0 = a.dS0; bp.ckpt = a.ckpt; bp.scratch = a.scratch;
+    bp.part = a.part; bp.part_stride = a.part_stride;
     bp.ckpt_steps = (long long)a.ckpt_steps; bp.status = a.status;
     bp.N = a.N; bp.T = a.T; bp.H = a.H; bp.Dv = a.Dv;
     const bool io_bf16 = a.io_dtype == KDA_BF16, g_bf16 = a.gate_dtype == KDA_BF16;

@@ -61,7 +61,15 @@ struct BackwardArgs {
     float *ckpt;                      // [ckpt_steps, H, Dv / 32, Dk, 32] states every kBwStep tokens
     size_t ckpt_steps;
     float *scratch;                   // per CTA: kBwStep states of a slice and kBwStep u rows
+    float *part;                      // per 32-wide value slice: partial dq, dk, dla, dbeta
+    size_t part_stride;               // floats per slice of `part`
 };
+// Floats of one value slice's partial row sums: dq, dk, dlog_alpha [T, H, Dk]
+// and dbeta [T, H], padded to a multiple of 64 floats (256 bytes).
+inline size_t backward_part_floats(int64_t T, int64_t H, int Dk) {
+    const size_t n = (size_t)T * H * (3 * (size_t)Dk + 1);
+    return (n + 63) / 64 * 64;
+}
 // The backward keeps the state every kBwStep tokens (two per chunk); one CTA
 // (sequence, head, 32-wide value slice) recomputes kBwStep states at a time.
 constexpr int kBwStep = 32;
@@ -82,6 +90,29 @@ inline size_t packet_slots_bound(int64_t T, int64_t N, int64_t H) {
     return (size_t)((T + kChunk - 1) / kChunk + N) * (size_t)H;
 }
 
+// Driver API function `name` resolved through the runtime (the library does
+// not link libcuda), or null when the driver lacks it.
+void *driver_fn(const char *name);
+
+// Makes the device that owns the caller's tensors current for one API call
+// and, when that meant a switch, restores the context that was current on
+// entry (a primary context, a driver-API context the caller pushed, or none)
+// when it goes out of scope, on every return path.
+class DeviceGuard {
+  public:
+    DeviceGuard() = default;
+    DeviceGuard(const DeviceGuard &) = delete;
+    DeviceGuard &operator=(const DeviceGuard &) = delete;
+    ~DeviceGuard();
+    // Switch to `dev` (no-op when it is current already).  False when the
+    // switch failed; the caller's context is restored either way.
+    bool use(int dev);
+
+  private:
+    bool switched_ = false;
+    CUcontext saved_ = nullptr;
+};
+
 // TMA descriptor of a bf16 [T, H, D] tensor with a box of {box_x, 1, 64}
 // (innermost first) and a 32/64/128-byte swizzle (0 = none).
 bool make_tmap_bf16_3d(CUtensorMap *m, const void *base, int T, int H, int D, int box_x,
@@ -98,6 +129,10 @@ template <> __device__ __forceinline__ float from_f32<float>(float x) { return x
 template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
     return __float2bfloat16_rn(x);
 }
+
+// In-chunk cumulative decay exp(-80): the smallest Gam the chunked
+// factorisation exp(g_r - g_s) = Gam_r / Gam_s keeps inside fp32 range.
+constexpr float kMinChunkDecay = 1.8048513e-35f;
 
 // Record the first error code seen by any thread; later codes are dropped.
 __device__ __forceinline__ void set_status(int32_t *status, int32_t code) {

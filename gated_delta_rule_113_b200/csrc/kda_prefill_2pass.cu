@@ -100,9 +100,17 @@ __device__ __forceinline__ Item item_of(long long m, int H, const int32_t *chunk
         if (chunk_off[mid] <= g) lo = mid;
         else hi = mid;
     }
-    const int j = g - chunk_off[lo];
-    it.c0 = cu[lo] + j * kChunk;
-    it.L = min(kChunk, cu[lo + 1] - it.c0);
+    // 64-bit: with saturated offsets (overlapping sequences) j can exceed
+    // the sequence's chunk count; such an item gets no rows (L = 0).
+    const long long c0 = (long long)cu[lo] + (long long)(g - chunk_off[lo]) * kChunk;
+    const long long L = (long long)cu[lo + 1] - c0;
+    if (c0 < 0 || c0 > 0x7fffffffLL || L <= 0) {
+        it.c0 = 0;
+        it.L = 0;
+    } else {
+        it.c0 = (int)c0;
+        it.L = (int)(L < kChunk ? L : kChunk);
+    }
     return it;
 }
 
@@ -248,7 +256,7 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     grid_launch_dependents();
     grid_dependency_wait();
     long long total = (long long)p.chunk_off[p.N] * p.H;
-    if (total > p.slots) {   // overlapping (malformed) sequences: never write past the workspace
+    if (total < 0 || total > p.slots) {   // overlapping (malformed) sequences: never write past the workspace
         if (blockIdx.x == 0 && threadIdx.x == 0) set_status(p.status, KDA_ERR_SEQLENS);
         total = p.slots;
     }
@@ -467,7 +475,7 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             }
             if (t == 0) KDA_TRACE1(i, 1);
             prep_chunk(t, sbase + Ly::kKQ + s * 32768, sbase + Ly::kKI + s * 16384, sGP, sSUF,
-                       sGL + s * 128, sB + s * 64, p.beta, it.c0, it.L, p.H, it.h, 1);
+                       sGL + s * 128, sB + s * 64, p.beta, it.c0, it.L, p.H, it.h, 1, p.status);
             if (t == 0) KDA_TRACE1(i, 2);
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[kbKqFull + s]);
@@ -667,7 +675,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
     }
     const int nchunks = (t1 - t0 + kChunk - 1) / kChunk;
     const int g0 = p.chunk_off[seq];
-    if ((long long)(g0 + nchunks) * p.H > p.slots) {
+    if (g0 < 0 || ((long long)g0 + nchunks) * p.H > p.slots) {
         if (tid == 0) set_status(p.status, KDA_ERR_SEQLENS);
         return;
     }

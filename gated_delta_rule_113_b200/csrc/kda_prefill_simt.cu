@@ -112,14 +112,21 @@ prefill_simt_kernel(const TIO *__restrict__ q, const TIO *__restrict__ k,
         __syncthreads();  // previous chunk fully consumed
 
         // ---- gates, scaled operands: one thread per key channel ----------
+        // exp(g) and exp(-g) stay in fp32 range while the in-chunk cumulative
+        // log-decay g is in [-80, 0]; a log_alpha above 0 or not finite, or a
+        // g below -80, records KDA_ERR_DECAY (this chain's results are then
+        // unspecified, nothing is read or written out of range).
         if (tid < DK) {
             const int c = tid;
             float g = 0.f;
+            bool bad = false;
             for (int r = 0; r < kChunk; ++r) {
                 float qg = 0.f, kg = 0.f, ki = 0.f;
                 if (r < L) {
                     const size_t row = ((size_t)(c0 + r) * H + h) * DK + c;
-                    g += to_f32(la[row]);
+                    const float lav = to_f32(la[row]);
+                    bad |= !(lav <= 0.f);
+                    g += lav;
                     const float kv = to_f32(k[row]);
                     const float e = expf(g);
                     qg = to_f32(q[row]) * e;
@@ -131,6 +138,8 @@ prefill_simt_kernel(const TIO *__restrict__ q, const TIO *__restrict__ k,
                 sm.Ki[r * LDK + c] = ki;
             }
             sm.gl[c] = expf(g);
+            bad |= !(g >= -80.f);
+            if (bad) set_status(status, KDA_ERR_DECAY);
         } else {
             for (int i = tid - DK; i < kChunk * kVs; i += kThreads - DK) {
                 const int r = i / kVs, j = i % kVs;

@@ -253,7 +253,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             if (!wait_or_abort(&bars[bRawFull + s], (n >> 1) & 1, abort_flag, p.status)) break;
             if (t == 0) KDA_TRACE_EVENT(n, 1);
             prep_chunk(t, sbase + Ly::kKQ + s * 32768, sbase + Ly::kKI + s * 16384, sGP, sSUF,
-                       sGL + s * 128, sB + s * 64, p.beta, c0, L, p.H, h, kBarPrep);
+                       sGL + s * 128, sB + s * 64, p.beta, c0, L, p.H, h, kBarPrep, p.status);
             __syncwarp();
             if (t == 0) KDA_TRACE_EVENT(n, 2);
             if (lane == 0) mbar_arrive(&bars[bKqFull + s]);

@@ -114,11 +114,15 @@ __device__ __forceinline__ uint64_t kmaj_step(int ks, uint32_t atom) {
 // alpha = 2^(log_alpha log2 e) once per element; Gam_r is the running product
 // of alpha inside the chunk and 1/Gam_r = (1/Gam_L) prod_{j>r} alpha_j, so no
 // element needs a second exponential or a division.
+//
+// The factorisation needs every log_alpha <= 0 (finite) and every channel's
+// Gam_L >= exp(-80); a chunk that breaks either records KDA_ERR_DECAY in
+// `status` (its chain's results are then unspecified; nothing else changes).
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void prep_chunk(int t, uint32_t kq_stage, uint32_t ki_stage,
                                            float *sGP, float *sSUF, float *sGL_s, float *sB_s,
                                            const __nv_bfloat16 *beta, int c0, int L, int H, int h,
-                                           uint32_t bar_id) {
+                                           uint32_t bar_id, int32_t *status) {
     const int cg = t & 15, rg = t >> 4;   // 8-channel group, 4-row group
     const int a = cg >> 3, ch = cg & 7;
     const uint32_t kq = kq_stage + a * 16384;
@@ -129,6 +133,7 @@ __device__ __forceinline__ void prep_chunk(int t, uint32_t kq_stage, uint32_t ki
         beta_r = __bfloat162float(beta[(size_t)(c0 + t - 128) * H + h]);
     // pass 0: alpha; in-group prefix and suffix products
     float pre[4][8], suf[4][8];
+    bool bad = false;   // a log_alpha above 0 or not finite
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const int r = rg * 4 + i;
@@ -138,6 +143,7 @@ __device__ __forceinline__ void prep_chunk(int t, uint32_t kq_stage, uint32_t ki
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
             const float la = (e & 1) ? bf16hi(w4[e >> 1]) : bf16lo(w4[e >> 1]);
+            bad |= !(la <= 0.f);
             pre[i][e] = ex2_approx(la * kLog2e);   // alpha for now
         }
     }
@@ -175,6 +181,7 @@ __device__ __forceinline__ void prep_chunk(int t, uint32_t kq_stage, uint32_t ki
             px *= gv[g];
         }
         sGL_s[t] = px;
+        bad |= !(px >= kMinChunkDecay);   // also catches a NaN product
         float sx = rcp_approx(px);   // 1/Gam_L, once per channel
 #pragma unroll
         for (int g = 15; g >= 0; --g) {
@@ -185,6 +192,7 @@ __device__ __forceinline__ void prep_chunk(int t, uint32_t kq_stage, uint32_t ki
         sB_s[t - 128] = beta_r;
     }
     named_bar(bar_id, kPrepThreads);
+    if (__any_sync(0xffffffffu, bad) && (t & 31) == 0) set_status(status, KDA_ERR_DECAY);
     // pass 1: Gam_r = pre_group * pre[i]; 1/Gam_r = (1/Gam_L) suf_group suf[i]
     float ef[8], ci[8];
     {

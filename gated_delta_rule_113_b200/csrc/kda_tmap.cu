@@ -25,7 +25,48 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+typedef CUresult (*CtxSetCurrentFn)(CUcontext);
+
 }  // namespace
+
+void *driver_fn(const char *name) {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint(name, &ptr, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    return ptr;
+}
+
+bool DeviceGuard::use(int dev) {
+    int cur = -1;
+    if (cudaGetDevice(&cur) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    if (cur == dev) return true;
+    if (!switched_) {
+        static CtxGetCurrentFn get_cur =
+            reinterpret_cast<CtxGetCurrentFn>(driver_fn("cuCtxGetCurrent"));
+        if (!get_cur || get_cur(&saved_) != CUDA_SUCCESS) return false;
+        switched_ = true;
+    }
+    if (cudaSetDevice(dev) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return true;
+}
+
+DeviceGuard::~DeviceGuard() {
+    if (!switched_) return;
+    static CtxSetCurrentFn set_cur =
+        reinterpret_cast<CtxSetCurrentFn>(driver_fn("cuCtxSetCurrent"));
+    if (set_cur) set_cur(saved_);
+}
 
 bool make_tmap_bf16_3d(CUtensorMap *m, const void *base, int T, int H, int D, int box_x,
                        int swizzle_bytes) {

@@ -16,17 +16,22 @@ __global__ void __launch_bounds__(1024) varlen_index_kernel(const int32_t *__res
                                                             int32_t *order, int32_t *chunk_off,
                                                             int32_t *work_ctr) {
     __shared__ int32_t s_len[kSortMax];
-    __shared__ int32_t s_part[1024];
+    __shared__ long long s_part[1024];
     __shared__ int s_bad;
+    __shared__ int s_sat;
     const int tid = threadIdx.x;
     sm100::grid_launch_dependents();   // the key-side pass may start its set-up now
+    if (tid == 0) s_sat = 0;
     if (chunk_off) {
         // chunk_off[n] = sum_{i<n} ceil(len_i / 64) (malformed sequences count
         // as empty): each thread scans a contiguous segment, then the block
-        // scans the segment totals.
+        // scans the segment totals.  Well-formed offsets keep the sums below
+        // T / 64 + N; overlapping (malformed) ones can push them past int32,
+        // so they are formed in 64 bits and stored saturated at INT32_MAX,
+        // which every consumer rejects as out of range.
         const int seg = (N + blockDim.x - 1) / blockDim.x;
         const int lo = tid * seg, hi = min(N, lo + seg);
-        int sum = 0;
+        long long sum = 0;
         for (int i = lo; i < hi; ++i) {
             const int a = cu[i], b = cu[i + 1];
             if (a >= 0 && b >= a && b <= T) sum += (b - a + kChunk - 1) / kChunk;
@@ -35,27 +40,36 @@ __global__ void __launch_bounds__(1024) varlen_index_kernel(const int32_t *__res
         __syncthreads();
         // exclusive scan of the segment totals (Hillis-Steele, log2(1024) steps)
         for (int off = 1; off < (int)blockDim.x; off <<= 1) {
-            const int x = tid >= off ? s_part[tid - off] : 0;
+            const long long x = tid >= off ? s_part[tid - off] : 0;
             __syncthreads();
             s_part[tid] += x;
             __syncthreads();
         }
-        const int incl = s_part[tid];
+        const long long incl = s_part[tid];
         __syncthreads();
         s_part[tid] = incl - sum;
         __syncthreads();
-        int run = s_part[tid];
+        long long run = s_part[tid];
+        bool sat = false;
+        auto store = [&](int i, long long x) {
+            if (x > 0x7fffffffLL) {
+                x = 0x7fffffffLL;
+                sat = true;
+            }
+            chunk_off[i] = (int32_t)x;
+        };
         for (int i = lo; i < hi; ++i) {
-            chunk_off[i] = run;
+            store(i, run);
             const int a = cu[i], b = cu[i + 1];
             if (a >= 0 && b >= a && b <= T) run += (b - a + kChunk - 1) / kChunk;
         }
-        if (hi == N && lo < hi) chunk_off[N] = run;
+        if (hi == N && lo < hi) store(N, run);
         if (N == 0 && tid == 0) chunk_off[0] = 0;
+        if (sat) s_sat = 1;
         __syncthreads();
     }
     if (tid == 0) {
-        s_bad = (cu[0] != 0 || cu[N] != T) ? 1 : 0;
+        s_bad = (cu[0] != 0 || cu[N] != T || s_sat) ? 1 : 0;
         if (work_ctr) *work_ctr = 0;   // the key-side pass claims items from here
     }
     __syncthreads();

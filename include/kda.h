@@ -32,7 +32,15 @@
  *     chunk needs the in-chunk cumulative log-decay of every channel to stay
  *     above -80 (fp32 exponent range): e.g. alpha >= exp(-1.25) per token at
  *     chunk 64.  That is the lower bound on the decay the method relies on;
- *     the library does not clamp log_alpha.
+ *     the library does not clamp log_alpha.  The chunked kernels check it:
+ *     a log_alpha above 0 or not finite, or a channel whose cumulative
+ *     log-decay over one chunk falls below -80, records KDA_ERR_DECAY in the
+ *     workspace status word (no trap, nothing read or written out of range).
+ *     The outputs and final state of the (sequence, head) chains that hold
+ *     such a chunk are then unspecified; every other chain is unaffected.
+ *   - Every entry point makes the device that owns its tensors current for
+ *     the launches and restores the caller's current context (device) before
+ *     it returns, on success and on error.
  */
 #ifndef KDA_H
 #define KDA_H
@@ -44,7 +52,7 @@
 extern "C" {
 #endif
 
-#define KDA_ABI_VERSION 3
+#define KDA_ABI_VERSION 4
 
 typedef enum kda_status {
     KDA_OK = 0,
@@ -55,7 +63,8 @@ typedef enum kda_status {
     KDA_ERR_CUDA = 5,         /* a CUDA runtime call or kernel launch failed      */
     KDA_ERR_TIMEOUT = 6,      /* a bounded device-side wait gave up               */
     KDA_ERR_SEQLENS = 7,      /* device saw cu_seqlens not 0..total_tokens monotone */
-    KDA_ERR_SLOT = 8          /* device saw a snapshot-pool slot outside the pool */
+    KDA_ERR_SLOT = 8,         /* device saw a snapshot-pool slot outside the pool */
+    KDA_ERR_DECAY = 9         /* device saw a gate outside the chunked form's range */
 } kda_status;
 
 typedef enum kda_dtype {
@@ -158,14 +167,19 @@ kda_status kda_forward(const void *q, const void *k, const void *v,
  *   - p->num_seqs > KDA_NOALLOC_MAX_SEQS is rejected with
  *     KDA_ERR_UNSUPPORTED before anything is enqueued;
  *   - the first call on a device looks up the array's device address (with
- *     that device current); make that first call before any stream capture;
+ *     that device current) and caches it for the CUDA context then current;
+ *     a call under another context of the device (a driver-API context the
+ *     caller pushed, or a primary context re-created after cudaDeviceReset)
+ *     looks it up again; make the first call in a context before any stream
+ *     capture;
  *   - every call shares the array and rewrites it before use; calls whose
  *     work overlaps on the GPU race on it, so order them on one stream;
  *   - it allocates nothing (no cudaMalloc, cudaFree or allocating library
  *     call) and runs exactly the kernels of kda_forward.
  *
- * Returns the same codes as kda_forward.  Malformed cu_seqlens contents are
- * still skipped safely on the device, but this path has no status readback.
+ * Returns the same codes as kda_forward.  What only the device can see
+ * (malformed cu_seqlens, a bounded wait that gave up, an out-of-range gate)
+ * goes to the array's status word; read it with kda_forward_noalloc_status.
  */
 #define KDA_NOALLOC_MAX_SEQS 16384
 kda_status kda_forward_noalloc(const void *q, const void *k, const void *v,
@@ -173,6 +187,17 @@ kda_status kda_forward_noalloc(const void *q, const void *k, const void *v,
                                const float *S0, const int32_t *cu_seqlens,
                                void *out, float *S_final, const kda_params *p,
                                void *stream);
+
+/*
+ * kda_forward_noalloc_status -- synchronise `stream`, then copy into *status
+ * the device status word that the last kda_forward_noalloc call on the device
+ * owning `device_ptr` (any device pointer of that call, e.g. its cu_seqlens)
+ * left in the library's scratch array: KDA_OK, or the first KDA_ERR_* code
+ * the device recorded.  Like kda_forward_noalloc it allocates nothing.
+ * Returns KDA_ERR_INVALID for NULL arguments or a host pointer, KDA_ERR_CUDA
+ * if the synchronisation or the copy fails.
+ */
+kda_status kda_forward_noalloc_status(const void *device_ptr, int32_t *status, void *stream);
 
 /*
  * kda_forward_snapshots -- kda_forward that also keeps the recurrent state in
@@ -273,8 +298,9 @@ kda_status kda_decode_multi(const void *q, const void *k, const void *v,
  * for this problem; 0 when `p` is NULL or invalid.  Must be 256-byte
  * aligned; needs no initialisation.  About
  * 2 (total_tokens / 64 + N) * H * Dk * Dv * 4 bytes of states (one every 32
- * tokens) plus N * H * (Dv / 32) * (32 * Dk * 32 + 1024) * 4 bytes of per-CTA
- * scratch.
+ * tokens), N * H * (Dv / 32) * (32 * Dk * 32 + 1024) * 4 bytes of per-CTA
+ * scratch and (Dv / 32) * total_tokens * H * (3 Dk + 1) * 4 bytes of
+ * per-slice partial sums.
  */
 size_t kda_backward_workspace_size(const kda_params *p);
 
@@ -297,9 +323,10 @@ size_t kda_backward_workspace_size(const kda_params *p);
  *   workspace  ws_bytes >= kda_backward_workspace_size(p), 256-byte aligned
  *
  * All gradients are fp32 whatever io_dtype and gate_dtype; the arithmetic is
- * fp32 on CUDA cores.  dq, dk, dlog_alpha and dbeta sum partial results of
- * the 32-wide value slices with atomic adds, so their last bits can differ
- * from one call to the next; dv and dS0 are written once.  The states are
+ * fp32 on CUDA cores.  dq, dk, dlog_alpha and dbeta are sums over the 32-wide
+ * value slices: each slice's partial sum goes to the workspace and a second
+ * kernel adds them in slice order, so repeated calls on the same inputs give
+ * bitwise identical gradients (no atomics anywhere).  The states are
  * recomputed (the forward runs twice: once to keep the state every 32
  * tokens, once per 32 tokens in reverse order),
  * so no state from kda_forward is needed.  The recurrence is evaluated token by
@@ -307,8 +334,8 @@ size_t kda_backward_workspace_size(const kda_params *p);
  * this file does not apply to this entry point.  `flags` is ignored.  Outputs may
  * not overlap inputs or each other.  Errors as kda_forward: host validation
  * codes, KDA_ERR_CUDA if a launch fails, KDA_ERR_SEQLENS recorded in the
- * workspace status word for malformed cu_seqlens (those sequences' gradients
- * are left as zero or unwritten).
+ * workspace status word for malformed cu_seqlens (the gradients are then
+ * unspecified; nothing is read or written out of range).
  */
 kda_status kda_backward(const void *q, const void *k, const void *v,
                         const void *log_alpha, const void *beta,

@@ -5,6 +5,8 @@ import ctypes
 import os
 import re
 
+import numpy as np
+
 import pytest
 
 import gated_delta_rule_113_b200 as kda
@@ -31,12 +33,12 @@ def test_library_loads_and_exports_every_declared_symbol():
     assert set(kda.EXPORTED_SYMBOLS) <= set(declared)
     text = open(os.path.join(HEADER, "kda.h")).read()
     assert lib.kda_abi_version() == int(re.search(r"#define KDA_ABI_VERSION (\d+)", text).group(1))
-    assert lib.kda_abi_version() == 3
+    assert lib.kda_abi_version() == 4
 
 
 def test_status_strings():
     lib = kda.load_library()
-    for code in range(0, 9):
+    for code in range(0, 10):
         assert lib.kda_status_string(code).startswith(b"KDA_")
     assert lib.kda_status_string(1234) == b"KDA_ERR_UNKNOWN"
 
@@ -191,10 +193,40 @@ def test_backward_workspace_size():
     lib = kda.load_library()
     p = _params()
     n = lib.kda_backward_workspace_size(ctypes.byref(p))
-    # the kept states and the per-CTA scratch dominate
+    # the kept states, the per-CTA scratch and the per-slice partial sums
     T, N, H, Dk, Dv = p.total_tokens, p.num_seqs, p.H, p.Dk, p.Dv
     states = 2 * ((T + 63) // 64 + N) * H * Dk * Dv * 4          # one every 32 tokens
     scratch = N * H * (Dv // 32) * (32 * Dk * 32 + 32 * 32) * 4
-    assert states + scratch <= n <= states + scratch + 4096 + 8 * N
+    part = (Dv // 32) * T * H * (3 * Dk + 1) * 4
+    assert states + scratch + part <= n <= states + scratch + part + 4096 + 8 * N + 256 * Dv
     assert lib.kda_backward_workspace_size(ctypes.byref(_params(Dk=96))) == 0
     assert lib.kda_backward_workspace_size(None) == 0
+
+
+def test_chunk_offset_scan_saturates_instead_of_wrapping():
+    """The varlen index counts the chunks of every well-formed (start, end)
+    pair of cu_seqlens.  With overlapping (malformed) offsets the pairs need
+    not tile the token axis, so the count can pass 2^31: 32768 pairs, every
+    other one spanning [0, 2^24), give 2^14 * 2^18 = 2^32 chunks.  A 32-bit
+    running sum wraps there (to 0 here, negative on the way), which the chain
+    kernel's bound check of g0 + nchunks against the packet count would not
+    catch; the kernel's 64-bit sum stored saturated at INT32_MAX always fails
+    that check.  This restates the kernel's scan in numpy at that size."""
+    T = 1 << 24
+    cu = np.tile(np.array([0, T], dtype=np.int64), 1 << 14)
+    cu = np.append(cu, 0)                         # 32768 pairs, every other one [0, T)
+    a, b = cu[:-1], cu[1:]
+    ok = (a >= 0) & (b >= a) & (b <= T)
+    chunks = np.where(ok, (b - a + 63) // 64, 0)
+    run64 = np.concatenate([[0], np.cumsum(chunks)])
+    assert run64[-1] == 1 << 32
+    wrapped = run64.astype(np.uint64).astype(np.uint32).astype(np.int32)
+    assert (wrapped < 0).any() and wrapped[-1] == 0   # what an int32 scan would store
+    stored = np.minimum(run64, 2**31 - 1).astype(np.int32)
+    H, slots = 1, ((T + 63) // 64 + len(a)) * 1     # packets the workspace holds
+    n_chunks = chunks
+    g0 = stored[:-1]
+    rejected = (g0 < 0) | ((g0.astype(np.int64) + n_chunks) * H > slots)
+    # every sequence whose offset passed the workspace is rejected, none wraps back in
+    assert rejected[ok & (run64[:-1] + n_chunks > slots)].all()
+    assert (stored >= 0).all()

@@ -290,3 +290,123 @@ def test_bounded_wait_times_out_and_the_context_stays_usable():
                             d["cu_seqlens"], workspace=ws)
     assert kda.workspace_status(ws) == 0
     _check(inp, out2, sf2, torch.bfloat16)
+
+
+# ------------------------------------------------- decay outside the chunk range
+KDA_ERR_DECAY = 9
+
+
+@pytest.mark.parametrize("path", PATHS)
+@pytest.mark.parametrize("bad", ["too_steep", "positive", "nan"])
+def test_decay_out_of_range_is_reported_and_other_chains_stay_exact(path, bad):
+    """The chunked kernels need log_alpha <= 0 and an in-chunk cumulative
+    log-decay above -80.  A chunk that breaks this records KDA_ERR_DECAY in the
+    workspace status word; the other (sequence, head) chains still match the
+    oracle (only the offending chain's results are unspecified)."""
+    w = WORKLOADS[1]
+    lens = [200, 150, 70]
+    inp = forward_inputs(w, lengths=lens, H=2, s0=True)
+    la = inp["log_alpha"].clone()
+    r0 = lens[0] + 64            # second chunk of sequence 1, head 1
+    if bad == "too_steep":       # -2 per token: cumulative -128 over the chunk
+        la[r0:r0 + 64, 1, :] = -2.0
+    elif bad == "positive":
+        la[r0 + 5, 1, 7] = 0.25
+    else:
+        la[r0 + 9, 1, 3] = float("nan")
+    inp["log_alpha"] = la
+    d = to_dev(inp)
+    n_ws = kda.forward_workspace_size(len(lens), sum(lens), 2, 128, 128)
+    ws = torch.empty(max(n_ws, 1 << 16), dtype=torch.uint8, device="cuda")
+    out, sf = kda.forward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["S0"],
+                          d["cu_seqlens"], workspace=ws, force_simt=path == "simt",
+                          fused_tc=path == "fused_tc")
+    assert kda.workspace_status(ws) == KDA_ERR_DECAY
+    # every chain except (sequence 1, head 1) against the oracle
+    cu = inp["cu_seqlens"].numpy()
+    for n in range(len(lens)):
+        for h in range(2):
+            if (n, h) == (1, 1):
+                continue
+            sl = slice(int(cu[n]), int(cu[n + 1]))
+            one = {k: inp[k][sl, h:h + 1].contiguous() for k in ("q", "k", "v", "log_alpha", "beta")}
+            one["S0"] = inp["S0"][n:n + 1, h:h + 1].contiguous()
+            one["cu_seqlens"] = torch.tensor([0, lens[n]], dtype=torch.int32)
+            ro, rs = _oracle(one)
+            go = as_np(out[sl, h:h + 1])
+            gs = as_np(sf[n:n + 1, h:h + 1])
+            assert err(go, ro, torch.bfloat16) <= tol(torch.bfloat16), (n, h)
+            assert err(gs, rs, torch.bfloat16) <= tol(torch.bfloat16), (n, h)
+
+
+def test_in_range_decay_leaves_the_status_ok():
+    w = WORKLOADS[1]
+    inp = forward_inputs(w, lengths=[64, 64], H=1)
+    inp["log_alpha"] = torch.full_like(inp["log_alpha"], -1.2)   # cumulative -76.8 per chunk
+    d = to_dev(inp)
+    n_ws = kda.forward_workspace_size(2, 128, 1, 128, 128)
+    ws = torch.empty(n_ws, dtype=torch.uint8, device="cuda")
+    out, sf = kda.forward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["S0"],
+                          d["cu_seqlens"], workspace=ws)
+    assert kda.workspace_status(ws) == 0
+    _check(inp, out, sf, torch.bfloat16)
+
+
+# ------------------------------------------------- the caller's current device
+def _driver():
+    lib = ctypes.CDLL("libcuda.so.1")
+    lib.cuCtxGetCurrent.argtypes = [ctypes.POINTER(ctypes.c_void_p)]
+    return lib
+
+
+def _current_ctx(drv):
+    c = ctypes.c_void_p()
+    assert drv.cuCtxGetCurrent(ctypes.byref(c)) == 0
+    return c.value
+
+
+def test_entry_points_leave_the_callers_device_and_context_current():
+    """Called straight through the C ABI (no Python device guard around it),
+    every entry point returns with the caller's device and CUDA context still
+    current.  On a machine with two GPUs the call also runs with the caller on
+    another device than the tensors'."""
+    lib = kda.load_library()
+    drv = _driver()
+    w = WORKLOADS[1]
+    inp = forward_inputs(w, lengths=[100, 40], H=2, s0=True)
+    n_gpus = torch.cuda.device_count()
+    for tensor_dev, caller_dev in [(0, 0)] + ([(1, 0), (0, 1)] if n_gpus > 1 else []):
+        dev = torch.device("cuda", tensor_dev)
+        d = to_dev(inp, dev)
+        T, H, Dk = d["q"].shape
+        out = torch.empty((T, H, 128), dtype=torch.bfloat16, device=dev)
+        sf = torch.empty((2, H, Dk, 128), dtype=torch.float32, device=dev)
+        p = kda.Params(2, T, H, Dk, 128, 64, 1, 1, 0)
+        n_ws = lib.kda_forward_workspace_size(ctypes.byref(p))
+        ws = torch.empty(n_ws, dtype=torch.uint8, device=dev)
+        ptr = lambda t: ctypes.c_void_p(t.data_ptr())
+        torch.cuda.set_device(caller_dev)
+        torch.cuda.synchronize(caller_dev)
+        ctx0 = _current_ctx(drv)
+        stream = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+        rc = lib.kda_forward(ptr(d["q"]), ptr(d["k"]), ptr(d["v"]), ptr(d["log_alpha"]),
+                             ptr(d["beta"]), ptr(d["S0"]), ptr(d["cu_seqlens"]), ptr(out),
+                             ptr(sf), ctypes.byref(p), ptr(ws), n_ws, stream)
+        assert rc == 0
+        assert torch.cuda.current_device() == caller_dev
+        assert _current_ctx(drv) == ctx0
+        st = ctypes.c_int32(-1)
+        assert lib.kda_workspace_status(ptr(ws), ctypes.byref(st), stream) == 0 and st.value == 0
+        assert torch.cuda.current_device() == caller_dev
+        assert _current_ctx(drv) == ctx0
+        # an error return (misaligned workspace) restores it too
+        bad_ws = ctypes.c_void_p(ws.data_ptr() + 16)
+        rc = lib.kda_forward(ptr(d["q"]), ptr(d["k"]), ptr(d["v"]), ptr(d["log_alpha"]),
+                             ptr(d["beta"]), ptr(d["S0"]), ptr(d["cu_seqlens"]), ptr(out),
+                             ptr(sf), ctypes.byref(p), bad_ws, n_ws - 16, stream)
+        assert rc == 4
+        assert torch.cuda.current_device() == caller_dev
+        assert _current_ctx(drv) == ctx0
+        torch.cuda.set_device(0)
+        ro, rs = _oracle(inp)
+        assert err(as_np(out), ro, torch.bfloat16) <= tol(torch.bfloat16)

@@ -25,6 +25,16 @@ constexpr int kPrepThreads = 256;  // threads running prep_chunk
 constexpr int kSolveThreads = 128; // threads running solve_chunk (4 warps, lane quarters 0..3)
 constexpr float kLog2e = 1.4426950408889634f;
 
+// Where a bounded wait gave up, for diagnosis: the first timeout of a call
+// stores (barrier's shared-memory offset | thread index << 16) in the word
+// after the status word's 32-byte line (status[8]) and the block index in
+// status[9].  Written only on that failure path.
+__device__ __forceinline__ void note_timeout(int32_t *status, const uint64_t *bar) {
+    if (!status) return;
+    const int32_t tag = (int32_t)((smem_u32(bar) & 0xFFFFu) | ((uint32_t)threadIdx.x << 16));
+    if (atomicCAS(status + 8, 0, tag) == 0) status[9] = (int32_t)blockIdx.x;
+}
+
 // Bounded wait on an mbarrier phase.  Waiting threads stay suspended in
 // try_wait (no issue slots taken from working warps) and wake when the phase
 // completes; a wait that outlasts 2 s gives up, records KDA_ERR_TIMEOUT and
@@ -40,6 +50,7 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity,
     }
     *abort_flag = 1;
     set_status(status, KDA_ERR_TIMEOUT);
+    note_timeout(status, bar);
     return false;
 }
 
@@ -60,6 +71,7 @@ __device__ __forceinline__ bool spin_or_abort(uint64_t *bar, uint32_t parity,
     }
     *abort_flag = 1;
     set_status(status, KDA_ERR_TIMEOUT);
+    note_timeout(status, bar);
     return false;
 }
 

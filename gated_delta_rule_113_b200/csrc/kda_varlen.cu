@@ -80,7 +80,11 @@ __global__ void __launch_bounds__(1024) varlen_index_kernel(const int32_t *__res
         if (N <= kSortMax) s_len[i] = ok ? (b - a) : 0;
     }
     __syncthreads();
-    if (tid == 0) *status = s_bad ? KDA_ERR_SEQLENS : KDA_OK;
+    if (tid == 0) {
+        *status = s_bad ? KDA_ERR_SEQLENS : KDA_OK;
+        status[8] = 0;   // where a bounded wait gave up, if one does (see note_timeout)
+        status[9] = 0;
+    }
     if (N > kSortMax) {
         for (int i = tid; i < N; i += blockDim.x) order[i] = i;
         return;

@@ -573,52 +573,79 @@ def bench_kda(args):
 
 def bench_backward(kda, dev, stream, world, w, d, T, N, H, Dk, Dv, steps=3):
     """kda_backward on the prefill workload: dL/d out random, dL/dS_final and
-    dL/dS0 included.  One call = the varlen index and the backward kernel.
+    dL/dS0 included.  Two paths, each timed: the chunked tensor-core one (the
+    default for bf16 with d = 128: the forward's two passes keeping every
+    chunk's entering state, the reverse chain, the gradient assembly) and the
+    fp32 CUDA-core one (token-level, 1e-4 accurate).
 
-    Algorithmic flops per token-head, counted once (no recomputation): the
+    Algorithmic work per token-head, counted once, is the same for both: the
     forward step 5 Dk Dv (decay, P^T k, rank-one write) and the reverse step
-    16 Dk Dv (dq, the read-out outer product, G u, G^T k, P du, dP, the decay
-    row sums and the decayed G).  The kernel runs on CUDA cores in fp32, so its
-    roof is the fp32 FMA rate: 148 SMs x 128 lanes x 2 flop x the SM clock."""
+    16 Dk Dv flop; bytes: q, k, v, log_alpha, beta and d_out read once, dq,
+    dk, dv, dlog_alpha (fp32) and dbeta written once, plus S0, dS_final and
+    dS0.  At ~100 flop per byte both paths are bound by HBM under this count;
+    the CUDA-core path's own roof is the fp32 FMA rate (148 SMs x 128 lanes x
+    2 flop x the SM clock)."""
     g = torch.Generator(device=dev).manual_seed(5)
     d_out = torch.randn((T, H, Dv), generator=g, device=dev).to(w.torch_dtype)
     dSf = torch.randn((N, H, Dk, Dv), generator=g, device=dev)
-    ws = torch.empty(kda.backward_workspace_size(N, T, H, Dk, Dv, w.torch_dtype),
-                     dtype=torch.uint8, device=dev)
-
-    def call():
-        return kda.backward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["S0"],
-                            d["cu_seqlens"], d_out=d_out, dS_final=dSf, workspace=ws)
-
-    for _ in range(2):
-        call()
-    if kda.workspace_status(ws) != 0:
-        raise RuntimeError("device status not OK after the backward warm-up")
-    barrier(world)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(steps):
-        call()
-    e1.record(stream)
-    barrier(world)
-    ms = max_over_ranks(e0.elapsed_time(e1), world) / steps
+    peaks, kind = load_peaks()
     flops = 21.0 * Dk * Dv * T * H
-    sms = torch.cuda.get_device_properties(dev).multi_processor_count
-    peaks, _ = load_peaks()
-    alu_tflops = sms * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
-    achieved = flops / (ms * 1e-3) / 1e12
     io = _es(w.torch_dtype)
-    moved = T * H * (3 * Dk * io + Dv * io + 2 + Dv * io + 3 * Dk * 4 + Dv * 4 + 4) + \
-        2 * N * H * Dk * Dv * 4
-    return {"workload": w.name, "value": world * T / (ms * 1e-3), "unit": "tokens/s",
-            "ms_per_call": ms, "gpu_launches": 2 * steps,
-            "grads": "dq, dk, dv, dlog_alpha, dbeta, dS0 (fp32); dS_final given",
-            "roofline": {"bound": "alu", "achieved": achieved, "peak": alu_tflops,
-                         "unit": "TFLOP/s", "frac": achieved / alu_tflops,
-                         "traffic": traffic_record("kda_backward"),
-                         "peak_kind": "derived: fp32 FMA, SMs x 128 x 2 x max SM clock",
-                         "algorithmic_flops": flops, "algorithmic_bytes": moved,
-                         "hbm_frac_algorithmic": moved / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}}
+    moved = T * H * (3 * Dk * io + Dv * io + io + Dv * io + 3 * Dk * 4 + Dv * 4 + 4) + \
+        3 * N * H * Dk * Dv * 4
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    alu_tflops = sms * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+
+    def timed(force_simt, reps):
+        ws = torch.empty(kda.backward_workspace_size(N, T, H, Dk, Dv, w.torch_dtype,
+                                                     force_simt=force_simt),
+                         dtype=torch.uint8, device=dev)
+
+        def call():
+            return kda.backward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["S0"],
+                                d["cu_seqlens"], d_out=d_out, dS_final=dSf, workspace=ws,
+                                force_simt=force_simt)
+
+        for _ in range(2):
+            call()
+        if kda.workspace_status(ws) != 0:
+            raise RuntimeError("device status not OK after the backward warm-up")
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            call()
+        e1.record(stream)
+        barrier(world)
+        return max_over_ranks(e0.elapsed_time(e1), world) / reps
+
+    tc = w.torch_dtype == torch.bfloat16 and Dk == 128 and Dv == 128
+    ms_tc = timed(False, 10) if tc else None
+    ms_f32 = timed(True, steps)
+    out = {"workload": w.name,
+           "grads": "dq, dk, dv, dlog_alpha, dbeta, dS0 (fp32); dS_final given",
+           "algorithmic_flops": flops, "algorithmic_bytes": moved}
+    if tc:
+        gbs = moved / (ms_tc * 1e-3) / 1e9
+        out["chunked_tc"] = {
+            "value": world * T / (ms_tc * 1e-3), "unit": "tokens/s", "ms_per_call": ms_tc,
+            "gpu_launches": 6 * 10,
+            "kernels": "varlen_index, kside, chain (state store), rchain, assemble",
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm_gbs"], "traffic": traffic_record("kda_backward_tc"),
+                         "peak_kind": f"{kind} HBM copy",
+                         "tensor_frac_algorithmic": flops / (ms_tc * 1e-3) / 1e12 / peaks["bf16_tflops"]},
+            "tolerance": "bf16: ||err||_F / ||oracle||_F <= 2e-2 per gradient"}
+    achieved = flops / (ms_f32 * 1e-3) / 1e12
+    out["fp32_cuda_cores"] = {
+        "value": world * T / (ms_f32 * 1e-3), "unit": "tokens/s", "ms_per_call": ms_f32,
+        "gpu_launches": 3 * steps,
+        "roofline": {"bound": "alu", "achieved": achieved, "peak": alu_tflops, "unit": "TFLOP/s",
+                     "frac": achieved / alu_tflops, "traffic": traffic_record("kda_backward"),
+                     "peak_kind": "derived: fp32 FMA, SMs x 128 x 2 x max SM clock",
+                     "hbm_frac_algorithmic": moved / (ms_f32 * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+        "tolerance": "fp32: relative 1e-4 per gradient"}
+    return out
 
 
 def bench_decode(kda, dev, stream, world, args):

@@ -266,21 +266,23 @@ def decode_multi(q, k, v, log_alpha, beta, S, *, S_tokens=None, out=None):
 
 
 def backward_workspace_size(N: int, T: int, H: int, Dk: int, Dv: int,
-                            dtype=torch.bfloat16) -> int:
-    """Bytes of device workspace ``kda_backward`` needs for this problem."""
+                            dtype=torch.bfloat16, force_simt=False) -> int:
+    """Bytes of device workspace ``kda_backward`` needs for this problem (the
+    chunked tensor-core path for bf16 with Dk = Dv = 128, unless ``force_simt``)."""
     d = KDA_BF16 if dtype == torch.bfloat16 else KDA_F32
-    p = Params(N, T, H, Dk, Dv, CHUNK, d, d, 0)
+    p = Params(N, T, H, Dk, Dv, CHUNK, d, d, FLAG_FORCE_SIMT if force_simt else 0)
     return int(load_library().kda_backward_workspace_size(ctypes.byref(p)))
 
 
 def backward(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, *, d_out, dS_final=None,
-             need_dS0=True, workspace=None):
+             need_dS0=True, workspace=None, force_simt=False):
     """Gradients through ``kda_backward`` of a loss with dL/d out = ``d_out``
     (and dL/dS_final = ``dS_final``, None: zero).
 
     Inputs as ``forward``.  Returns a dict of fp32 tensors: dq, dk, dlog_alpha
     [T, H, Dk], dv [T, H, Dv], dbeta [T, H] and dS0 [N, H, Dk, Dv] (None when
-    ``need_dS0`` is false).
+    ``need_dS0`` is false).  bf16 inputs with Dk = Dv = 128 take the chunked
+    tensor-core backward; ``force_simt`` selects the fp32 CUDA-core one.
     """
     lib = load_library()
     dev = q.device
@@ -305,7 +307,8 @@ def backward(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, *, d_out, dS_fi
          "dv": torch.empty((T, H, Dv), **f32), "dlog_alpha": torch.empty((T, H, Dk), **f32),
          "dbeta": torch.empty((T, H), **f32),
          "dS0": torch.empty((N, H, Dk, Dv), **f32) if need_dS0 else None}
-    p = Params(N, T, H, Dk, Dv, CHUNK, _dt(q), _dt(log_alpha), 0)
+    p = Params(N, T, H, Dk, Dv, CHUNK, _dt(q), _dt(log_alpha),
+               FLAG_FORCE_SIMT if force_simt else 0)
     ws_bytes = int(lib.kda_backward_workspace_size(ctypes.byref(p)))
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)

@@ -150,6 +150,7 @@ kda_status forward_impl(const void *q, const void *k, const void *v, const void 
     a.snap_slots = use_snap ? (long long)snap->n_slots : 0;
     a.snap_every_chunks = use_snap ? snap->every / kda::kChunk : 0;
     a.test_stall = (p->flags & KDA_FLAG_TEST_STALL) != 0;
+    a.ckpt = nullptr;
 
     // bf16 with Dk = Dv = 128: tensor cores, two-pass when the workspace holds
     // the operand packets, else the single fused kernel; otherwise CUDA cores.
@@ -274,12 +275,75 @@ size_t bw_workspace_bytes(const kda_params *p) {
                                    kda::backward_part_floats(p->total_tokens, p->H, p->Dk) *
                                    sizeof(float);
 }
+
+// Chunked tensor-core backward workspace: [header][order][chunk_off][packets]
+// [state entering every chunk][Gam_L dS' of every chunk], one 64 KB fp32
+// state per (chunk, head) in each of the last two.
+size_t bw_tc_ckpt_offset(const kda_params *p) {
+    return packets_offset(p) +
+           kda::packet_slots_bound(p->total_tokens, p->num_seqs, p->H) * kda::kPacketBytes;
+}
+size_t bw_tc_state_bytes(const kda_params *p) {
+    return kda::packet_slots_bound(p->total_tokens, p->num_seqs, p->H) * (size_t)p->Dk * p->Dv *
+           sizeof(float);
+}
+size_t bw_tc_workspace_bytes(const kda_params *p) {
+    return bw_tc_ckpt_offset(p) + 2 * bw_tc_state_bytes(p);
+}
+bool bw_tc_path(const kda_params *p) { return tc_shape(p) && !(p->flags & KDA_FLAG_FORCE_SIMT); }
 }  // namespace
 
 size_t kda_backward_workspace_size(const kda_params *p) {
     if (check_common(p) != KDA_OK || p->total_tokens < 0) return 0;
-    return bw_workspace_bytes(p);
+    return bw_tc_path(p) ? bw_tc_workspace_bytes(p) : bw_workspace_bytes(p);
 }
+
+namespace {
+// The chunked tensor-core backward: the varlen index, the forward's two
+// passes keeping every chunk's entering state (no output), then the reverse
+// chain and the gradient assembly.
+kda_status backward_tc(const void *q, const void *k, const void *v, const void *log_alpha,
+                       const void *beta, const float *S0, const int32_t *cu_seqlens,
+                       const void *d_out, const float *dS_final, float *dq, float *dk, float *dv,
+                       float *dlog_alpha, float *dbeta, float *dS0, const kda_params *p,
+                       void *workspace, cudaStream_t s) {
+    char *ws = static_cast<char *>(workspace);
+    kda::ForwardArgs a;
+    memset(&a, 0, sizeof(a));
+    a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta;
+    a.S0 = S0; a.cu_seqlens = cu_seqlens; a.out = nullptr; a.S_final = nullptr;
+    a.N = p->num_seqs; a.T = p->total_tokens; a.H = p->H; a.Dk = p->Dk; a.Dv = p->Dv;
+    a.io_dtype = p->io_dtype; a.gate_dtype = p->gate_dtype;
+    a.status = reinterpret_cast<int32_t *>(ws);
+    a.work_ctr = a.status + 4;
+    a.order = reinterpret_cast<int32_t *>(ws + kWsHeader);
+    a.chunk_off = reinterpret_cast<int32_t *>(ws + chunk_off_offset(p));
+    a.packets = reinterpret_cast<unsigned char *>(ws + packets_offset(p));
+    a.packet_slots = kda::packet_slots_bound(p->total_tokens, p->num_seqs, p->H);
+    a.ckpt = reinterpret_cast<float *>(ws + bw_tc_ckpt_offset(p));
+    if (kda::launch_varlen_index(a, s) != cudaSuccess) return KDA_ERR_CUDA;
+    if (p->total_tokens > 0 && kda::launch_prefill_two_pass(a, s) != cudaSuccess) return KDA_ERR_CUDA;
+    kda::BackwardTcArgs b;
+    b.q = q; b.k = k; b.v = v; b.log_alpha = log_alpha; b.beta = beta; b.d_out = d_out;
+    b.dS_final = dS_final; b.cu_seqlens = cu_seqlens;
+    b.dq = dq; b.dk = dk; b.dv = dv; b.dla = dlog_alpha; b.dbeta = dbeta; b.dS0 = dS0;
+    b.N = p->num_seqs; b.T = p->total_tokens; b.H = p->H;
+    b.status = a.status; b.order = a.order; b.chunk_off = a.chunk_off;
+    b.packets = a.packets; b.packet_slots = a.packet_slots;
+    b.ckpt = a.ckpt;
+    b.dxs = reinterpret_cast<float *>(ws + bw_tc_ckpt_offset(p) + bw_tc_state_bytes(p));
+    if (p->total_tokens > 0) {
+        if (kda::launch_backward_tc(b, s) != cudaSuccess) return KDA_ERR_CUDA;
+    } else if (dS0) {
+        // no tokens: dS0 = dS_final (or zero), sequence by sequence
+        const size_t bytes = (size_t)p->num_seqs * p->H * p->Dk * p->Dv * sizeof(float);
+        const cudaError_t e = dS_final ? cudaMemcpyAsync(dS0, dS_final, bytes, cudaMemcpyDeviceToDevice, s)
+                                       : cudaMemsetAsync(dS0, 0, bytes, s);
+        if (e != cudaSuccess) return KDA_ERR_CUDA;
+    }
+    return KDA_OK;
+}
+}  // namespace
 
 kda_status kda_backward(const void *q, const void *k, const void *v, const void *log_alpha,
                         const void *beta, const float *S0, const int32_t *cu_seqlens,
@@ -298,12 +362,17 @@ kda_status kda_backward(const void *q, const void *k, const void *v, const void 
                           dv, dlog_alpha, dbeta, dS0, workspace};
     for (const void *x : ptrs)
         if (x && !aligned16(x)) return KDA_ERR_ALIGN;
-    if (!workspace || ((uintptr_t)workspace & 255u) || ws_bytes < bw_workspace_bytes(p))
+    const bool tc_path = bw_tc_path(p);
+    if (!workspace || ((uintptr_t)workspace & 255u) ||
+        ws_bytes < (tc_path ? bw_tc_workspace_bytes(p) : bw_workspace_bytes(p)))
         return KDA_ERR_WORKSPACE;
     if ((long long)p->num_seqs * p->H * (p->Dv / 32) > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
     kda::DeviceGuard guard;
     st = select_device(ptrs, 16, guard);
     if (st != KDA_OK) return st;
+    if (tc_path)
+        return backward_tc(q, k, v, log_alpha, beta, S0, cu_seqlens, d_out, dS_final, dq, dk, dv,
+                           dlog_alpha, dbeta, dS0, p, workspace, static_cast<cudaStream_t>(stream));
 
     char *ws = static_cast<char *>(workspace);
     kda::ForwardArgs ix;   // the varlen index: validation, order, chunk offsets

@@ -35,6 +35,7 @@ struct ForwardArgs {
     const int32_t *s0_slot;     // [N] start slot per sequence, negative: S0; or null
     long long snap_slots;
     int snap_every_chunks;      // 0: no snapshots
+    float *ckpt;                // two-pass path: state entering every chunk [slots, Dk, Dv], or null
     bool test_stall;            // chain pass waits on a barrier nobody arrives on
 };
 
@@ -74,6 +75,24 @@ inline size_t backward_part_floats(int64_t T, int64_t H, int Dk) {
 // (sequence, head, 32-wide value slice) recomputes kBwStep states at a time.
 constexpr int kBwStep = 32;
 inline size_t backward_scratch_floats(int Dk) { return (size_t)kBwStep * Dk * 32 + kBwStep * 32; }
+
+// Chunked tensor-core backward (bf16, Dk = Dv = 128): what the reverse chain
+// and the gradient assembly need after the forward's two passes ran with
+// ForwardArgs::ckpt = ckpt.
+struct BackwardTcArgs {
+    const void *q, *k, *v, *log_alpha, *beta, *d_out;   // bf16
+    const float *dS_final;            // or null
+    const int32_t *cu_seqlens;
+    float *dq, *dk, *dv, *dla, *dbeta;
+    float *dS0;                       // or null
+    int N, T, H;
+    int32_t *status, *order, *chunk_off;
+    const unsigned char *packets;
+    size_t packet_slots;
+    float *ckpt;                      // [slots, Dk, Dv] state entering every chunk
+    float *dxs;                       // [slots, Dk, Dv] Gam_L dS' of every chunk
+};
+cudaError_t launch_backward_tc(const BackwardTcArgs &a, cudaStream_t s);
 
 cudaError_t launch_varlen_index(const ForwardArgs &a, cudaStream_t s);
 cudaError_t launch_backward(const BackwardArgs &a, cudaStream_t s);

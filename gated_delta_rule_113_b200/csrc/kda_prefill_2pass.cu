@@ -83,37 +83,6 @@ constexpr uint32_t kPkTP = 49152;
 constexpr uint32_t kPkGL = 65536;
 static_assert(kPkGL + 512 <= kPacketBytes, "packet layout");
 
-// Maps item index m (= global chunk g * H + head) to its chunk.
-struct Item {
-    int h, c0, L;
-    int m;   // packet index m; negative: this CTA has no further item
-};
-__device__ __forceinline__ Item item_of(long long m, int H, const int32_t *chunk_off,
-                                        const int32_t *cu, int N) {
-    const int g = (int)(m / H);
-    Item it;
-    it.m = (int)m;
-    it.h = (int)(m % H);
-    int lo = 0, hi = N;   // largest n with chunk_off[n] <= g
-    while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (chunk_off[mid] <= g) lo = mid;
-        else hi = mid;
-    }
-    // 64-bit: with saturated offsets (overlapping sequences) j can exceed
-    // the sequence's chunk count; such an item gets no rows (L = 0).
-    const long long c0 = (long long)cu[lo] + (long long)(g - chunk_off[lo]) * kChunk;
-    const long long L = (long long)cu[lo + 1] - c0;
-    if (c0 < 0 || c0 > 0x7fffffffLL || L <= 0) {
-        it.c0 = 0;
-        it.L = 0;
-    } else {
-        it.c0 = (int)c0;
-        it.L = (int)(L < kChunk ? L : kChunk);
-    }
-    return it;
-}
-
 // PT = P Tb from its M = 64 accumulator (row r in TMEM lane 32 (r / 16) +
 // r % 16) to bf16 rows 64..127 of the Tb|PT tile.  Run by the eight prep
 // warps: warp w reads lane quarter w % 4 and columns 32 (w / 4) .. + 31.
@@ -635,6 +604,7 @@ struct ChParams {
     const int32_t *s0_slot;      // [N] start slot per sequence, or null
     long long snap_slots;
     int snap_every;              // chunks between snapshots; 0: none
+    float *ckpt;                 // [packet slots, Dk, Dv] fp32: the state entering every chunk, or null
     int test_stall;              // MMA issuer first waits on cbNever
     int N, T, H;
 };
@@ -867,6 +837,14 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
             if (!spin_or_abort(&bars[cbFull + s], (j / Ly::kStages) & 1, abort_flag, p.status)) { ok = false; break; }
             gl_cur = reinterpret_cast<const float *>(sm + s * Ly::kStage + Ly::kGL)[c];
             if (c == 0) KDA_TRACE2(j, 7);
+            if (p.ckpt) {   // the state entering chunk j, for the chunked backward
+                float *dst = p.ckpt + ((size_t)(g0 + j) * p.H + h) * kDK * kDV + (size_t)c * kDV +
+                             (size_t)vs * VS;
+#pragma unroll
+                for (int jj = 0; jj < VS; jj += 4)
+                    *reinterpret_cast<float4 *>(dst + jj) =
+                        make_float4(S[jj], S[jj + 1], S[jj + 2], S[jj + 3]);
+            }
             {
                 const uint32_t sb = sbase + Ly::kSB;
 #pragma unroll
@@ -922,7 +900,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
                     uint32_t v[32];
                     tmem_ld32(tmem_addr(tmem, 32 * wq, Ly::kTmD1 + d * VS + jj), v);
                     tmem_wait_ld();
-                    if (r < L) {
+                    if (r < L && p.out) {
                         __nv_bfloat16 *dst = p.out + ((size_t)(c0 + r) * p.H + h) * kDV + vs * VS + jj;
 #pragma unroll
                         for (int e = 0; e < 32; e += 8) {
@@ -1046,6 +1024,7 @@ cudaError_t launch_prefill_two_pass(const ForwardArgs &a, cudaStream_t s) {
     cp.s0_slot = a.s0_slot;
     cp.snap_slots = a.snap_slots;
     cp.snap_every = a.snap_every_chunks;
+    cp.ckpt = a.ckpt;
     cp.test_stall = a.test_stall ? 1 : 0;
     cp.N = a.N;
     cp.T = a.T;

@@ -75,6 +75,37 @@ __device__ __forceinline__ bool spin_or_abort(uint64_t *bar, uint32_t parity,
     return false;
 }
 
+// Maps item index m (= global chunk g * H + head) to its chunk.
+struct Item {
+    int h, c0, L;
+    int m;   // packet index m; negative: this CTA has no further item
+};
+__device__ __forceinline__ Item item_of(long long m, int H, const int32_t *chunk_off,
+                                        const int32_t *cu, int N) {
+    const int g = (int)(m / H);
+    Item it;
+    it.m = (int)m;
+    it.h = (int)(m % H);
+    int lo = 0, hi = N;   // largest n with chunk_off[n] <= g
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (chunk_off[mid] <= g) lo = mid;
+        else hi = mid;
+    }
+    // 64-bit: with saturated offsets (overlapping sequences) j can exceed
+    // the sequence's chunk count; such an item gets no rows (L = 0).
+    const long long c0 = (long long)cu[lo] + (long long)(g - chunk_off[lo]) * kChunk;
+    const long long L = (long long)cu[lo + 1] - c0;
+    if (c0 < 0 || c0 > 0x7fffffffLL || L <= 0) {
+        it.c0 = 0;
+        it.L = 0;
+    } else {
+        it.c0 = (int)c0;
+        it.L = (int)(L < kChunk ? L : kChunk);
+    }
+    return it;
+}
+
 // 16-byte shared store / load helpers
 __device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
                                        uint32_t d) {
@@ -280,42 +311,18 @@ __device__ __forceinline__ void write_p(int sw, int lane, uint32_t tmem, uint32_
     }
 }
 
-// kEarlyP: write P and release D_AP (one arrival on `ap_free`) right after
-// reading L.  Otherwise P stays in TMEM: the caller writes it with write_p()
-// and arrives on `ap_free` itself, later.
-template <bool kEarlyP = true>
-__device__ __forceinline__ void solve_chunk(int sw, int lane, uint32_t tmem, uint32_t tm_ap,
-                                            uint32_t p_tile, float *sL, float *sT, float *sXw,
-                                            const float *sB_s, uint64_t *ap_free,
-                                            uint32_t bar_id) {
-    const int t = sw * 32 + lane;
+// ---------------------------------------------------------------------------
+// T = (I + L)^{-1} for a strictly lower 64 x 64 fp32 L in sL (row stride
+// kLDL), run by 4 warps (sw = 0..3) that synchronise on named barrier
+// `bar_id`: the four 16x16 diagonal blocks by substitution, then a block
+// forward substitution by 8-column strips with mma.sync tf32.  Blocks of sT
+// above the diagonal blocks must be zero on entry (they are never written).
+// sXw is 4 x [16][17] fp32 warp-private scratch.  On return each warp has
+// written its strips; the caller orders them before any other reader.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void invert_unit_lower(int sw, int lane, const float *sL, float *sT,
+                                                  float *sXw, uint32_t bar_id) {
     const int g = lane >> 2, tq = lane & 3;
-    if (sw < 2) {
-        // L = strict_lower(diag(b) A)
-        const int r = 32 * sw + lane;
-        uint32_t v0[32], v1[32];
-        tmem_ld32(tmem_addr(tmem, 32 * sw, tm_ap), v0);
-        tmem_ld32(tmem_addr(tmem, 32 * sw, tm_ap + 32), v1);
-        tmem_wait_ld();
-        const float br = sB_s[r];
-        float *Lr = sL + r * kLDL;
-#pragma unroll
-        for (int c = 0; c < 64; c += 4) {
-            const uint32_t *src = c < 32 ? &v0[c] : &v1[c - 32];
-            float4 w;
-            w.x = (c + 0 < r) ? br * __uint_as_float(src[0]) : 0.f;
-            w.y = (c + 1 < r) ? br * __uint_as_float(src[1]) : 0.f;
-            w.z = (c + 2 < r) ? br * __uint_as_float(src[2]) : 0.f;
-            w.w = (c + 3 < r) ? br * __uint_as_float(src[3]) : 0.f;
-            *reinterpret_cast<float4 *>(Lr + c) = w;
-        }
-    } else if (kEarlyP) {
-        write_p(sw, lane, tmem, tm_ap, p_tile);
-    }
-    tc_fence_before();
-    named_bar(bar_id, kSolveThreads);
-    if (kEarlyP && t == 0) mbar_arrive(ap_free);
-
     // phase 1: invert the four 16x16 diagonal blocks, one block per warp, one
     // column per lane (lanes 0-15)
     if (lane < 16) {
@@ -395,7 +402,44 @@ __device__ __forceinline__ void solve_chunk(int sw, int lane, uint32_t tmem, uin
             }
         }
     }
+}
 
+// kEarlyP: write P and release D_AP (one arrival on `ap_free`) right after
+// reading L.  Otherwise P stays in TMEM: the caller writes it with write_p()
+// and arrives on `ap_free` itself, later.
+template <bool kEarlyP = true>
+__device__ __forceinline__ void solve_chunk(int sw, int lane, uint32_t tmem, uint32_t tm_ap,
+                                            uint32_t p_tile, float *sL, float *sT, float *sXw,
+                                            const float *sB_s, uint64_t *ap_free,
+                                            uint32_t bar_id) {
+    const int t = sw * 32 + lane;
+    if (sw < 2) {
+        // L = strict_lower(diag(b) A)
+        const int r = 32 * sw + lane;
+        uint32_t v0[32], v1[32];
+        tmem_ld32(tmem_addr(tmem, 32 * sw, tm_ap), v0);
+        tmem_ld32(tmem_addr(tmem, 32 * sw, tm_ap + 32), v1);
+        tmem_wait_ld();
+        const float br = sB_s[r];
+        float *Lr = sL + r * kLDL;
+#pragma unroll
+        for (int c = 0; c < 64; c += 4) {
+            const uint32_t *src = c < 32 ? &v0[c] : &v1[c - 32];
+            float4 w;
+            w.x = (c + 0 < r) ? br * __uint_as_float(src[0]) : 0.f;
+            w.y = (c + 1 < r) ? br * __uint_as_float(src[1]) : 0.f;
+            w.z = (c + 2 < r) ? br * __uint_as_float(src[2]) : 0.f;
+            w.w = (c + 3 < r) ? br * __uint_as_float(src[3]) : 0.f;
+            *reinterpret_cast<float4 *>(Lr + c) = w;
+        }
+    } else if (kEarlyP) {
+        write_p(sw, lane, tmem, tm_ap, p_tile);
+    }
+    tc_fence_before();
+    named_bar(bar_id, kSolveThreads);
+    if (kEarlyP && t == 0) mbar_arrive(ap_free);
+
+    invert_unit_lower(sw, lane, sL, sT, sXw, bar_id);
 }
 
 // Tb = T diag(b) -> bf16 into rows 0..63 of the K-major tile at `tp`, one

@@ -191,7 +191,7 @@ def test_backward_host_validation(over, params, code):
 
 def test_backward_workspace_size():
     lib = kda.load_library()
-    p = _params()
+    p = _params(flags=1)   # the fp32 CUDA-core backward
     n = lib.kda_backward_workspace_size(ctypes.byref(p))
     # the kept states, the per-CTA scratch and the per-slice partial sums
     T, N, H, Dk, Dv = p.total_tokens, p.num_seqs, p.H, p.Dk, p.Dv
@@ -230,3 +230,16 @@ def test_chunk_offset_scan_saturates_instead_of_wrapping():
     # every sequence whose offset passed the workspace is rejected, none wraps back in
     assert rejected[ok & (run64[:-1] + n_chunks > slots)].all()
     assert (stored >= 0).all()
+
+
+def test_chunked_backward_workspace_size():
+    """bf16 with d_k = d_v = 128: the chunked tensor-core backward keeps the
+    forward's operand packets and two fp32 states (the state entering the
+    chunk and the gradient reaching it) per (chunk, head)."""
+    lib = kda.load_library()
+    p = _params()
+    n = lib.kda_backward_workspace_size(ctypes.byref(p))
+    T, N, H = p.total_tokens, p.num_seqs, p.H
+    slots = ((T + 63) // 64 + N) * H
+    need = slots * (66048 + 2 * 128 * 128 * 4)
+    assert need <= n <= need + 4096 + 8 * N

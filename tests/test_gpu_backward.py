@@ -40,7 +40,7 @@ def _run(inp, need_dS0=True):
     dsf = inp["dS_final"].cuda() if inp["dS_final"] is not None else None
     g = kda.backward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["S0"],
                      d["cu_seqlens"], d_out=inp["d_out"].cuda(), dS_final=dsf,
-                     need_dS0=need_dS0)
+                     need_dS0=need_dS0, force_simt=True)
     torch.cuda.synchronize()
     return g
 
@@ -80,11 +80,9 @@ def test_backward_without_dS0_and_on_empty_sequences():
     g_full = _run(inp)
     g_part = _run(inp, need_dS0=False)
     assert g_part["dS0"] is None
-    # dv is written by one CTA per column; dq, dk, dlog_alpha and dbeta add the
-    # value slices' partial sums atomically, in an order that can vary
-    assert torch.equal(g_full["dv"], g_part["dv"])
-    for name in ("dq", "dk", "dlog_alpha", "dbeta"):
-        assert rel_fro(as_np(g_full[name]), as_np(g_part[name])) <= 1e-6
+    # every gradient is a fixed sequence of operations: leaving dS0 out changes none
+    for name in ("dq", "dk", "dv", "dlog_alpha", "dbeta"):
+        assert torch.equal(g_full[name], g_part[name]), name
     # an empty sequence passes dS_final straight to dS0
     assert torch.equal(g_full["dS0"][0].cpu(), inp["dS_final"][0])
     _check(inp, g_full)
@@ -97,12 +95,13 @@ def test_backward_malformed_seqlens_reported_not_faulting():
     d = to_dev(inp)
     cu = torch.tensor([0, T, 0, T, 0, T, 0, T, 0, T], dtype=torch.int32, device="cuda")
     N = cu.numel() - 1
-    n_ws = kda.backward_workspace_size(N, T, H, 128, 128)
-    buf = torch.zeros(n_ws + (1 << 20), dtype=torch.uint8, device="cuda")
-    kda.backward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], None, cu,
-                 d_out=inp["d_out"].cuda(), workspace=buf[:n_ws])
-    assert kda.workspace_status(buf[:n_ws]) == 7
-    assert not buf[n_ws:].any()            # nothing written past the workspace
+    for simt in (True, False):
+        n_ws = kda.backward_workspace_size(N, T, H, 128, 128, force_simt=simt)
+        buf = torch.zeros(n_ws + (1 << 20), dtype=torch.uint8, device="cuda")
+        kda.backward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], None, cu,
+                     d_out=inp["d_out"].cuda(), workspace=buf[:n_ws], force_simt=simt)
+        assert kda.workspace_status(buf[:n_ws]) == 7
+        assert not buf[n_ws:].any()            # nothing written past the workspace
 
 
 def test_backward_fp32_io_bf16_gates():
@@ -148,14 +147,15 @@ def test_backward_with_no_tokens_passes_dS_final_to_dS0():
     cu = torch.zeros(3, dtype=torch.int32, device="cuda")
     e = torch.empty((0, H, D), dtype=torch.bfloat16, device="cuda")
     dSf = torch.randn((2, H, D, D), device="cuda")
-    g = kda.backward(e, e, e, e, torch.empty((0, H), dtype=torch.bfloat16, device="cuda"), None,
-                     cu, d_out=e, dS_final=dSf)
-    torch.cuda.synchronize()
-    assert torch.equal(g["dS0"], dSf)
-    g0 = kda.backward(e, e, e, e, torch.empty((0, H), dtype=torch.bfloat16, device="cuda"), None,
-                      cu, d_out=e)
-    torch.cuda.synchronize()
-    assert torch.equal(g0["dS0"], torch.zeros_like(dSf))
+    for simt in (True, False):
+        g = kda.backward(e, e, e, e, torch.empty((0, H), dtype=torch.bfloat16, device="cuda"),
+                         None, cu, d_out=e, dS_final=dSf, force_simt=simt)
+        torch.cuda.synchronize()
+        assert torch.equal(g["dS0"], dSf)
+        g0 = kda.backward(e, e, e, e, torch.empty((0, H), dtype=torch.bfloat16, device="cuda"),
+                          None, cu, d_out=e, force_simt=simt)
+        torch.cuda.synchronize()
+        assert torch.equal(g0["dS0"], torch.zeros_like(dSf))
 
 
 def test_backward_is_bitwise_reproducible():

@@ -244,14 +244,6 @@ rchain_kernel(const __grid_constant__ CUtensorMap tm_do, RcParams p) {
             const float g = reinterpret_cast<const float *>(sm + stage(i) + Ly::kGL)[c];
 #pragma unroll
             for (int jj = 0; jj < VS; ++jj) dS[jj] *= g;
-            {
-                float *dst = p.dxs + ((size_t)(g0 + j) * p.H + h) * kDK * kDV + (size_t)c * kDV +
-                             (size_t)vs * VS;
-#pragma unroll
-                for (int jj = 0; jj < VS; jj += 4)
-                    *reinterpret_cast<float4 *>(dst + jj) =
-                        make_float4(dS[jj], dS[jj + 1], dS[jj + 2], dS[jj + 3]);
-            }
 #pragma unroll
             for (int q8 = 0; q8 < VS / 8; ++q8)
                 sts128(xb + vs_off<VS>(c, q8), pack2(dS[8 * q8], dS[8 * q8 + 1]),
@@ -261,6 +253,14 @@ rchain_kernel(const __grid_constant__ CUtensorMap tm_do, RcParams p) {
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[rbXbFull]);
+            {   // fp32 dX_j for the assembly, off the chain: after the proxy fence
+                float *dst = p.dxs + ((size_t)(g0 + j) * p.H + h) * kDK * kDV + (size_t)c * kDV +
+                             (size_t)vs * VS;
+#pragma unroll
+                for (int jj = 0; jj < VS; jj += 4)
+                    *reinterpret_cast<float4 *>(dst + jj) =
+                        make_float4(dS[jj], dS[jj + 1], dS[jj + 2], dS[jj + 3]);
+            }
             // dU (M = 64 accumulator: row r in TMEM lane 32 (r / 16) + r % 16)
             // -> bf16 rows 0-63 of the [dU; dO] operand
             if (!spin_or_abort(&bars[rbDuAcc], i & 1, abort_flag, p.status)) { ok = false; break; }
@@ -464,11 +464,19 @@ __global__ void __launch_bounds__(kAsmThreads, 1) assemble_kernel(AsmParams p) {
 
     // ---------------------------------------------------------------- P0
     // log_alpha and beta; sT cleared (the inverse writes only its blocks)
-    for (int i = t; i < 64 * 16; i += kAsmThreads) {   // 16 B per thread and step
-        const int r = i >> 4, c8 = (i & 15) * 8;
-        uint4 x = make_uint4(0, 0, 0, 0);
-        if (r < L) x = *reinterpret_cast<const uint4 *>(p.la + rowk(r) + c8);
-        *reinterpret_cast<uint4 *>(sLa + r * 128 + c8) = x;
+    {   // 4 x 16 B per thread, all loads in flight before the stores
+        uint4 x[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int i = t + u * kAsmThreads, r = i >> 4, c8 = (i & 15) * 8;
+            x[u] = r < L ? __ldg(reinterpret_cast<const uint4 *>(p.la + rowk(r) + c8))
+                         : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int i = t + u * kAsmThreads, r = i >> 4, c8 = (i & 15) * 8;
+            *reinterpret_cast<uint4 *>(sLa + r * 128 + c8) = x[u];
+        }
     }
     if (t < 64) sB[t] = t < L ? __bfloat162float(p.beta[(size_t)(c0 + t) * H + h]) : 0.f;
     for (int i = t; i < 64 * kLDL; i += kAsmThreads) sT[i] = 0.f;
@@ -486,23 +494,29 @@ __global__ void __launch_bounds__(kAsmThreads, 1) assemble_kernel(AsmParams p) {
         if (bad) set_status(p.status, KDA_ERR_DECAY);
     }
     __syncthreads();
-    // Kg, Qg, Ki as bf16 tiles (rows past L are zero: k, q read as zero)
-    for (int i = t; i < 64 * 32; i += kAsmThreads) {   // 4 elements per thread and step
-        const int r = i >> 5, c4 = (i & 31) * 4;
-        float kv[4] = {0.f, 0.f, 0.f, 0.f}, qv[4] = {0.f, 0.f, 0.f, 0.f};
-        if (r < L) {
-            const uint2 kk = *reinterpret_cast<const uint2 *>(p.k + rowk(r) + c4);
-            const uint2 qq = *reinterpret_cast<const uint2 *>(p.q + rowk(r) + c4);
-            kv[0] = bf16lo(kk.x); kv[1] = bf16hi(kk.x); kv[2] = bf16lo(kk.y); kv[3] = bf16hi(kk.y);
-            qv[0] = bf16lo(qq.x); qv[1] = bf16hi(qq.x); qv[2] = bf16lo(qq.y); qv[3] = bf16hi(qq.y);
-        }
-        const float4 ga = *reinterpret_cast<const float4 *>(sGam + r * 128 + c4);
-        const float gm[4] = {ga.x, ga.y, ga.z, ga.w};
+    // Kg, Qg, Ki as bf16 tiles (rows past L are zero: k, q read as zero); the
+    // global loads of all eight steps are issued before any store
+    {
+        uint2 kk[8], qq[8];
 #pragma unroll
-        for (int e = 0; e < 4; e += 2) {
-            st_bf16x2(toff(tKg, r, c4 + e), kv[e] * gm[e], kv[e + 1] * gm[e + 1]);
-            st_bf16x2(toff(tQg, r, c4 + e), qv[e] * gm[e], qv[e + 1] * gm[e + 1]);
-            st_bf16x2(toff(tKi, r, c4 + e), kv[e] / gm[e], kv[e + 1] / gm[e + 1]);
+        for (int u = 0; u < 8; ++u) {
+            const int i = t + u * kAsmThreads, r = i >> 5, c4 = (i & 31) * 4;
+            kk[u] = r < L ? __ldg(reinterpret_cast<const uint2 *>(p.k + rowk(r) + c4)) : make_uint2(0, 0);
+            qq[u] = r < L ? __ldg(reinterpret_cast<const uint2 *>(p.q + rowk(r) + c4)) : make_uint2(0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int i = t + u * kAsmThreads, r = i >> 5, c4 = (i & 31) * 4;
+            const float kv[4] = {bf16lo(kk[u].x), bf16hi(kk[u].x), bf16lo(kk[u].y), bf16hi(kk[u].y)};
+            const float qv[4] = {bf16lo(qq[u].x), bf16hi(qq[u].x), bf16lo(qq[u].y), bf16hi(qq[u].y)};
+            const float4 ga = *reinterpret_cast<const float4 *>(sGam + r * 128 + c4);
+            const float gm[4] = {ga.x, ga.y, ga.z, ga.w};
+#pragma unroll
+            for (int e = 0; e < 4; e += 2) {
+                st_bf16x2(toff(tKg, r, c4 + e), kv[e] * gm[e], kv[e + 1] * gm[e + 1]);
+                st_bf16x2(toff(tQg, r, c4 + e), qv[e] * gm[e], qv[e + 1] * gm[e + 1]);
+                st_bf16x2(toff(tKi, r, c4 + e), kv[e] / gm[e], kv[e + 1] / gm[e + 1]);
+            }
         }
     }
     // Gam at this thread's accumulator positions (64 x 128 layout)
@@ -544,17 +558,26 @@ __global__ void __launch_bounds__(kAsmThreads, 1) assemble_kernel(AsmParams p) {
     } else {
         const float *Sg = p.ckpt + (size_t)m * kDK * kDV;
         const float *Xg = p.dxs + (size_t)m * kDK * kDV;
-        for (int r = w - 4; r < 128; r += 4) {
-            const float4 a = *reinterpret_cast<const float4 *>(Sg + (size_t)r * kDV + 4 * lane);
-            const float4 b = *reinterpret_cast<const float4 *>(Xg + (size_t)r * kDV + 4 * lane);
-            st_bf16x2(toff(tS, r, 4 * lane), a.x, a.y);
-            st_bf16x2(toff(tS, r, 4 * lane + 2), a.z, a.w);
-            st_bf16x2(toff(tX, r, 4 * lane), b.x, b.y);
-            st_bf16x2(toff(tX, r, 4 * lane + 2), b.z, b.w);
-            float d = a.x * b.x + a.y * b.y + a.z * b.z + a.w * b.w;
+        // rows w - 4 + 4 i, eight rows (16 loads of 16 B) in flight per batch
+        for (int r0 = w - 4; r0 < 128; r0 += 32) {
+            float4 a[8], b[8];
 #pragma unroll
-            for (int o = 16; o >= 1; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
-            if (lane == 0) sSdx[r] = d;
+            for (int u = 0; u < 8; ++u) {
+                a[u] = __ldg(reinterpret_cast<const float4 *>(Sg + (size_t)(r0 + 4 * u) * kDV + 4 * lane));
+                b[u] = __ldg(reinterpret_cast<const float4 *>(Xg + (size_t)(r0 + 4 * u) * kDV + 4 * lane));
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int r = r0 + 4 * u;
+                st_bf16x2(toff(tS, r, 4 * lane), a[u].x, a[u].y);
+                st_bf16x2(toff(tS, r, 4 * lane + 2), a[u].z, a[u].w);
+                st_bf16x2(toff(tX, r, 4 * lane), b[u].x, b[u].y);
+                st_bf16x2(toff(tX, r, 4 * lane + 2), b[u].z, b[u].w);
+                float d = a[u].x * b[u].x + a[u].y * b[u].y + a[u].z * b[u].z + a[u].w * b[u].w;
+#pragma unroll
+                for (int o = 16; o >= 1; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+                if (lane == 0) sSdx[r] = d;
+            }
         }
     }
     __syncthreads();
@@ -576,17 +599,24 @@ __global__ void __launch_bounds__(kAsmThreads, 1) assemble_kernel(AsmParams p) {
         st_bf16x2(toff(tTb, r, s), tr[nt][0] * sB[s], tr[nt][1] * sB[s + 1]);
         st_bf16x2(toff(tTb, r + 8, s), tr[nt][2] * sB[s], tr[nt][3] * sB[s + 1]);
     }
-    for (int i = t; i < 64 * 32; i += kAsmThreads) {
-        const int r = i >> 5, c4 = (i & 31) * 4;
-        uint2 vv = make_uint2(0, 0), oo = make_uint2(0, 0);
-        if (r < L) {
-            vv = *reinterpret_cast<const uint2 *>(p.v + rowk(r) + c4);
-            oo = *reinterpret_cast<const uint2 *>(p.dout + rowk(r) + c4);
+    {
+        uint2 vv[8], oo[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int i = t + u * kAsmThreads, r = i >> 5, c4 = (i & 31) * 4;
+            vv[u] = r < L ? __ldg(reinterpret_cast<const uint2 *>(p.v + rowk(r) + c4)) : make_uint2(0, 0);
+            oo[u] = r < L ? __ldg(reinterpret_cast<const uint2 *>(p.dout + rowk(r) + c4)) : make_uint2(0, 0);
         }
-        asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(toff(tV, r, c4)), "r"(vv.x), "r"(vv.y)
-                     : "memory");
-        asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(toff(tDO, r, c4)), "r"(oo.x), "r"(oo.y)
-                     : "memory");
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int i = t + u * kAsmThreads, r = i >> 5, c4 = (i & 31) * 4;
+            asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(toff(tV, r, c4)), "r"(vv[u].x),
+                         "r"(vv[u].y)
+                         : "memory");
+            asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(toff(tDO, r, c4)), "r"(oo[u].x),
+                         "r"(oo[u].y)
+                         : "memory");
+        }
     }
     __syncthreads();
 
@@ -646,23 +676,32 @@ __global__ void __launch_bounds__(kAsmThreads, 1) assemble_kernel(AsmParams p) {
     zero(acc);
     wmma<8, false, false>(acc, tDO, m0, tS, n0, 0, 128, lane);
     wmma<8, false, true>(acc, tP, m0, tKi, n0, 0, 64, lane);
+    {
+        uint32_t qq[8][2];
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
+        for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
-        for (int e2 = 0; e2 < 2; ++e2) {
-            const int r = m0 + g8 + 8 * e2;
-            const int col = n0 + 8 * nt + 2 * q4;
-            float qv[2] = {0.f, 0.f};
-            if (r < L) {
-                const uint32_t qq = *reinterpret_cast<const uint32_t *>(p.q + rowk(r) + col);
-                qv[0] = bf16lo(qq);
-                qv[1] = bf16hi(qq);
-                *reinterpret_cast<float2 *>(p.dq + rowk(r) + col) =
-                    make_float2(acc[nt][2 * e2] * gam[nt][2 * e2], acc[nt][2 * e2 + 1] * gam[nt][2 * e2 + 1]);
+            for (int e2 = 0; e2 < 2; ++e2) {
+                const int r = m0 + g8 + 8 * e2;
+                qq[nt][e2] = r < L ? __ldg(reinterpret_cast<const unsigned int *>(
+                                         p.q + rowk(r) + n0 + 8 * nt + 2 * q4))
+                                   : 0u;
             }
-            dg[nt][2 * e2] = acc[nt][2 * e2] * qv[0] * gam[nt][2 * e2];
-            dg[nt][2 * e2 + 1] = acc[nt][2 * e2 + 1] * qv[1] * gam[nt][2 * e2 + 1];
-        }
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+            for (int e2 = 0; e2 < 2; ++e2) {
+                const int r = m0 + g8 + 8 * e2;
+                const int col = n0 + 8 * nt + 2 * q4;
+                const float qv0 = bf16lo(qq[nt][e2]), qv1 = bf16hi(qq[nt][e2]);
+                if (r < L)
+                    *reinterpret_cast<float2 *>(p.dq + rowk(r) + col) =
+                        make_float2(acc[nt][2 * e2] * gam[nt][2 * e2],
+                                    acc[nt][2 * e2 + 1] * gam[nt][2 * e2 + 1]);
+                dg[nt][2 * e2] = acc[nt][2 * e2] * qv0 * gam[nt][2 * e2];
+                dg[nt][2 * e2 + 1] = acc[nt][2 * e2 + 1] * qv1 * gam[nt][2 * e2 + 1];
+            }
+    }
     // ---------------------------------------------------------------- P9: dW = -dU S^T
     zero(acc);
     wmma<8, false, false>(acc, tR1, m0, tS, n0, 0, 128, lane);
@@ -745,18 +784,23 @@ __global__ void __launch_bounds__(kAsmThreads, 1) assemble_kernel(AsmParams p) {
     // ---------------------------------------------------------------- P14
     // dK = dKg Gam + dKi / Gam; dG = dKg Kg + dQg Qg - dKi Ki into the S region
     float *sdG = reinterpret_cast<float *>(sm + Ly::kS);
+    uint32_t kk[8][2];
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+        for (int e2 = 0; e2 < 2; ++e2) {
+            const int r = m0 + g8 + 8 * e2;
+            kk[nt][e2] = r < L ? __ldg(reinterpret_cast<const unsigned int *>(
+                                     p.k + rowk(r) + n0 + 8 * nt + 2 * q4))
+                               : 0u;
+        }
 #pragma unroll
     for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
         for (int e2 = 0; e2 < 2; ++e2) {
             const int r = m0 + g8 + 8 * e2;
             const int col = n0 + 8 * nt + 2 * q4;
-            float kv[2] = {0.f, 0.f};
-            if (r < L) {
-                const uint32_t kk = *reinterpret_cast<const uint32_t *>(p.k + rowk(r) + col);
-                kv[0] = bf16lo(kk);
-                kv[1] = bf16hi(kk);
-            }
+            const float kv[2] = {bf16lo(kk[nt][e2]), bf16hi(kk[nt][e2])};
             float dkv[2], dgv[2];
 #pragma unroll
             for (int e = 0; e < 2; ++e) {

@@ -837,14 +837,6 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
             if (!spin_or_abort(&bars[cbFull + s], (j / Ly::kStages) & 1, abort_flag, p.status)) { ok = false; break; }
             gl_cur = reinterpret_cast<const float *>(sm + s * Ly::kStage + Ly::kGL)[c];
             if (c == 0) KDA_TRACE2(j, 7);
-            if (p.ckpt) {   // the state entering chunk j, for the chunked backward
-                float *dst = p.ckpt + ((size_t)(g0 + j) * p.H + h) * kDK * kDV + (size_t)c * kDV +
-                             (size_t)vs * VS;
-#pragma unroll
-                for (int jj = 0; jj < VS; jj += 4)
-                    *reinterpret_cast<float4 *>(dst + jj) =
-                        make_float4(S[jj], S[jj + 1], S[jj + 2], S[jj + 3]);
-            }
             {
                 const uint32_t sb = sbase + Ly::kSB;
 #pragma unroll
@@ -859,6 +851,16 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[cbSbFull]);
             if (c == 0) KDA_TRACE2(j, 8);
+            // the state entering chunk j, for the chunked backward: stored after
+            // the proxy fence above so that fence never waits for it
+            if (p.ckpt) {
+                float *dst = p.ckpt + ((size_t)(g0 + j) * p.H + h) * kDK * kDV + (size_t)c * kDV +
+                             (size_t)vs * VS;
+#pragma unroll
+                for (int jj = 0; jj < VS; jj += 4)
+                    *reinterpret_cast<float4 *>(dst + jj) =
+                        make_float4(S[jj], S[jj + 1], S[jj + 2], S[jj + 3]);
+            }
             // Snapshot stores go after a proxy fence, never just before one: the
             // fence would wait for them to complete.  Rows 64-127 next fence a
             // chunk later; rows 0-63 fence the U operand below, so they store

@@ -9,7 +9,7 @@ with.  To keep every rank busy the heads are processed in groups: rank r
 starts head group g as soon as rank r - 1 has sent the state after its
 segment for that group, then sends its own state for g on to rank r + 1.
 With G groups and W ranks each rank is idle for W - 1 group-steps of the
-G + W - 1.
+G + W - 1; ``choose_group_size`` picks G from H, W and the SM count.
 
 The exchange is one fp32 state per head of a group (Hg x 64 KiB at
 d_k = d_v = 128), sent point to point with ``torch.distributed.send`` /
@@ -23,6 +23,35 @@ from typing import Callable, Optional
 import torch
 
 
+def choose_group_size(H: int, world: int, n_sms: int = 148, ctas_per_head: int = 4) -> int:
+    """Heads per group for ``cp_prefill`` on ``world`` ranks of ``n_sms`` SMs.
+
+    One group call runs the chain pass over ``ctas_per_head`` CTAs per head
+    (32-wide value slices) and each of those walks the rank's whole segment:
+    its time is set by the chain's per-chunk latency, not by the number of
+    heads, until the call has enough heads to fill the GPU (about n_sms /
+    ctas_per_head).  The rank pipeline over G groups keeps each rank busy for
+    G of G + W - 1 group steps, so the job takes (G + W - 1) t(H / G) with
+    t(h) = max(t_latency, h t_head).  Below the fill point t is flat and one
+    group is fastest (the split then serves memory capacity: every rank holds
+    only its segment); above it, groups of about the fill size balance the
+    two terms.
+    """
+    if H < 1 or world < 1 or n_sms < 1 or ctas_per_head < 1:
+        raise ValueError("H, world, n_sms and ctas_per_head must be positive")
+    fill = max(1, -(-n_sms // ctas_per_head))   # heads that fill the GPU in one call
+    if H <= fill or world == 1:
+        return H
+    groups = -(-H // fill)
+    return -(-H // groups)                         # equal groups of at most `fill` heads
+
+
+def busy_fraction(H: int, group_size: int, world: int) -> float:
+    """Fraction of group steps each rank computes in the pipeline: G / (G + W - 1)."""
+    G = len(head_groups(H, group_size))
+    return G / (G + world - 1)
+
+
 def head_groups(H: int, group_size: int):
     """[(h0, h1), ...] covering 0..H in groups of at most ``group_size`` heads."""
     if group_size < 1:
@@ -30,7 +59,8 @@ def head_groups(H: int, group_size: int):
     return [(h0, min(H, h0 + group_size)) for h0 in range(0, H, group_size)]
 
 
-def cp_prefill(q, k, v, log_alpha, beta, S0=None, *, rank: int, world: int, group_size: int,
+def cp_prefill(q, k, v, log_alpha, beta, S0=None, *, rank: int, world: int,
+               group_size: Optional[int] = None,
                send_state: Callable[[torch.Tensor, int], None],
                recv_state: Callable[[torch.Tensor, int], None],
                forward: Optional[Callable] = None, state_dtype=torch.float32):
@@ -42,7 +72,8 @@ def cp_prefill(q, k, v, log_alpha, beta, S0=None, *, rank: int, world: int, grou
     only (None: zero).  ``send_state(t, peer)`` / ``recv_state(t, peer)`` move
     one contiguous state tensor; ``forward`` defaults to the library's
     prefill with the signature of ``gated_delta_rule_113_b200.forward``
-    (states in ``state_dtype``, fp32 for the library).
+    (states in ``state_dtype``, fp32 for the library).  ``group_size`` None:
+    ``choose_group_size(H, world)`` (the same on every rank).
 
     Returns (out [T_r, H, Dv], S_final [1, H, Dk, Dv] on the last rank, None
     elsewhere).
@@ -52,6 +83,8 @@ def cp_prefill(q, k, v, log_alpha, beta, S0=None, *, rank: int, world: int, grou
         forward = library_forward
     T, H, Dk = q.shape
     Dv = v.shape[-1]
+    if group_size is None:
+        group_size = choose_group_size(H, world)
     out = torch.empty((T, H, Dv), dtype=q.dtype, device=q.device)
     S_last = torch.empty((1, H, Dk, Dv), dtype=state_dtype, device=q.device) \
         if rank == world - 1 else None

@@ -138,3 +138,23 @@ def test_threaded_ranks_on_one_gpu_match_the_oracle():
                             inp["S0"], inp["cu_seqlens"].numpy())
     assert rel_fro(as_np(out), ro) <= TOL_BF16
     assert rel_fro(as_np(results[world - 1][1]), rs) <= TOL_BF16
+
+
+def test_group_size_rule():
+    """Groups fill the GPU per call (about SMs / 4 heads at four chain CTAs per
+    head) before the rank pipeline gets more of them; the busy fraction is
+    G / (G + W - 1)."""
+    from gated_delta_rule_113_b200.context_parallel import (busy_fraction, choose_group_size,
+                                                            head_groups)
+    # 32 heads (the long-context workloads) never fill 148 SMs: one group
+    assert choose_group_size(32, 8) == 32
+    assert busy_fraction(32, 32, 8) == 1 / 8
+    # 128 heads on 148 SMs: four groups of 32 (each call 128 of 148 SMs)
+    assert choose_group_size(128, 8) == 32
+    assert busy_fraction(128, 32, 8) == 4 / 11
+    # uneven head counts split into equal groups no larger than the fill size
+    gs = choose_group_size(100, 4)
+    assert gs <= 37 and len(head_groups(100, gs)) == 3
+    assert choose_group_size(64, 1) == 64          # one rank: no pipeline to feed
+    with pytest.raises(ValueError):
+        choose_group_size(0, 2)

@@ -84,23 +84,25 @@ constexpr uint32_t kPkGL = 65536;
 static_assert(kPkGL + 512 <= kPacketBytes, "packet layout");
 
 // PT = P Tb from its M = 64 accumulator (row r in TMEM lane 32 (r / 16) +
-// r % 16) to bf16 rows 64..127 of the Tb|PT tile.  Run by the eight prep
-// warps: warp w reads lane quarter w % 4 and columns 32 (w / 4) .. + 31.
-__device__ __forceinline__ void convert_pt8(int w, int lane, uint32_t tmem, uint32_t tm_pt,
+// r % 16) to bf16 rows 64..127 of the Tb|PT tile, by the four solve warps:
+// warp sw reads lane quarter sw, all 64 columns.
+__device__ __forceinline__ void convert_pt4(int sw, int lane, uint32_t tmem, uint32_t tm_pt,
                                             uint32_t tp) {
-    const int qt = w & 3, hh = w >> 2;
-    uint32_t v[32];
-    tmem_ld32(tmem_addr(tmem, 32 * qt, tm_pt + 32 * hh), v);
-    tmem_wait_ld();
-    if (lane < 16) {
-        const int r = 64 + 16 * qt + lane;
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-            sts128(tp + sw128_off(r, 4 * hh + j),
-                   pack2(__uint_as_float(v[8 * j]), __uint_as_float(v[8 * j + 1])),
-                   pack2(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3])),
-                   pack2(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5])),
-                   pack2(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7])));
+    for (int hh = 0; hh < 2; ++hh) {
+        uint32_t v[32];
+        tmem_ld32(tmem_addr(tmem, 32 * sw, tm_pt + 32 * hh), v);
+        tmem_wait_ld();
+        if (lane < 16) {
+            const int r = 64 + 16 * sw + lane;
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                sts128(tp + sw128_off(r, 4 * hh + j),
+                       pack2(__uint_as_float(v[8 * j]), __uint_as_float(v[8 * j + 1])),
+                       pack2(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3])),
+                       pack2(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5])),
+                       pack2(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7])));
+        }
     }
     fence_proxy_async();
     tc_fence_before();
@@ -155,8 +157,8 @@ enum KsBars {
     kbApFull = 6,    // [2] A/P product -> solve (two TMEM accumulators)
     kbApFree = 8,    // [2] solve has read D_AP[s] -> A/P issuer
     kbTbFull = 10,   // solve -> PT issuer (Tb and P final, D_AP read)
-    kbPtAcc = 11,    // PT = P Tb product -> prep warps
-    kbPtReady = 12,  // count 8: PT written as bf16 -> W issuer
+    kbPtAcc = 11,    // PT = P Tb product -> solve warps
+    kbPtReady = 12,  // count 4: PT written as bf16 (solve warps) -> W issuer
     kbTpFree = 13,   // the Tb|PT tile has been read -> Tb write of the next chunk
     kbWaccFull = 14, // [W; PW] product -> prep warps
     kbWReady = 15,   // count 8: -W and Qe written -> stores (and D_W free)
@@ -239,7 +241,8 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         for (int i = 0; i < kbNum; ++i) {
             uint32_t cnt = 1;
             if (i >= kbKqFull && i < kbKqFull + kKsStages) cnt = kPrepThreads / 32;
-            if (i == kbWReady || i == kbPtReady) cnt = kPrepThreads / 32;
+            if (i == kbWReady) cnt = kPrepThreads / 32;
+            if (i == kbPtReady) cnt = 4;
             mbar_init(&bars[i], cnt);
         }
         *abort_flag = 0;
@@ -412,14 +415,10 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     } else if (warp >= kKsPrep0 && warp < kKsPrep0 + kPrepThreads / 32) {
         // ----------------------------------------------------------- prep
         const int t = tid - kKsPrep0 * 32;
-        // After preparing chunk i these warps turn chunk i-1's PT and [W; PW]
-        // products into bf16 operands, so the solve warps only solve.
+        // After preparing chunk i these warps turn chunk i-1's [W; PW] product
+        // into the bf16 -W and Qe operands (the solve warps convert PT).
         auto convert = [&](int m) -> bool {
             const int sm3 = m % kKsStages;
-            if (!wait_or_abort(&bars[kbPtAcc], m & 1, abort_flag, p.status)) return false;
-            tc_fence_after();
-            convert_pt8(warp, lane, tmem, Ly::kTmPT, sbase + Ly::kTP);
-            if (lane == 0) mbar_arrive(&bars[kbPtReady]);
             if (!wait_or_abort(&bars[kbWaccFull], m & 1, abort_flag, p.status)) return false;
             tc_fence_after();
             if (t == 0) KDA_TRACE1(m, 7);
@@ -487,6 +486,13 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 mbar_arrive(&bars[kbTbFull]);
             }
             if (t == 0) KDA_TRACE1(i, 5);
+            // PT = P Tb (issued by the store warp) -> bf16 rows 64-127 of the
+            // Tb|PT tile, here rather than by the prep warps, which are busy
+            // with the next chunk by then
+            if (!wait_or_abort(&bars[kbPtAcc], i & 1, abort_flag, p.status)) break;
+            tc_fence_after();
+            convert_pt4(sw, lane, tmem, Ly::kTmPT, sbase + Ly::kTP);
+            if (lane == 0) mbar_arrive(&bars[kbPtReady]);
         }
     } else if (warp == kKsMma) {
         // --------------------------------- A/P issuer (lane 0), Ki stores (lane 1)
@@ -508,14 +514,8 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                     mbar_arrive(&bars[kbApFull + a]);
                 break;
             }
-            if (lane == 1) {
-                unsigned char *dst = p.packets + (size_t)m * kPacketBytes;
-                bulk_store(dst + kPkKI, sm + Ly::kKI + s * 16384, 16384);
-                bulk_store(dst + kPkGL, sGL + s * 128, 512);
-                bulk_commit();
-                bulk_wait_read_all();
-                mbar_arrive(&bars[kbKiFree + s]);
-            }
+            // the product first: lane 1's bulk store blocks the warp until its
+            // copy has read shared memory
             if (lane == 0) {
                 const uint32_t kq = sbase + Ly::kKQ + s * 32768;
                 const uint64_t d_kq = smem_desc(kq, 16, 1024, kSw128);
@@ -531,6 +531,14 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                     mma_commit(&bars[kbApFull + a]);
                     KDA_TRACE1(i, 3);
                 }
+            }
+            if (lane == 1) {
+                unsigned char *dst = p.packets + (size_t)m * kPacketBytes;
+                bulk_store(dst + kPkKI, sm + Ly::kKI + s * 16384, 16384);
+                bulk_store(dst + kPkGL, sGL + s * 128, 512);
+                bulk_commit();
+                bulk_wait_read_all();
+                mbar_arrive(&bars[kbKiFree + s]);
             }
             if (!__shfl_sync(0xffffffffu, ok, 0)) break;
         }

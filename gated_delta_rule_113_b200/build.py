@@ -36,14 +36,24 @@ def _headers():
     return glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(INCLUDE, "*.h"))
 
 
-def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
-    os.makedirs(BUILD_DIR, exist_ok=True)
+# The bounds-checking variant (-DKDA_DEBUG_BOUNDS): every checked global
+# index that would leave its buffer is skipped and recorded as KDA_ERR_BOUNDS
+# in the device status word; a test build, not the product path.
+LIB_DEBUG_BOUNDS = os.path.join(PKG, "libkda_debug_bounds.so")
+
+
+def build(force: bool = False, verbose: bool = False, extra_flags=(), debug_bounds=False) -> str:
+    build_dir = BUILD_DIR + ("_debug_bounds" if debug_bounds else "")
+    lib = LIB_DEBUG_BOUNDS if debug_bounds else LIB
+    if debug_bounds:
+        extra_flags = tuple(extra_flags) + ("-DKDA_DEBUG_BOUNDS",)
+    os.makedirs(build_dir, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     hdr_time = max((os.path.getmtime(h) for h in _headers()), default=0.0)
     nvcc = _nvcc()
 
     def compile_one(src):
-        obj = os.path.join(BUILD_DIR, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(build_dir, os.path.basename(src)[:-3] + ".o")
         if (not force and os.path.exists(obj)
                 and os.path.getmtime(obj) >= max(os.path.getmtime(src), hdr_time)):
             return obj, False
@@ -59,16 +69,17 @@ def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
         results = list(ex.map(compile_one, srcs))
     objs = [o for o, _ in results]
     changed = any(c for _, c in results)
-    if force or changed or not os.path.exists(LIB) or \
-            os.path.getmtime(LIB) < max(os.path.getmtime(o) for o in objs):
-        tmp = LIB + f".tmp{os.getpid()}"
+    if force or changed or not os.path.exists(lib) or \
+            os.path.getmtime(lib) < max(os.path.getmtime(o) for o in objs):
+        tmp = lib + f".tmp{os.getpid()}"
         cmd = [nvcc, *ARCH, "-shared", "-Xcompiler", "-fPIC", "-o", tmp, *objs]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-        os.replace(tmp, LIB)
-    return LIB
+        os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
     print(build(force="--force" in sys.argv, verbose=True))
+    print(build(force="--force" in sys.argv, verbose=True, debug_bounds=True))

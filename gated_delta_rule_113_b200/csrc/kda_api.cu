@@ -86,6 +86,7 @@ const char *kda_status_string(kda_status s) {
     case KDA_ERR_SLOT: return "KDA_ERR_SLOT: snapshot-pool slot outside the pool";
     case KDA_ERR_DECAY:
         return "KDA_ERR_DECAY: log_alpha > 0 or not finite, or in-chunk cumulative log-decay below -80";
+    case KDA_ERR_BOUNDS: return "KDA_ERR_BOUNDS: index outside its buffer (bounds-checking build)";
     }
     return "KDA_ERR_UNKNOWN";
 }

@@ -253,7 +253,8 @@ rchain_kernel(const __grid_constant__ CUtensorMap tm_do, RcParams p) {
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[rbXbFull]);
-            {   // fp32 dX_j for the assembly, off the chain: after the proxy fence
+            if (KDA_IN_RANGE(((long long)g0 + j) * p.H + h < p.slots, p.status)) {
+                // fp32 dX_j for the assembly, off the chain: after the proxy fence
                 float *dst = p.dxs + ((size_t)(g0 + j) * p.H + h) * kDK * kDV + (size_t)c * kDV +
                              (size_t)vs * VS;
 #pragma unroll
@@ -437,7 +438,9 @@ __global__ void __launch_bounds__(kAsmThreads, 1) assemble_kernel(AsmParams p) {
     const long long m = blockIdx.x;
     if (total < 0 || total > p.slots || m >= total) return;
     const Item it = item_of(m, p.H, p.chunk_off, p.cu, p.N);
-    const int h = it.h, c0 = it.c0, L = it.L;
+    const int h = it.h, c0 = it.c0;
+    // rows past the token axis are never touched (the debug build checks it)
+    const int L = KDA_IN_RANGE(it.L == 0 || (long long)it.c0 + it.L <= p.T, p.status) ? it.L : 0;
     const size_t H = (size_t)p.H;
     auto rowk = [&](int r) { return ((size_t)(c0 + r) * H + h) * kDK; };   // [T, H, 128] row start
 

@@ -158,6 +158,20 @@ __device__ __forceinline__ void set_status(int32_t *status, int32_t code) {
     if (status) atomicCAS(status, 0, code);
 }
 
+// Index checks of the bounds-checking build (-DKDA_DEBUG_BOUNDS): a global
+// access whose index would leave its buffer is skipped and KDA_ERR_BOUNDS is
+// recorded in the status word (no trap).  In the regular build the check is
+// the constant true and compiles away.
+__device__ __forceinline__ bool debug_in_range(bool ok, int32_t *status) {
+    if (!ok) set_status(status, KDA_ERR_BOUNDS);
+    return ok;
+}
+#ifdef KDA_DEBUG_BOUNDS
+#define KDA_IN_RANGE(cond, status) ::kda::debug_in_range((cond), (status))
+#else
+#define KDA_IN_RANGE(cond, status) true
+#endif
+
 // Token range of sequence n, or false when cu_seqlens is malformed there.
 __device__ __forceinline__ bool seq_range(const int32_t *cu, int n, int T, int &t0, int &t1) {
     t0 = cu[n];

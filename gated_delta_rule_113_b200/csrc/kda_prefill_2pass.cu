@@ -360,6 +360,7 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             if (!__shfl_sync(0xffffffffu, ok, 0)) break;
             const int m = items[s].m;
             if (m < 0) break;
+            if (!KDA_IN_RANGE((long long)m < p.slots, p.status)) break;
             unsigned char *dst = p.packets + (size_t)m * kPacketBytes;
             if (lane == 0) {   // PT = P Tb  (M = 64, B = Tb read MN-major)
                 tc_fence_after();
@@ -532,7 +533,7 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                     KDA_TRACE1(i, 3);
                 }
             }
-            if (lane == 1) {
+            if (lane == 1 && KDA_IN_RANGE((long long)m < p.slots, p.status)) {
                 unsigned char *dst = p.packets + (size_t)m * kPacketBytes;
                 bulk_store(dst + kPkKI, sm + Ly::kKI + s * 16384, 16384);
                 bulk_store(dst + kPkGL, sGL + s * 128, 512);
@@ -811,7 +812,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
         auto store_snapshot = [&](int j) {
             if (j <= 0 || snap_base < 0 || j % p.snap_every != 0 || j * kChunk > t1 - t0) return;
             const long long slot = snap_base + j / p.snap_every - 1;
-            if (slot < p.snap_slots) {
+            if (slot < p.snap_slots && KDA_IN_RANGE(slot >= 0, p.status)) {
                 float *dst = p.snap_pool + ((size_t)slot * p.H + h) * kDK * kDV + (size_t)c * kDV +
                              (size_t)vs * VS;
 #pragma unroll
@@ -861,7 +862,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
             if (c == 0) KDA_TRACE2(j, 8);
             // the state entering chunk j, for the chunked backward: stored after
             // the proxy fence above so that fence never waits for it
-            if (p.ckpt) {
+            if (p.ckpt && KDA_IN_RANGE(((long long)g0 + j) * p.H + h < p.slots, p.status)) {
                 float *dst = p.ckpt + ((size_t)(g0 + j) * p.H + h) * kDK * kDV + (size_t)c * kDV +
                              (size_t)vs * VS;
 #pragma unroll
@@ -910,7 +911,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
                     uint32_t v[32];
                     tmem_ld32(tmem_addr(tmem, 32 * wq, Ly::kTmD1 + d * VS + jj), v);
                     tmem_wait_ld();
-                    if (r < L && p.out) {
+                    if (r < L && p.out && KDA_IN_RANGE(c0 + r < p.T, p.status)) {
                         __nv_bfloat16 *dst = p.out + ((size_t)(c0 + r) * p.H + h) * kDV + vs * VS + jj;
 #pragma unroll
                         for (int e = 0; e < 32; e += 8) {
@@ -928,7 +929,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
                 if (lane == 0) mbar_arrive(&bars[cbD1Free + d]);
             }
         }
-        if (ok && p.Sf) {
+        if (ok && p.Sf && KDA_IN_RANGE(seq < p.N, p.status)) {
             float *dst = p.Sf + sbase_g + (size_t)c * kDV;
 #pragma unroll
             for (int jj = 0; jj < VS; jj += 4)

@@ -98,7 +98,7 @@ __global__ void __launch_bounds__(1024) varlen_index_kernel(const int32_t *__res
             const int lj = s_len[j];
             rank += (lj > li) || (lj == li && j < i);
         }
-        order[rank] = i;
+        if (KDA_IN_RANGE(rank < N, status)) order[rank] = i;
     }
 }
 

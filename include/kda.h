@@ -64,7 +64,8 @@ typedef enum kda_status {
     KDA_ERR_TIMEOUT = 6,      /* a bounded device-side wait gave up               */
     KDA_ERR_SEQLENS = 7,      /* device saw cu_seqlens not 0..total_tokens monotone */
     KDA_ERR_SLOT = 8,         /* device saw a snapshot-pool slot outside the pool */
-    KDA_ERR_DECAY = 9         /* device saw a gate outside the chunked form's range */
+    KDA_ERR_DECAY = 9,        /* device saw a gate outside the chunked form's range */
+    KDA_ERR_BOUNDS = 10       /* debug builds only: an index outside its buffer (skipped) */
 } kda_status;
 
 typedef enum kda_dtype {

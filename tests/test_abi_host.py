@@ -38,7 +38,7 @@ def test_library_loads_and_exports_every_declared_symbol():
 
 def test_status_strings():
     lib = kda.load_library()
-    for code in range(0, 10):
+    for code in range(0, 11):
         assert lib.kda_status_string(code).startswith(b"KDA_")
     assert lib.kda_status_string(1234) == b"KDA_ERR_UNKNOWN"
 

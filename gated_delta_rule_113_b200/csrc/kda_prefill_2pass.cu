@@ -560,9 +560,16 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 }
 
 // ============================================================ pass 2
-constexpr int kChWarps = 6;   // 0-3 chain, 4 loader, 5 MMA
-constexpr int kChThreads = kChWarps * 32;
-enum ChRole { kChLoad = 4, kChMma = 5 };
+// Warp roles of the chain pass: kChain chain warps (4, or 8 for 128-wide
+// slices: warp w keeps rows 32 (w % 4) .. + 31 and columns (w / 4) kCols ..
+// + kCols - 1 of the slice), then the loader and the MMA issuer.
+template <int VS>
+struct ChShape {
+    static constexpr int kChain = VS == 128 ? 8 : 4;
+    static constexpr int kCols = VS * 4 / kChain;
+    static constexpr int kLoad = kChain, kMma = kChain + 1;
+    static constexpr int kThreads = (kChain + 2) * 32;
+};
 enum ChBars {
     cbFull = 0,       // [3] packet + value tile landed (two used when VS = 64)
     cbStageFree = 3,  // [3] every product reading a stage done
@@ -584,7 +591,7 @@ struct ChLayout {
     static constexpr uint32_t kV = (kPkGL + 512 + 1023) / 1024 * 1024;
     static constexpr uint32_t kStage = (kV + 64 * VS * 2 + 1023) / 1024 * 1024;
     static_assert(kPkGL + 512 == kPacketBytes, "the packet is one contiguous copy");
-    // three stages fit beside the 32-wide operands, two beside the 64-wide ones
+    // three stages fit beside the 32-wide operands, two beside the wider ones
     static constexpr int kStages = VS == 32 ? 3 : 2;
     static constexpr uint32_t kSB = kStages * kStage;
     static constexpr uint32_t kUB = kSB + 128 * VS * 2;
@@ -628,9 +635,11 @@ struct ChParams {
 // Only the last two steps and the product of the bf16 S with [-W; Qe] lie on
 // the chain from one chunk's state to the next.
 template <int VS>
-__global__ void __launch_bounds__(kChThreads, 1)
+__global__ void __launch_bounds__(ChShape<VS>::kThreads, 1)
 chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
     using Ly = ChLayout<VS>;
+    using Sh = ChShape<VS>;
+    constexpr int kChLoad = Sh::kLoad, kChMma = Sh::kMma, NC = Sh::kCols;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t sbase = smem_u32(sm);
@@ -663,8 +672,8 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
     if (tid == 0) {
         for (int i = 0; i < cbNum; ++i) {
             uint32_t cnt = 1;
-            if (i == cbSbFull) cnt = 4;
-            if (i == cbUbFull || i == cbD1Free || i == cbD1Free + 1) cnt = 2;
+            if (i == cbSbFull) cnt = Sh::kChain;
+            if (i == cbUbFull || i == cbD1Free || i == cbD1Free + 1) cnt = Sh::kChain / 2;
             mbar_init(&bars[i], cnt);
         }
         *abort_flag = 0;
@@ -706,6 +715,8 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
                 bulk_load(st + off, packet(j) + off, len, full);
             }
             if (lane == 4) tma_load_3d(st + Ly::kV, &tm_v, full, vs * VS, h, t0 + j * kChunk);
+            if (VS == 128 && lane == 7)   // the second 64-wide atom of the slice
+                tma_load_3d(st + Ly::kV + 64 * 128, &tm_v, full, 64, h, t0 + j * kChunk);
             if (lane == 5 && j + Ly::kStages < nchunks)
                 bulk_prefetch_l2(packet(j + Ly::kStages), (uint32_t)kPacketBytes);
             n_issued = j + 1;
@@ -784,11 +795,12 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
         }
     } else {
         // ------------------------------------------------------ chain warps
-        const int c = tid;                 // state row (key channel) 0..127
-        const int wq = warp;               // TMEM lane quarter
-        float S[VS];
+        const int wq = warp & 3;           // TMEM lane quarter
+        const int c = 32 * wq + lane;      // state row (key channel) 0..127
+        const int col0 = (warp >> 2) * NC; // this thread's columns of the slice
+        float S[NC];
         {
-            const float *src = p.S0 ? p.S0 + sbase_g + (size_t)c * kDV : nullptr;
+            const float *src = p.S0 ? p.S0 + sbase_g + (size_t)c * kDV + col0 : nullptr;
             if (p.s0_slot) {   // resume from a pool slot (prefix-cache hit)
                 const long long slot = p.s0_slot[seq];
                 if (slot >= p.snap_slots) {
@@ -796,11 +808,11 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
                     src = nullptr;
                 } else if (slot >= 0) {
                     src = p.snap_pool + ((size_t)slot * p.H + h) * kDK * kDV + (size_t)vs * VS +
-                          (size_t)c * kDV;
+                          (size_t)c * kDV + col0;
                 }
             }
 #pragma unroll
-            for (int jj = 0; jj < VS; jj += 4) {
+            for (int jj = 0; jj < NC; jj += 4) {
                 float4 v = src ? *reinterpret_cast<const float4 *>(src + jj) : make_float4(0, 0, 0, 0);
                 S[jj] = v.x; S[jj + 1] = v.y; S[jj + 2] = v.z; S[jj + 3] = v.w;
             }
@@ -814,9 +826,9 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
             const long long slot = snap_base + j / p.snap_every - 1;
             if (slot < p.snap_slots && KDA_IN_RANGE(slot >= 0, p.status)) {
                 float *dst = p.snap_pool + ((size_t)slot * p.H + h) * kDK * kDV + (size_t)c * kDV +
-                             (size_t)vs * VS;
+                             (size_t)vs * VS + col0;
 #pragma unroll
-                for (int jj = 0; jj < VS; jj += 4)
+                for (int jj = 0; jj < NC; jj += 4)
                     *reinterpret_cast<float4 *>(dst + jj) =
                         make_float4(S[jj], S[jj + 1], S[jj + 2], S[jj + 3]);
             } else if (c == 0) {
@@ -830,9 +842,9 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
                 tc_fence_after();
                 if (c == 0) KDA_TRACE2(j - 1, 6);
 #pragma unroll
-                for (int jj = 0; jj < VS; jj += 32) {
+                for (int jj = 0; jj < NC; jj += 32) {
                     uint32_t v[32];
-                    tmem_ld32(tmem_addr(tmem, 32 * wq, Ly::kTmD2 + jj), v);
+                    tmem_ld32(tmem_addr(tmem, 32 * wq, Ly::kTmD2 + col0 + jj), v);
                     tmem_wait_ld();
 #pragma unroll
                     for (int e = 0; e < 32; ++e) S[jj + e] = gl_cur * (S[jj + e] + __uint_as_float(v[e]));
@@ -849,8 +861,8 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
             {
                 const uint32_t sb = sbase + Ly::kSB;
 #pragma unroll
-                for (int q8 = 0; q8 < VS / 8; ++q8) {
-                    sts128(sb + vs_off<VS>(c, q8), pack2(S[8 * q8], S[8 * q8 + 1]),
+                for (int q8 = 0; q8 < NC / 8; ++q8) {
+                    sts128(sb + vs_off<VS>(c, col0 / 8 + q8, 128), pack2(S[8 * q8], S[8 * q8 + 1]),
                            pack2(S[8 * q8 + 2], S[8 * q8 + 3]), pack2(S[8 * q8 + 4], S[8 * q8 + 5]),
                            pack2(S[8 * q8 + 6], S[8 * q8 + 7]));
                 }
@@ -864,9 +876,9 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
             // the proxy fence above so that fence never waits for it
             if (p.ckpt && KDA_IN_RANGE(((long long)g0 + j) * p.H + h < p.slots, p.status)) {
                 float *dst = p.ckpt + ((size_t)(g0 + j) * p.H + h) * kDK * kDV + (size_t)c * kDV +
-                             (size_t)vs * VS;
+                             (size_t)vs * VS + col0;
 #pragma unroll
-                for (int jj = 0; jj < VS; jj += 4)
+                for (int jj = 0; jj < NC; jj += 4)
                     *reinterpret_cast<float4 *>(dst + jj) =
                         make_float4(S[jj], S[jj + 1], S[jj + 2], S[jj + 3]);
             }
@@ -883,13 +895,13 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
                 if (c == 0) KDA_TRACE2(j, 9);
                 const uint32_t ub = sbase + Ly::kUB;
 #pragma unroll
-                for (int jj = 0; jj < VS; jj += 32) {
+                for (int jj = 0; jj < NC; jj += 32) {
                     uint32_t v[32];
-                    tmem_ld32(tmem_addr(tmem, 32 * wq, Ly::kTmD1 + d * VS + jj), v);
+                    tmem_ld32(tmem_addr(tmem, 32 * wq, Ly::kTmD1 + d * VS + col0 + jj), v);
                     tmem_wait_ld();
 #pragma unroll
                     for (int e = 0; e < 32; e += 8) {
-                        sts128(ub + vs_off<VS>(c, (jj + e) / 8),
+                        sts128(ub + vs_off<VS>(c, (col0 + jj + e) / 8, 64),
                                pack2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])),
                                pack2(__uint_as_float(v[e + 2]), __uint_as_float(v[e + 3])),
                                pack2(__uint_as_float(v[e + 4]), __uint_as_float(v[e + 5])),
@@ -907,12 +919,13 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
                 const int c0 = t0 + j * kChunk, L = min(kChunk, t1 - c0);
                 const int r = c - 64;
 #pragma unroll
-                for (int jj = 0; jj < VS; jj += 32) {
+                for (int jj = 0; jj < NC; jj += 32) {
                     uint32_t v[32];
-                    tmem_ld32(tmem_addr(tmem, 32 * wq, Ly::kTmD1 + d * VS + jj), v);
+                    tmem_ld32(tmem_addr(tmem, 32 * wq, Ly::kTmD1 + d * VS + col0 + jj), v);
                     tmem_wait_ld();
                     if (r < L && p.out && KDA_IN_RANGE(c0 + r < p.T, p.status)) {
-                        __nv_bfloat16 *dst = p.out + ((size_t)(c0 + r) * p.H + h) * kDV + vs * VS + jj;
+                        __nv_bfloat16 *dst =
+                            p.out + ((size_t)(c0 + r) * p.H + h) * kDV + vs * VS + col0 + jj;
 #pragma unroll
                         for (int e = 0; e < 32; e += 8) {
                             uint4 w;
@@ -930,9 +943,9 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
             }
         }
         if (ok && p.Sf && KDA_IN_RANGE(seq < p.N, p.status)) {
-            float *dst = p.Sf + sbase_g + (size_t)c * kDV;
+            float *dst = p.Sf + sbase_g + (size_t)c * kDV + col0;
 #pragma unroll
-            for (int jj = 0; jj < VS; jj += 4)
+            for (int jj = 0; jj < NC; jj += 4)
                 *reinterpret_cast<float4 *>(dst + jj) = make_float4(S[jj], S[jj + 1], S[jj + 2], S[jj + 3]);
         }
     }
@@ -982,14 +995,15 @@ cudaError_t launch_dependent(void (*kern)(KArgs...), unsigned grid, unsigned blo
 
 template <int VS>
 cudaError_t launch_chain(const ChParams &cp, int T, cudaStream_t s) {
-    CUtensorMap mv;
-    if (!make_tmap_bf16_3d(&mv, cp.v_base, T, cp.H, kDV, VS, VS * 2)) return cudaErrorInvalidValue;
+    CUtensorMap mv;   // 128-wide slices load their V tile as two 64-wide boxes
+    constexpr int box = VS < 64 ? VS : 64;
+    if (!make_tmap_bf16_3d(&mv, cp.v_base, T, cp.H, kDV, box, box * 2)) return cudaErrorInvalidValue;
     auto kern = chain_kernel<VS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)ChLayout<VS>::kAlloc);
     if (e != cudaSuccess) return e;
     const unsigned grid2 = (unsigned)cp.N * cp.H * (kDV / VS);
-    return launch_dependent(kern, grid2, kChThreads, ChLayout<VS>::kAlloc, s, mv, cp);
+    return launch_dependent(kern, grid2, ChShape<VS>::kThreads, ChLayout<VS>::kAlloc, s, mv, cp);
 }
 
 }  // namespace
@@ -1042,11 +1056,15 @@ cudaError_t launch_prefill_two_pass(const ForwardArgs &a, cudaStream_t s) {
     cp.H = a.H;
     cp.v_base = a.v;
     // pass 2: one CTA per (sequence, head, value slice), longest sequences
-    // first.  32-wide slices give
-    // the most parallel chains; once they would not fit on the GPU in one
-    // wave, 64-wide slices do twice the work per MMA instruction instead.
-    if ((long long)a.N * a.H * (kDV / 32) > sm_count()) return launch_chain<64>(cp, T, s);
-    return launch_chain<32>(cp, T, s);
+    // first.  32-wide slices give the most parallel chains (the chain is then
+    // bound by its per-chunk latency); once they would not fit on the GPU in
+    // one wave the pass is bound by shared-memory traffic, which wider slices
+    // cut per chunk and head: the packet lands once instead of two or four
+    // times, and a wider MMA reads its A operand once for more columns.
+    const long long chains = (long long)a.N * a.H;
+    if (chains * (kDV / 32) <= sm_count()) return launch_chain<32>(cp, T, s);
+    if (chains * (kDV / 64) <= sm_count()) return launch_chain<64>(cp, T, s);
+    return launch_chain<128>(cp, T, s);
 }
 
 }  // namespace kda

@@ -84,25 +84,23 @@ constexpr uint32_t kPkGL = 65536;
 static_assert(kPkGL + 512 <= kPacketBytes, "packet layout");
 
 // PT = P Tb from its M = 64 accumulator (row r in TMEM lane 32 (r / 16) +
-// r % 16) to bf16 rows 64..127 of the Tb|PT tile, by the four solve warps:
-// warp sw reads lane quarter sw, all 64 columns.
-__device__ __forceinline__ void convert_pt4(int sw, int lane, uint32_t tmem, uint32_t tm_pt,
+// r % 16) to bf16 rows 64..127 of the Tb|PT tile, by the eight prep warps:
+// warp w reads lane quarter w % 4, columns 32 (w / 4) .. + 31.
+__device__ __forceinline__ void convert_pt8(int w, int lane, uint32_t tmem, uint32_t tm_pt,
                                             uint32_t tp) {
+    const int qt = w & 3, hh = w >> 2;
+    uint32_t v[32];
+    tmem_ld32(tmem_addr(tmem, 32 * qt, tm_pt + 32 * hh), v);
+    tmem_wait_ld();
+    if (lane < 16) {
+        const int r = 64 + 16 * qt + lane;
 #pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-        uint32_t v[32];
-        tmem_ld32(tmem_addr(tmem, 32 * sw, tm_pt + 32 * hh), v);
-        tmem_wait_ld();
-        if (lane < 16) {
-            const int r = 64 + 16 * sw + lane;
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                sts128(tp + sw128_off(r, 4 * hh + j),
-                       pack2(__uint_as_float(v[8 * j]), __uint_as_float(v[8 * j + 1])),
-                       pack2(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3])),
-                       pack2(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5])),
-                       pack2(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7])));
-        }
+        for (int j = 0; j < 4; ++j)
+            sts128(tp + sw128_off(r, 4 * hh + j),
+                   pack2(__uint_as_float(v[8 * j]), __uint_as_float(v[8 * j + 1])),
+                   pack2(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3])),
+                   pack2(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5])),
+                   pack2(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7])));
     }
     fence_proxy_async();
     tc_fence_before();
@@ -158,12 +156,12 @@ enum KsBars {
     kbApFree = 8,    // [2] solve has read D_AP[s] -> A/P issuer
     kbTbFull = 10,   // solve -> PT issuer (Tb and P final, D_AP read)
     kbPtAcc = 11,    // PT = P Tb product -> solve warps
-    kbPtReady = 12,  // count 4: PT written as bf16 (solve warps) -> W issuer
+    kbPtReady = 12,  // count 8: PT written as bf16 (prep warps) -> W issuer
     kbTpFree = 13,   // the Tb|PT tile has been read -> Tb write of the next chunk
     kbWaccFull = 14, // [W; PW] product -> prep warps
     kbWReady = 15,   // count 8: -W and Qe written -> stores (and D_W free)
     kbStored = 16,   // [3] every store of a stage has read shared memory -> TMA
-    kbKiFree = 19,   // [3] Ki and Gam_L have been read out of the stage
+    kbKiFree = 19,   // [3] count 3: Ki and Gam_L have been read out of the stage
     kbDrain = 22,    // [2] A/P issuer, PT/W issuer
     kbNum = 24
 };
@@ -242,7 +240,8 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             uint32_t cnt = 1;
             if (i >= kbKqFull && i < kbKqFull + kKsStages) cnt = kPrepThreads / 32;
             if (i == kbWReady) cnt = kPrepThreads / 32;
-            if (i == kbPtReady) cnt = 4;
+            if (i == kbPtReady) cnt = kPrepThreads / 32;
+            if (i >= kbKiFree && i < kbKiFree + kKsStages) cnt = 3;
             mbar_init(&bars[i], cnt);
         }
         *abort_flag = 0;
@@ -393,8 +392,8 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 ok = wait_or_abort(&bars[kbWReady], i & 1, abort_flag, p.status);
             }
             if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-            if (lane < 2) {   // [-W; Qe], one 16 KB atom per lane
-                bulk_store(dst + kPkKQ + lane * 16384, kq + lane * 16384, 16384);
+            if (lane < 4) {   // [-W; Qe] in four 8 KB pieces, one per lane
+                bulk_store(dst + kPkKQ + lane * 8192, kq + lane * 8192, 8192);
                 bulk_commit();
             }
             if (lane == 0) KDA_TRACE1(i, 9);
@@ -416,10 +415,16 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     } else if (warp >= kKsPrep0 && warp < kKsPrep0 + kPrepThreads / 32) {
         // ----------------------------------------------------------- prep
         const int t = tid - kKsPrep0 * 32;
-        // After preparing chunk i these warps turn chunk i-1's [W; PW] product
-        // into the bf16 -W and Qe operands (the solve warps convert PT).
+        // After preparing chunk i these warps turn chunk i-1's products into
+        // bf16 operands: PT into rows 64-127 of the Tb|PT tile, then [W; PW]
+        // into -W and Qe.
         auto convert = [&](int m) -> bool {
             const int sm3 = m % kKsStages;
+            // PT = P Tb first: the [W; PW] product waits for it
+            if (!wait_or_abort(&bars[kbPtAcc], m & 1, abort_flag, p.status)) return false;
+            tc_fence_after();
+            convert_pt8(warp, lane, tmem, Ly::kTmPT, sbase + Ly::kTP);
+            if (lane == 0) mbar_arrive(&bars[kbPtReady]);
             if (!wait_or_abort(&bars[kbWaccFull], m & 1, abort_flag, p.status)) return false;
             tc_fence_after();
             if (t == 0) KDA_TRACE1(m, 7);
@@ -487,16 +492,9 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 mbar_arrive(&bars[kbTbFull]);
             }
             if (t == 0) KDA_TRACE1(i, 5);
-            // PT = P Tb (issued by the store warp) -> bf16 rows 64-127 of the
-            // Tb|PT tile, here rather than by the prep warps, which are busy
-            // with the next chunk by then
-            if (!wait_or_abort(&bars[kbPtAcc], i & 1, abort_flag, p.status)) break;
-            tc_fence_after();
-            convert_pt4(sw, lane, tmem, Ly::kTmPT, sbase + Ly::kTP);
-            if (lane == 0) mbar_arrive(&bars[kbPtReady]);
         }
     } else if (warp == kKsMma) {
-        // --------------------------------- A/P issuer (lane 0), Ki stores (lane 1)
+        // ------------------------------ A/P issuer (lane 0), Ki stores (lanes 1-3)
         // Ki and Gam_L are final once the prep is done.  They leave from here,
         // as soon as they are, rather than from the store warp, which works on
         // the products that follow the solve.
@@ -515,8 +513,8 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                     mbar_arrive(&bars[kbApFull + a]);
                 break;
             }
-            // the product first: lane 1's bulk store blocks the warp until its
-            // copy has read shared memory
+            // the product first: the bulk stores block the warp until their
+            // copies have read shared memory
             if (lane == 0) {
                 const uint32_t kq = sbase + Ly::kKQ + s * 32768;
                 const uint64_t d_kq = smem_desc(kq, 16, 1024, kSw128);
@@ -533,12 +531,16 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                     KDA_TRACE1(i, 3);
                 }
             }
-            if (lane == 1 && KDA_IN_RANGE((long long)m < p.slots, p.status)) {
-                unsigned char *dst = p.packets + (size_t)m * kPacketBytes;
-                bulk_store(dst + kPkKI, sm + Ly::kKI + s * 16384, 16384);
-                bulk_store(dst + kPkGL, sGL + s * 128, 512);
-                bulk_commit();
-                bulk_wait_read_all();
+            if (lane >= 1 && lane <= 3) {   // Ki (two 8 KB atoms) and Gam_L, one copy per lane
+                if (KDA_IN_RANGE((long long)m < p.slots, p.status)) {
+                    unsigned char *dst = p.packets + (size_t)m * kPacketBytes;
+                    if (lane < 3)
+                        bulk_store(dst + kPkKI + (lane - 1) * 8192, sm + Ly::kKI + s * 16384 + (lane - 1) * 8192, 8192);
+                    else
+                        bulk_store(dst + kPkGL, sGL + s * 128, 512);
+                    bulk_commit();
+                    bulk_wait_read_all();
+                }
                 mbar_arrive(&bars[kbKiFree + s]);
             }
             if (!__shfl_sync(0xffffffffu, ok, 0)) break;
@@ -717,8 +719,11 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
             if (lane == 4) tma_load_3d(st + Ly::kV, &tm_v, full, vs * VS, h, t0 + j * kChunk);
             if (VS == 128 && lane == 7)   // the second 64-wide atom of the slice
                 tma_load_3d(st + Ly::kV + 64 * 128, &tm_v, full, 64, h, t0 + j * kChunk);
-            if (lane == 5 && j + Ly::kStages < nchunks)
-                bulk_prefetch_l2(packet(j + Ly::kStages), (uint32_t)kPacketBytes);
+            if (j + Ly::kStages < nchunks) {   // warm L2 for the copies of chunk j + kStages
+                if (lane == 5) bulk_prefetch_l2(packet(j + Ly::kStages), (uint32_t)kPacketBytes);
+                if (lane == 8) tma_prefetch_3d(&tm_v, vs * VS, h, t0 + (j + Ly::kStages) * kChunk);
+                if (VS == 128 && lane == 9) tma_prefetch_3d(&tm_v, 64, h, t0 + (j + Ly::kStages) * kChunk);
+            }
             n_issued = j + 1;
             if (lane == 0) KDA_TRACE2(j, 0);
 #ifdef KDA_TRACE
@@ -778,7 +783,18 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
                     mma_bf16(d1, d_kq + kmaj_step(ks, 16384), d_sb + vs_step<VS>(ks), kIdV, 1);
                 mma_commit(&bars[cbUFull]);
                 KDA_TRACE2(j, 3);
-                if (j + 1 < nchunks && !issue_u0(j + 1)) break;
+                // The next chunk's [Tb; PT] V goes in now if its tiles have
+                // landed; otherwise after dS, which must not queue behind a
+                // copy still in flight.
+                bool u0_next = j + 1 >= nchunks;
+                if (!u0_next) {
+                    const int s1 = (j + 1) % Ly::kStages, d1n = (j + 1) & 1;
+                    if (mbar_test_wait(&bars[cbFull + s1], ((j + 1) / Ly::kStages) & 1) &&
+                        (j + 1 < 2 || mbar_test_wait(&bars[cbD1Free + d1n], ((j - 1) >> 1) & 1))) {
+                        if (!issue_u0(j + 1)) break;
+                        u0_next = true;
+                    }
+                }
                 if (!spin_or_abort(&bars[cbUbFull], j & 1, abort_flag, p.status)) break;
                 KDA_TRACE2(j, 4);
                 tc_fence_after();
@@ -789,6 +805,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
                 mma_commit(&bars[cbDsFull]);
                 mma_commit(&bars[cbStageFree + s]);
                 KDA_TRACE2(j, 5);
+                if (!u0_next && !issue_u0(j + 1)) break;
             }
             mma_commit(&bars[cbDrain]);
             mbar_wait(&bars[cbDrain], 0);

@@ -114,7 +114,9 @@ __device__ __forceinline__ void convert_wqe8(int w, int lane, uint32_t tmem, uin
                                              uint32_t kq_stage) {
     const int qt = w & 3, hh = w >> 2;
     const int r = 32 * qt + lane;
-#pragma unroll
+    // one code path for both halves: -W = 0 - W over the Kg rows, Qe = Qg - PW
+    const uint32_t keep = qt < 2 ? 0u : 0xFFFFFFFFu;
+#pragma unroll 1
     for (int half = 0; half < 2; ++half) {
         uint32_t v[32];
         tmem_ld32(tmem_addr(tmem, 32 * qt, tm_w + 64 * hh + 32 * half), v);
@@ -122,20 +124,13 @@ __device__ __forceinline__ void convert_wqe8(int w, int lane, uint32_t tmem, uin
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const uint32_t addr = kq_stage + hh * 16384 + sw128_off(r, 4 * half + j);
+            const uint4 qv = lds128(addr);
+            const uint32_t qw[4] = {qv.x & keep, qv.y & keep, qv.z & keep, qv.w & keep};
             uint32_t o[4];
-            if (qt < 2) {
 #pragma unroll
-                for (int e2 = 0; e2 < 4; ++e2)
-                    o[e2] = pack2(-__uint_as_float(v[8 * j + 2 * e2]),
-                                  -__uint_as_float(v[8 * j + 2 * e2 + 1]));
-            } else {
-                const uint4 qv = lds128(addr);
-                const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
-#pragma unroll
-                for (int e2 = 0; e2 < 4; ++e2)
-                    o[e2] = pack2(bf16lo(qw[e2]) - __uint_as_float(v[8 * j + 2 * e2]),
-                                  bf16hi(qw[e2]) - __uint_as_float(v[8 * j + 2 * e2 + 1]));
-            }
+            for (int e2 = 0; e2 < 4; ++e2)
+                o[e2] = pack2(bf16lo(qw[e2]) - __uint_as_float(v[8 * j + 2 * e2]),
+                              bf16hi(qw[e2]) - __uint_as_float(v[8 * j + 2 * e2 + 1]));
             sts128(addr, o[0], o[1], o[2], o[3]);
         }
     }
@@ -148,40 +143,42 @@ __device__ __forceinline__ void convert_wqe8(int w, int lane, uint32_t tmem, uin
 constexpr int kKsWarps = 15;   // 0-7 prep, 8-11 solve, 12 TMA loads, 13 MMA, 14 packet stores
 constexpr int kKsThreads = kKsWarps * 32;
 enum KsRole { kKsPrep0 = 0, kKsSolve0 = 8, kKsTma = 12, kKsMma = 13, kKsStore = 14 };
-constexpr int kKsStages = 3;   // ring depth of the raw/processed key-query tiles
+// Item i holds key-query stage i % kKqStages from its load until its packet
+// has left (most of the pipeline) and gate stage i % kKiStages only until the
+// A/P product and the Ki store have read it, so the key-query ring is deeper.
+constexpr int kKqStages = 4;   // raw k|q -> Kg|Qg -> -W|Qe
+constexpr int kKiStages = 2;   // raw log_alpha -> prefix scratch -> Ki
 enum KsBars {
-    kbRawFull = 0,   // [3] TMA -> prep
-    kbKqFull = 3,    // [3] count 8: prep -> A/P issuer, stores (Ki, Gam_L final)
-    kbApFull = 6,    // [2] A/P product -> solve (two TMEM accumulators)
-    kbApFree = 8,    // [2] solve has read D_AP[s] -> A/P issuer
-    kbTbFull = 10,   // solve -> PT issuer (Tb and P final, D_AP read)
-    kbPtAcc = 11,    // PT = P Tb product -> solve warps
-    kbPtReady = 12,  // count 8: PT written as bf16 (prep warps) -> W issuer
-    kbTpFree = 13,   // the Tb|PT tile has been read -> Tb write of the next chunk
-    kbWaccFull = 14, // [W; PW] product -> prep warps
-    kbWReady = 15,   // count 8: -W and Qe written -> stores (and D_W free)
-    kbStored = 16,   // [3] every store of a stage has read shared memory -> TMA
-    kbKiFree = 19,   // [3] count 3: Ki and Gam_L have been read out of the stage
-    kbDrain = 22,    // [2] A/P issuer, PT/W issuer
-    kbNum = 24
+    kbRawFull = 0,   // [4] TMA -> prep (per key-query stage; covers the gate tiles)
+    kbKqFull = 4,    // [4] count 8: prep -> A/P issuer, Ki stores
+    kbApFull = 8,    // [2] A/P product -> solve (two TMEM accumulators)
+    kbApFree = 10,   // [2] solve has read D_AP[s] -> A/P issuer
+    kbTbFull = 12,   // solve -> PT issuer (Tb and P final)
+    kbPtAcc = 13,    // PT = P Tb product -> prep warps (convert), solve (P tile free)
+    kbPtReady = 14,  // count 8: PT written as bf16 (prep warps) -> W issuer
+    kbTpFree = 15,   // the Tb|PT tile has been read -> Tb write of the next chunk
+    kbWaccFull = 16, // [W; PW] product -> prep warps
+    kbWReady = 17,   // count 8: -W and Qe written -> stores (and D_W free)
+    kbStored = 18,   // [4] the packet's -W|Qe copies have read the key-query stage -> TMA
+    kbKiFree = 22,   // [2] count 4: A/P product done, Ki and Gam_L copies read -> TMA
+    kbDrain = 24,    // [2] A/P issuer, PT/W issuer
+    kbNum = 26
 };
 
 struct KsLayout {
-    static constexpr uint32_t kKQ = 0;                              // 3 x 32 KB
-    static constexpr uint32_t kKI = kKQ + kKsStages * 32768;        // 3 x 16 KB
-    static constexpr uint32_t kTP = kKI + kKsStages * 16384;        // 16 KB: Tb | PT
+    static constexpr uint32_t kKQ = 0;                              // 4 x 32 KB
+    static constexpr uint32_t kKI = kKQ + kKqStages * 32768;        // 2 x 16 KB (also the prep's scan scratch)
+    static constexpr uint32_t kTP = kKI + kKiStages * 16384;        // 16 KB: Tb | PT
     static constexpr uint32_t kP = kTP + 16384;                       // 8 KB: P
     static constexpr uint32_t kL = kP + 8192;
     static constexpr uint32_t kT = kL + 64 * kLDL * 4;
     static constexpr uint32_t kXw = kT + 64 * kLDL * 4;     // fp32 4 x [16][17]
-    static constexpr uint32_t kGP = kXw + 4 * 16 * 17 * 4;
-    static constexpr uint32_t kSUF = kGP + 16 * 128 * 4;
-    static constexpr uint32_t kGL = kSUF + 16 * 128 * 4;    // [3][128]
-    static constexpr uint32_t kB = kGL + kKsStages * 128 * 4;       // [3][64]
-    static constexpr uint32_t kBar = kB + kKsStages * 64 * 4;
-    static constexpr uint32_t kMisc = kBar + 24 * 8;
-    static constexpr uint32_t kItem = kMisc + 16;   // [3] Item of the tile in each stage
-    static constexpr uint32_t kAlloc = kItem + kKsStages * sizeof(Item) + 1024;
+    static constexpr uint32_t kGL = kXw + 4 * 16 * 17 * 4;  // [2][128], per gate stage
+    static constexpr uint32_t kB = kGL + kKiStages * 128 * 4;       // [4][64], per key-query stage
+    static constexpr uint32_t kBar = kB + kKqStages * 64 * 4;
+    static constexpr uint32_t kMisc = kBar + kbNum * 8;
+    static constexpr uint32_t kItem = kMisc + 16;   // [4] Item of each key-query stage
+    static constexpr uint32_t kAlloc = kItem + kKqStages * sizeof(Item) + 1024;
     static_assert(kAlloc <= 232448, "shared memory budget exceeded");
     static constexpr uint32_t kTmAP = 0;     // + (i & 1) * 64 (two A/P accumulators)
     static constexpr uint32_t kTmW = 128;    // [W; PW], 128 columns
@@ -213,8 +210,6 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     float *sL = reinterpret_cast<float *>(sm + Ly::kL);
     float *sT = reinterpret_cast<float *>(sm + Ly::kT);
     float *sXw = reinterpret_cast<float *>(sm + Ly::kXw);
-    float *sGP = reinterpret_cast<float *>(sm + Ly::kGP);
-    float *sSUF = reinterpret_cast<float *>(sm + Ly::kSUF);
     float *sGL = reinterpret_cast<float *>(sm + Ly::kGL);
     float *sB = reinterpret_cast<float *>(sm + Ly::kB);
 
@@ -238,10 +233,10 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     if (tid == 0) {
         for (int i = 0; i < kbNum; ++i) {
             uint32_t cnt = 1;
-            if (i >= kbKqFull && i < kbKqFull + kKsStages) cnt = kPrepThreads / 32;
+            if (i >= kbKqFull && i < kbKqFull + kKqStages) cnt = kPrepThreads / 32;
             if (i == kbWReady) cnt = kPrepThreads / 32;
             if (i == kbPtReady) cnt = kPrepThreads / 32;
-            if (i >= kbKiFree && i < kbKiFree + kKsStages) cnt = 3;
+            if (i >= kbKiFree && i < kbKiFree + kKiStages) cnt = 4;
             mbar_init(&bars[i], cnt);
         }
         *abort_flag = 0;
@@ -269,7 +264,6 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         // ------------------------------------------------------ TMA loads
         // Copies issued by one thread are serviced one after another, so each
         // of the six tiles of a stage is issued by its own lane.
-        static_assert(kKsStages == 3, "the look-ahead below keeps three items");
         // Items are claimed three ahead of their load so their tiles can be
         // warmed in L2; lane 0 claims and looks the coordinates up (global
         // memory) and broadcasts them.
@@ -302,15 +296,19 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         warm(nx2);
         int n_loaded = 0;
         bool ended = false;
+#pragma unroll 1
         for (int i = 0;; ++i) {
-            const int s = i % kKsStages;
+            const int s = i % kKqStages, si = i % kKiStages;
             const Item it = nx0;
             nx0 = nx1;
             nx1 = nx2;
-            // the packet of item i-3 must have left stage s
+            // the packet of item i-4 must have left key-query stage s
             bool ok = true;
-            if (lane == 0 && i >= kKsStages)
-                ok = wait_or_abort(&bars[kbStored + s], ((i / kKsStages) - 1) & 1, abort_flag, p.status);
+            if (lane == 0 && i >= kKqStages)
+                ok = wait_or_abort(&bars[kbStored + s], ((i / kKqStages) - 1) & 1, abort_flag, p.status);
+            // and item i-2 must be done with gate stage si
+            if (lane == 0 && ok && it.m >= 0 && i >= kKiStages)
+                ok = wait_or_abort(&bars[kbKiFree + si], ((i / kKiStages) - 1) & 1, abort_flag, p.status);
             if (!__shfl_sync(0xffffffffu, ok, 0)) break;
             uint64_t *full = &bars[kbRawFull + s];
             if (it.m < 0) {   // no more items: tell the prep, which tells the rest
@@ -328,7 +326,7 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             __syncwarp();
             if (lane < 6) {
                 const uint32_t dst = which < 2 ? Ly::kKQ + s * 32768 + a * 16384 + which * 8192
-                                               : Ly::kKI + s * 16384 + a * 8192;
+                                               : Ly::kKI + si * 16384 + a * 8192;
                 tma_load_3d(sm + dst, tm, full, a * 64, it.h, it.c0);
             }
             if (lane == 0) KDA_TRACE1(i, 0);
@@ -337,17 +335,18 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             warm(nx2);
         }
         // Armed loads must land before the CTA may exit.  The end marker went
-        // to the stage of item n_loaded - 3, whose load the Stored wait above
+        // to the stage of item n_loaded - 4, whose load the Stored wait above
         // already saw consumed (and whose phase the marker has moved past).
         if (lane == 0)
-            for (int i = max(0, n_loaded - kKsStages + (ended ? 1 : 0)); i < n_loaded; ++i)
-                mbar_wait(&bars[kbRawFull + i % kKsStages], (i / kKsStages) & 1);
+            for (int i = max(0, n_loaded - kKqStages + (ended ? 1 : 0)); i < n_loaded; ++i)
+                mbar_wait(&bars[kbRawFull + i % kKqStages], (i / kKqStages) & 1);
     } else if (warp == kKsStore) {
         // ------------------------------------------------- packet stores
         // Lane 0 waits and issues the products that follow the solve; the
         // copies are spread over lanes, each lane tracking its own groups.
+#pragma unroll 1
         for (int i = 0;; ++i) {
-            const int s = i % kKsStages;
+            const int s = i % kKqStages;
             unsigned char *kq = sm + Ly::kKQ + s * 32768;
             unsigned char *tp = sm + Ly::kTP;
             bool ok = true;
@@ -398,10 +397,7 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             }
             if (lane == 0) KDA_TRACE1(i, 9);
             bulk_wait_read_all();
-            // Ki and Gam_L leave from the A/P warp; their reads finished too
-            if (lane == 0)
-                ok = wait_or_abort(&bars[kbKiFree + s], (i / kKsStages) & 1, abort_flag, p.status);
-            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+            __syncwarp();
             if (lane == 0) {
                 KDA_TRACE1(i, 10);
                 mbar_arrive(&bars[kbStored + s]);
@@ -418,55 +414,68 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         // After preparing chunk i these warps turn chunk i-1's products into
         // bf16 operands: PT into rows 64-127 of the Tb|PT tile, then [W; PW]
         // into -W and Qe.
+        // Thread 0 waits on each mbarrier and named_bar_or() shares the
+        // outcome: the eight warps leave together on a failed wait, so none is
+        // left at one of prep_chunk's named barriers.
         auto convert = [&](int m) -> bool {
-            const int sm3 = m % kKsStages;
+            const int sm4 = m % kKqStages;
             // PT = P Tb first: the [W; PW] product waits for it
-            if (!wait_or_abort(&bars[kbPtAcc], m & 1, abort_flag, p.status)) return false;
+            bool w = t != 0 || wait_or_abort(&bars[kbPtAcc], m & 1, abort_flag, p.status);
+            if (named_bar_or(1, kPrepThreads, !w)) return false;
             tc_fence_after();
             convert_pt8(warp, lane, tmem, Ly::kTmPT, sbase + Ly::kTP);
             if (lane == 0) mbar_arrive(&bars[kbPtReady]);
-            if (!wait_or_abort(&bars[kbWaccFull], m & 1, abort_flag, p.status)) return false;
+            w = t != 0 || wait_or_abort(&bars[kbWaccFull], m & 1, abort_flag, p.status);
+            if (named_bar_or(1, kPrepThreads, !w)) return false;
             tc_fence_after();
             if (t == 0) KDA_TRACE1(m, 7);
-            convert_wqe8(warp, lane, tmem, Ly::kTmW, sbase + Ly::kKQ + sm3 * 32768);
+            convert_wqe8(warp, lane, tmem, Ly::kTmW, sbase + Ly::kKQ + sm4 * 32768);
             if (lane == 0) mbar_arrive(&bars[kbWReady]);
             if (t == 0) KDA_TRACE1(m, 8);
             return true;
         };
-        bool ok = true;
+        // Iteration i prepares item i (while there is one) and then converts
+        // item i-1; the end marker stops the preps, one more pass converts
+        // the last item.  One call site each keeps the code small.
         int n_items = 0;
+        bool more = true;
+#pragma unroll 1
         for (int i = 0;; ++i) {
-            const int s = i % kKsStages;
-            if (!wait_or_abort(&bars[kbRawFull + s], (i / kKsStages) & 1, abort_flag, p.status)) {
-                ok = false;
-                break;
-            }
-            const Item it = items[s];
-            if (it.m < 0) {   // pass the end on
+            if (more) {
+                const int s = i % kKqStages, si = i % kKiStages;
+                const bool w = t != 0 || wait_or_abort(&bars[kbRawFull + s], (i / kKqStages) & 1,
+                                                       abort_flag, p.status);
+                if (named_bar_or(1, kPrepThreads, !w)) break;
+                const Item it = items[s];
+                if (it.m < 0) {   // pass the end on
+                    more = false;
+                } else {
+                    if (t == 0) KDA_TRACE1(i, 1);
+                    float *scratch = reinterpret_cast<float *>(sm + Ly::kKI + si * 16384);
+                    prep_chunk<true>(t, sbase + Ly::kKQ + s * 32768, sbase + Ly::kKI + si * 16384,
+                                     scratch, scratch + 16 * 128, sGL + si * 128, sB + s * 64,
+                                     p.beta, it.c0, it.L, p.H, it.h, 1, p.status);
+                    if (t == 0) KDA_TRACE1(i, 2);
+                    n_items = i + 1;
+                }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars[kbKqFull + s]);
-                break;
             }
-            if (t == 0) KDA_TRACE1(i, 1);
-            prep_chunk(t, sbase + Ly::kKQ + s * 32768, sbase + Ly::kKI + s * 16384, sGP, sSUF,
-                       sGL + s * 128, sB + s * 64, p.beta, it.c0, it.L, p.H, it.h, 1, p.status);
-            if (t == 0) KDA_TRACE1(i, 2);
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[kbKqFull + s]);
-            n_items = i + 1;
-            if (i >= 1 && !convert(i - 1)) {
-                ok = false;
-                break;
-            }
+            if (i >= 1 && i - 1 < n_items && !convert(i - 1)) break;
+            if (!more) break;
         }
-        if (ok && n_items > 0) convert(n_items - 1);
     } else if (warp >= kKsSolve0 && warp < kKsSolve0 + 4) {
         // ---------------------------------------------------------- solve
         const int sw = warp - kKsSolve0;
         const int t = tid - kKsSolve0 * 32;
+        // One thread waits on each mbarrier and named_bar_or() shares the
+        // outcome, so the four warps leave together on a failed wait and never
+        // strand one another at a named barrier.
+#pragma unroll 1
         for (int i = 0;; ++i) {
-            const int s = i % kKsStages, a = i & 1;
-            if (!wait_or_abort(&bars[kbApFull + a], (i >> 1) & 1, abort_flag, p.status)) break;
+            const int s = i % kKqStages, a = i & 1;
+            bool ok = t != 0 || wait_or_abort(&bars[kbApFull + a], (i >> 1) & 1, abort_flag, p.status);
+            if (named_bar_or(2, kSolveThreads, !ok)) break;
             if (items[s].m < 0) {   // pass the end on, after the store warp has taken
                                     // TbFull's previous phase (TpFree follows it)
                 if (t == 0 && (i < 1 || wait_or_abort(&bars[kbTpFree], (i - 1) & 1, abort_flag,
@@ -476,21 +485,26 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             }
             tc_fence_after();
             if (t == 0) KDA_TRACE1(i, 4);
-            solve_chunk<false>(sw, lane, tmem, Ly::kTmAP + a * 64, sbase + Ly::kP, sL, sT, sXw,
-                               sB + s * 64, nullptr, 2);
-            // P leaves TMEM only now: the previous chunk's PT product must be
-            // done with the P tile, which by this time it long is
-            if (i >= 1 && sw >= 2 && !wait_or_abort(&bars[kbPtAcc], (i - 1) & 1, abort_flag, p.status))
-                break;
-            write_p(sw, lane, tmem, Ly::kTmAP + a * 64, sbase + Ly::kP);
-            tc_fence_before();
-            // the previous chunk's Tb|PT tile must have been read
-            if (i >= 1 && !wait_or_abort(&bars[kbTpFree], (i - 1) & 1, abort_flag, p.status)) break;
-            write_tb(sw, lane, sbase + Ly::kTP, sT, sB + s * 64, 2);
-            if (t == 0) {
-                mbar_arrive(&bars[kbApFree + a]);
-                mbar_arrive(&bars[kbTbFull]);
+            // D_AP -> L (warps 0, 1: rows 0-63) and -> the bf16 P tile (warps
+            // 2, 3: rows 64-127), side by side; the P tile is free once the
+            // previous chunk's PT product is done
+            if (sw < 2) {
+                build_l(sw, lane, tmem, Ly::kTmAP + a * 64, sL, sB + s * 64);
+            } else {
+                if (lane == 0 && i >= 1)
+                    ok = wait_or_abort(&bars[kbPtAcc], (i - 1) & 1, abort_flag, p.status);
+                if (__shfl_sync(0xffffffffu, ok, 0)) write_p(sw, lane, tmem, Ly::kTmAP + a * 64, sbase + Ly::kP);
+                ok = __shfl_sync(0xffffffffu, ok, 0);
             }
+            tc_fence_before();
+            if (named_bar_or(2, kSolveThreads, !ok)) break;
+            if (t == 0) mbar_arrive(&bars[kbApFree + a]);
+            invert_unit_lower(sw, lane, sL, sT, sXw, 2);
+            // the previous chunk's Tb|PT tile must have been read
+            if (t == 0 && i >= 1) ok = wait_or_abort(&bars[kbTpFree], (i - 1) & 1, abort_flag, p.status);
+            if (named_bar_or(2, kSolveThreads, !ok)) break;
+            write_tb(sw, lane, sbase + Ly::kTP, sT, sB + s * 64, 2);
+            if (t == 0) mbar_arrive(&bars[kbTbFull]);
             if (t == 0) KDA_TRACE1(i, 5);
         }
     } else if (warp == kKsMma) {
@@ -499,11 +513,12 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         // as soon as they are, rather than from the store warp, which works on
         // the products that follow the solve.
         constexpr uint32_t kIdAP = idesc_bf16(128, 64, 0, 0);
+#pragma unroll 1
         for (int i = 0;; ++i) {
-            const int s = i % kKsStages, a = i & 1;
+            const int s = i % kKqStages, si = i % kKiStages, a = i & 1;
             bool ok = true;
             if (lane == 0)
-                ok = wait_or_abort(&bars[kbKqFull + s], (i / kKsStages) & 1, abort_flag, p.status);
+                ok = wait_or_abort(&bars[kbKqFull + s], (i / kKqStages) & 1, abort_flag, p.status);
             if (!__shfl_sync(0xffffffffu, ok, 0)) break;
             const int m = items[s].m;
             if (m < 0) {   // pass the end on, after the same wait a product takes,
@@ -518,7 +533,7 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             if (lane == 0) {
                 const uint32_t kq = sbase + Ly::kKQ + s * 32768;
                 const uint64_t d_kq = smem_desc(kq, 16, 1024, kSw128);
-                const uint64_t d_ki = smem_desc(sbase + Ly::kKI + s * 16384, 16, 1024, kSw128);
+                const uint64_t d_ki = smem_desc(sbase + Ly::kKI + si * 16384, 16, 1024, kSw128);
                 if (i >= 2)
                     ok = wait_or_abort(&bars[kbApFree + a], ((i - 2) >> 1) & 1, abort_flag, p.status);
                 if (ok) {
@@ -528,6 +543,7 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                         mma_bf16(tmem + Ly::kTmAP + a * 64, d_kq + kmaj_step(ks, 16384),
                                  d_ki + kmaj_step(ks, 8192), kIdAP, ks > 0);
                     mma_commit(&bars[kbApFull + a]);
+                    mma_commit(&bars[kbKiFree + si]);   // the product has read the gate stage
                     KDA_TRACE1(i, 3);
                 }
             }
@@ -535,13 +551,14 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 if (KDA_IN_RANGE((long long)m < p.slots, p.status)) {
                     unsigned char *dst = p.packets + (size_t)m * kPacketBytes;
                     if (lane < 3)
-                        bulk_store(dst + kPkKI + (lane - 1) * 8192, sm + Ly::kKI + s * 16384 + (lane - 1) * 8192, 8192);
+                        bulk_store(dst + kPkKI + (lane - 1) * 8192,
+                                   sm + Ly::kKI + si * 16384 + (lane - 1) * 8192, 8192);
                     else
-                        bulk_store(dst + kPkGL, sGL + s * 128, 512);
+                        bulk_store(dst + kPkGL, sGL + si * 128, 512);
                     bulk_commit();
                     bulk_wait_read_all();
                 }
-                mbar_arrive(&bars[kbKiFree + s]);
+                mbar_arrive(&bars[kbKiFree + si]);
             }
             if (!__shfl_sync(0xffffffffu, ok, 0)) break;
         }
@@ -701,6 +718,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
         // One copy for the packet (lane 0) and one for the value tile (lane
         // 1): copies from different threads are serviced concurrently.
         int n_issued = 0;
+#pragma unroll 1
         for (int j = 0; j < nchunks; ++j) {
             const int s = j % Ly::kStages;
             bool ok = true;
@@ -769,6 +787,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
             // failure-path check: a wait that can only run out of time
             bool ok = !p.test_stall || spin_or_abort(&bars[cbNever], 0, abort_flag, p.status);
             ok = ok && nchunks > 0 && issue_u0(0);
+#pragma unroll 1
             for (int j = 0; j < nchunks && ok; ++j) {
                 const int s = j % Ly::kStages, d = j & 1;
                 const uint32_t st = sbase + s * Ly::kStage;
@@ -852,6 +871,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
                 set_status(p.status, KDA_ERR_SLOT);
             }
         };
+#pragma unroll 1
         for (int j = 0; j <= nchunks && ok; ++j) {
             if (j > 0) {
                 // S <- Diag(Gam_L) (S + dS) for chunk j-1

@@ -38,10 +38,11 @@ __device__ __forceinline__ void note_timeout(int32_t *status, const uint64_t *ba
 // Bounded wait on an mbarrier phase.  Waiting threads stay suspended in
 // try_wait (no issue slots taken from working warps) and wake when the phase
 // completes; a wait that outlasts 2 s gives up, records KDA_ERR_TIMEOUT and
-// raises the CTA's abort flag so every role winds down.
-__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity,
-                                              volatile int *abort_flag, int32_t *status) {
-    if (mbar_try_wait(bar, parity)) return true;
+// raises the CTA's abort flag so every role winds down.  Only the first
+// try_wait is inlined: the loop lives in one out-of-line copy, which keeps the
+// many call sites of a warp-specialised kernel small in the instruction cache.
+static __device__ __noinline__ bool wait_or_abort_slow(uint64_t *bar, uint32_t parity,
+                                                volatile int *abort_flag, int32_t *status) {
     const uint64_t start = globaltimer_ns();
     for (;;) {
         if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
@@ -53,12 +54,18 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity,
     note_timeout(status, bar);
     return false;
 }
+__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity,
+                                              volatile int *abort_flag, int32_t *status) {
+    if (mbar_try_wait(bar, parity)) return true;
+    return wait_or_abort_slow(bar, parity, abort_flag, status);
+}
 
 // Bounded wait that polls instead of suspending: for the few threads on a
 // latency-critical chain, where the wake-up of a suspended waiter costs
-// hundreds of cycles.  Same 2 s limit and abort protocol as wait_or_abort.
-__device__ __forceinline__ bool spin_or_abort(uint64_t *bar, uint32_t parity,
-                                              volatile int *abort_flag, int32_t *status) {
+// hundreds of cycles.  Same 2 s limit and abort protocol as wait_or_abort;
+// the first 64 polls are inlined, the rest run out of line.
+static __device__ __noinline__ bool spin_or_abort_slow(uint64_t *bar, uint32_t parity,
+                                                volatile int *abort_flag, int32_t *status) {
     uint64_t start = 0;
     for (uint32_t n = 1;; ++n) {
         if (mbar_test_wait(bar, parity)) return true;
@@ -74,13 +81,20 @@ __device__ __forceinline__ bool spin_or_abort(uint64_t *bar, uint32_t parity,
     note_timeout(status, bar);
     return false;
 }
+__device__ __forceinline__ bool spin_or_abort(uint64_t *bar, uint32_t parity,
+                                              volatile int *abort_flag, int32_t *status) {
+#pragma unroll 1
+    for (int n = 0; n < 64; ++n)
+        if (mbar_test_wait(bar, parity)) return true;
+    return spin_or_abort_slow(bar, parity, abort_flag, status);
+}
 
 // Maps item index m (= global chunk g * H + head) to its chunk.
 struct Item {
     int h, c0, L;
     int m;   // packet index m; negative: this CTA has no further item
 };
-__device__ __forceinline__ Item item_of(long long m, int H, const int32_t *chunk_off,
+static __device__ __noinline__ Item item_of(long long m, int H, const int32_t *chunk_off,
                                         const int32_t *cu, int N) {
     const int g = (int)(m / H);
     Item it;
@@ -157,7 +171,9 @@ __device__ __forceinline__ uint64_t kmaj_step(int ks, uint32_t atom) {
 // (rows 0-63) and q (rows 64-127) and the KI stage raw log_alpha, as the TMA
 // left them.  On exit (after a proxy fence) they hold Kg, Qg and Ki; rows at
 // or past L are zero.  sGL_s receives Gam_L (128 channels), sB_s beta (64
-// rows, zero past L).  sGP / sSUF are [16][128] fp32 scratch.
+// rows, zero past L).  sGP / sSUF are [16][128] fp32 scratch; with
+// kScratchInKI they are the two 8 KB halves of the KI stage itself, free once
+// every raw log_alpha has been read (one more barrier) and overwritten by Ki.
 //
 // alpha = 2^(log_alpha log2 e) once per element; Gam_r is the running product
 // of alpha inside the chunk and 1/Gam_r = (1/Gam_L) prod_{j>r} alpha_j, so no
@@ -167,6 +183,7 @@ __device__ __forceinline__ uint64_t kmaj_step(int ks, uint32_t atom) {
 // Gam_L >= exp(-80); a chunk that breaks either records KDA_ERR_DECAY in
 // `status` (its chain's results are then unspecified; nothing else changes).
 // ---------------------------------------------------------------------------
+template <bool kScratchInKI = false>
 __device__ __forceinline__ void prep_chunk(int t, uint32_t kq_stage, uint32_t ki_stage,
                                            float *sGP, float *sSUF, float *sGL_s, float *sB_s,
                                            const __nv_bfloat16 *beta, int c0, int L, int H, int h,
@@ -210,6 +227,7 @@ __device__ __forceinline__ void prep_chunk(int t, uint32_t kq_stage, uint32_t ki
             pre[i][e] = px;          // prod_{j <= i} alpha_j
         }
     }
+    if (kScratchInKI) named_bar(bar_id, kPrepThreads);   // every log_alpha read before sGP lands on it
     {
         float *gpp = sGP + rg * 128 + cg * 8;
         *reinterpret_cast<float4 *>(gpp) = make_float4(pre[3][0], pre[3][1], pre[3][2], pre[3][3]);
@@ -252,7 +270,8 @@ __device__ __forceinline__ void prep_chunk(int t, uint32_t kq_stage, uint32_t ki
         ci[0] = q0.x; ci[1] = q0.y; ci[2] = q0.z; ci[3] = q0.w;
         ci[4] = q1.x; ci[5] = q1.y; ci[6] = q1.z; ci[7] = q1.w;
     }
-    // the next chunk's pass 0 overwrites sGP: everyone must have read it
+    // the next chunk's pass 0 (or, with kScratchInKI, this chunk's Ki)
+    // overwrites sGP and sSUF: everyone must have read them
     named_bar(bar_id, kPrepThreads);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -260,8 +279,8 @@ __device__ __forceinline__ void prep_chunk(int t, uint32_t kq_stage, uint32_t ki
         uint32_t gb[4], gib[4];
 #pragma unroll
         for (int e2 = 0; e2 < 4; ++e2) {
-            gb[e2] = pack_bf16_alu(ef[2 * e2] * pre[i][2 * e2], ef[2 * e2 + 1] * pre[i][2 * e2 + 1]);
-            gib[e2] = pack_bf16_alu(ci[2 * e2] * suf[i][2 * e2], ci[2 * e2 + 1] * suf[i][2 * e2 + 1]);
+            gb[e2] = pack2(ef[2 * e2] * pre[i][2 * e2], ef[2 * e2 + 1] * pre[i][2 * e2 + 1]);
+            gib[e2] = pack2(ci[2 * e2] * suf[i][2 * e2], ci[2 * e2 + 1] * suf[i][2 * e2 + 1]);
         }
         if (r >= L) {  // rows past the end of the sequence are zero
 #pragma unroll
@@ -409,6 +428,29 @@ __device__ __forceinline__ void invert_unit_lower(int sw, int lane, const float 
     }
 }
 
+// L = strict_lower(diag(b) A) from rows 0..63 of the A/P accumulator (TMEM
+// column tm_ap) into sL, by the two warps owning TMEM lanes 0..63 (sw = 0, 1).
+__device__ __forceinline__ void build_l(int sw, int lane, uint32_t tmem, uint32_t tm_ap, float *sL,
+                                        const float *sB_s) {
+    const int r = 32 * sw + lane;
+    uint32_t v0[32], v1[32];
+    tmem_ld32(tmem_addr(tmem, 32 * sw, tm_ap), v0);
+    tmem_ld32(tmem_addr(tmem, 32 * sw, tm_ap + 32), v1);
+    tmem_wait_ld();
+    const float br = sB_s[r];
+    float *Lr = sL + r * kLDL;
+#pragma unroll
+    for (int c = 0; c < 64; c += 4) {
+        const uint32_t *src = c < 32 ? &v0[c] : &v1[c - 32];
+        float4 w;
+        w.x = (c + 0 < r) ? br * __uint_as_float(src[0]) : 0.f;
+        w.y = (c + 1 < r) ? br * __uint_as_float(src[1]) : 0.f;
+        w.z = (c + 2 < r) ? br * __uint_as_float(src[2]) : 0.f;
+        w.w = (c + 3 < r) ? br * __uint_as_float(src[3]) : 0.f;
+        *reinterpret_cast<float4 *>(Lr + c) = w;
+    }
+}
+
 // kEarlyP: write P and release D_AP (one arrival on `ap_free`) right after
 // reading L.  Otherwise P stays in TMEM: the caller writes it with write_p()
 // and arrives on `ap_free` itself, later.
@@ -419,24 +461,7 @@ __device__ __forceinline__ void solve_chunk(int sw, int lane, uint32_t tmem, uin
                                             uint32_t bar_id) {
     const int t = sw * 32 + lane;
     if (sw < 2) {
-        // L = strict_lower(diag(b) A)
-        const int r = 32 * sw + lane;
-        uint32_t v0[32], v1[32];
-        tmem_ld32(tmem_addr(tmem, 32 * sw, tm_ap), v0);
-        tmem_ld32(tmem_addr(tmem, 32 * sw, tm_ap + 32), v1);
-        tmem_wait_ld();
-        const float br = sB_s[r];
-        float *Lr = sL + r * kLDL;
-#pragma unroll
-        for (int c = 0; c < 64; c += 4) {
-            const uint32_t *src = c < 32 ? &v0[c] : &v1[c - 32];
-            float4 w;
-            w.x = (c + 0 < r) ? br * __uint_as_float(src[0]) : 0.f;
-            w.y = (c + 1 < r) ? br * __uint_as_float(src[1]) : 0.f;
-            w.z = (c + 2 < r) ? br * __uint_as_float(src[2]) : 0.f;
-            w.w = (c + 3 < r) ? br * __uint_as_float(src[3]) : 0.f;
-            *reinterpret_cast<float4 *>(Lr + c) = w;
-        }
+        build_l(sw, lane, tmem, tm_ap, sL, sB_s);
     } else if (kEarlyP) {
         write_p(sw, lane, tmem, tm_ap, p_tile);
     }

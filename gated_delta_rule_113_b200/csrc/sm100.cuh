@@ -129,6 +129,18 @@ __device__ __forceinline__ void tc_fence_after() {
 __device__ __forceinline__ void named_bar(uint32_t id, uint32_t threads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
+// named barrier that also ORs a predicate over the participating threads, so
+// warps that leave a loop on a failed wait all leave it together
+__device__ __forceinline__ bool named_bar_or(uint32_t id, uint32_t threads, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, %2, %3, p;\n"
+        " selp.u32 %0, 1, 0, q;\n}"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id), "r"(threads)
+        : "memory");
+    return r != 0;
+}
 
 // ---------------------------------------------------------------- TMA
 // 3-D tiled load, global -> this CTA's shared memory, completion counted

@@ -121,7 +121,8 @@ rchain_kernel(const __grid_constant__ CUtensorMap tm_do, RcParams p) {
     if (tid == 0) {
         for (int i = 0; i < rbNum; ++i)
             mbar_init(&bars[i], (i == rbXbFull || i == rbDuFull) ? 4u : 1u);
-        *abort_flag = 0;
+        abort_flag[0] = 0;
+        abort_flag[1] = 0;
         fence_mbar_init();
     }
     if (warp == 4 && lane == 0) prefetch_tmap(&tm_do);
@@ -308,6 +309,7 @@ rchain_kernel(const __grid_constant__ CUtensorMap tm_do, RcParams p) {
     }
     tc_fence_before();
     __syncthreads();
+    if (tid == 0) report_abort(abort_flag, p.status);
     if (warp == 5) {
         tc_fence_after();
         tmem_dealloc(tmem, Ly::kTmCols);
@@ -327,25 +329,6 @@ __device__ __forceinline__ uint32_t toff(const Tile &t, int r, int c) {
     return t.base + (uint32_t)(r * t.rl * 2) +
            ((((uint32_t)c >> 3) ^ ((uint32_t)r & 7u)) << 4) + (uint32_t)(c & 7) * 2u;
 }
-__device__ __forceinline__ void ldsm_x4(uint32_t a, uint32_t (&r)[4]) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"(a));
-}
-__device__ __forceinline__ void ldsm_x4_t(uint32_t a, uint32_t (&r)[4]) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"(a));
-}
-__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
-                                         uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-        "{%8,%9}, {%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
 // acc (16 rows from m0, NT x 8 columns from n0) += A B over k in [kb, ke).
 // A_T: A is stored transposed (rows = k); B_KN: B is stored k-major (rows =
 // k), else n-major (rows = n).

@@ -83,28 +83,44 @@ constexpr uint32_t kPkTP = 49152;
 constexpr uint32_t kPkGL = 65536;
 static_assert(kPkGL + 512 <= kPacketBytes, "packet layout");
 
-// PT = P Tb from its M = 64 accumulator (row r in TMEM lane 32 (r / 16) +
-// r % 16) to bf16 rows 64..127 of the Tb|PT tile, by the eight prep warps:
-// warp w reads lane quarter w % 4, columns 32 (w / 4) .. + 31.
-__device__ __forceinline__ void convert_pt8(int w, int lane, uint32_t tmem, uint32_t tm_pt,
-                                            uint32_t tp) {
-    const int qt = w & 3, hh = w >> 2;
-    uint32_t v[32];
-    tmem_ld32(tmem_addr(tmem, 32 * qt, tm_pt + 32 * hh), v);
-    tmem_wait_ld();
-    if (lane < 16) {
-        const int r = 64 + 16 * qt + lane;
+// PT = P Tb into bf16 rows 64..127 of the Tb|PT tile, on the four solve
+// warps with the warp-level bf16 MMA (fp32 accumulation, as a tcgen05
+// product would): warp sw owns columns 16 sw .. 16 sw + 15 of every row; P is
+// lower-inclusive, so row tile mt sums key tiles 0..mt only.  Doing this here
+// saves a tensor-memory round trip between the solve and the W product.
+__device__ __forceinline__ void pt_product(int sw, int lane, uint32_t p_tile, uint32_t tp) {
+    const int l7 = lane & 7, mi = lane >> 3, g = lane >> 2, tq = lane & 3;
+    // B fragments of this warp's two column tiles for the four key tiles,
+    // loaded once; ten independent accumulator chains of at most 4 products
+    uint32_t bf[4][4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-            sts128(tp + sw128_off(r, 4 * hh + j),
-                   pack2(__uint_as_float(v[8 * j]), __uint_as_float(v[8 * j + 1])),
-                   pack2(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3])),
-                   pack2(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5])),
-                   pack2(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7])));
+    for (int ks = 0; ks < 4; ++ks)
+        ldsm_x4_t(tp + sw128_off(16 * ks + l7 + (mi & 1) * 8, 2 * sw + (mi >> 1)), bf[ks]);
+    float acc[4][2][4];
+#pragma unroll
+    for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {
+#pragma unroll
+        for (int mt = ks; mt < 4; ++mt) {
+            uint32_t af[4];
+            ldsm_x4(p_tile + sw128_off(16 * mt + l7 + (mi & 1) * 8, 2 * ks + (mi >> 1)), af);
+            mma16816(acc[mt][0], af, bf[ks][0], bf[ks][1]);
+            mma16816(acc[mt][1], af, bf[ks][2], bf[ks][3]);
+        }
     }
-    fence_proxy_async();
-    tc_fence_before();
-    __syncwarp();
+#pragma unroll
+    for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            const int r = 64 + 16 * mt + g, chunk = 2 * sw + nt;
+            sts32(tp + sw128_off(r, chunk) + 4 * tq, pack2(acc[mt][nt][0], acc[mt][nt][1]));
+            sts32(tp + sw128_off(r + 8, chunk) + 4 * tq, pack2(acc[mt][nt][2], acc[mt][nt][3]));
+        }
 }
 
 // [W; PW] (TMEM lanes 0..127) -> -W over the Kg rows and Qe = Qg - PW over
@@ -153,16 +169,14 @@ enum KsBars {
     kbKqFull = 4,    // [4] count 8: prep -> A/P issuer, Ki stores
     kbApFull = 8,    // [2] A/P product -> solve (two TMEM accumulators)
     kbApFree = 10,   // [2] solve has read D_AP[s] -> A/P issuer
-    kbTbFull = 12,   // solve -> PT issuer (Tb and P final)
-    kbPtAcc = 13,    // PT = P Tb product -> prep warps (convert), solve (P tile free)
-    kbPtReady = 14,  // count 8: PT written as bf16 (prep warps) -> W issuer
-    kbTpFree = 15,   // the Tb|PT tile has been read -> Tb write of the next chunk
-    kbWaccFull = 16, // [W; PW] product -> prep warps
-    kbWReady = 17,   // count 8: -W and Qe written -> stores (and D_W free)
-    kbStored = 18,   // [4] the packet's -W|Qe copies have read the key-query stage -> TMA
-    kbKiFree = 22,   // [2] count 4: A/P product done, Ki and Gam_L copies read -> TMA
-    kbDrain = 24,    // [2] A/P issuer, PT/W issuer
-    kbNum = 26
+    kbTbFull = 12,   // solve -> W issuer (Tb and PT written)
+    kbTpFree = 13,   // the Tb|PT tile has been read -> Tb write of the next chunk
+    kbWaccFull = 14, // [W; PW] product -> prep warps
+    kbWReady = 15,   // count 8: -W and Qe written -> stores (and D_W free)
+    kbStored = 16,   // [4] the packet's -W|Qe copies have read the key-query stage -> TMA
+    kbKiFree = 20,   // [2] count 4: A/P product done, Ki and Gam_L copies read -> TMA
+    kbDrain = 22,    // [2] A/P issuer, W issuer
+    kbNum = 24
 };
 
 struct KsLayout {
@@ -182,8 +196,7 @@ struct KsLayout {
     static_assert(kAlloc <= 232448, "shared memory budget exceeded");
     static constexpr uint32_t kTmAP = 0;     // + (i & 1) * 64 (two A/P accumulators)
     static constexpr uint32_t kTmW = 128;    // [W; PW], 128 columns
-    static constexpr uint32_t kTmPT = 256;   // PT (M = 64: 16 lanes per quarter), 64 columns
-    static constexpr uint32_t kTmCols = 512;
+    static constexpr uint32_t kTmCols = 256;
 };
 
 struct KsParams {
@@ -235,11 +248,11 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             uint32_t cnt = 1;
             if (i >= kbKqFull && i < kbKqFull + kKqStages) cnt = kPrepThreads / 32;
             if (i == kbWReady) cnt = kPrepThreads / 32;
-            if (i == kbPtReady) cnt = kPrepThreads / 32;
             if (i >= kbKiFree && i < kbKiFree + kKiStages) cnt = 4;
             mbar_init(&bars[i], cnt);
         }
-        *abort_flag = 0;
+        abort_flag[0] = 0;
+        abort_flag[1] = 0;
         fence_mbar_init();
     }
     if (warp == kKsTma && lane == 0) {
@@ -350,29 +363,16 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             unsigned char *kq = sm + Ly::kKQ + s * 32768;
             unsigned char *tp = sm + Ly::kTP;
             bool ok = true;
-            // The products after the solve are issued here rather than by the
-            // A/P issuer, so the next chunk's A/P product never queues behind
-            // this chunk's solve.  D_PT and D_W are free: this lane already
-            // waited for the previous chunk's conversions out of them.
+            // The W product is issued here rather than by the A/P issuer, so
+            // the next chunk's A/P product never queues behind this chunk's
+            // solve.  D_W is free: this lane already waited for the previous
+            // chunk's conversion out of it.
             if (lane == 0) ok = wait_or_abort(&bars[kbTbFull], i & 1, abort_flag, p.status);
             if (!__shfl_sync(0xffffffffu, ok, 0)) break;
             const int m = items[s].m;
             if (m < 0) break;
             if (!KDA_IN_RANGE((long long)m < p.slots, p.status)) break;
             unsigned char *dst = p.packets + (size_t)m * kPacketBytes;
-            if (lane == 0) {   // PT = P Tb  (M = 64, B = Tb read MN-major)
-                tc_fence_after();
-                constexpr uint32_t kIdPT = idesc_bf16(64, 64, 0, 1);
-                const uint64_t d_p = smem_desc(sbase + Ly::kP, 16, 1024, kSw128);
-                const uint64_t d_tb = smem_desc(sbase + Ly::kTP, 8192, 1024, kSw128);
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16(tmem + Ly::kTmPT, d_p + ((uint64_t)(ks * 32) >> 4),
-                             d_tb + ((uint64_t)(ks * 2048) >> 4), kIdPT, ks > 0);
-                mma_commit(&bars[kbPtAcc]);
-                ok = wait_or_abort(&bars[kbPtReady], i & 1, abort_flag, p.status);
-            }
-            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
             if (lane == 0) {   // [W; PW] = [Tb; PT] Kg
                 tc_fence_after();
                 constexpr uint32_t kIdW = idesc_bf16(128, 128, 0, 1);
@@ -411,21 +411,14 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     } else if (warp >= kKsPrep0 && warp < kKsPrep0 + kPrepThreads / 32) {
         // ----------------------------------------------------------- prep
         const int t = tid - kKsPrep0 * 32;
-        // After preparing chunk i these warps turn chunk i-1's products into
-        // bf16 operands: PT into rows 64-127 of the Tb|PT tile, then [W; PW]
-        // into -W and Qe.
+        // After preparing chunk i these warps turn chunk i-1's [W; PW] product
+        // into the bf16 -W and Qe operands.
         // Thread 0 waits on each mbarrier and named_bar_or() shares the
         // outcome: the eight warps leave together on a failed wait, so none is
         // left at one of prep_chunk's named barriers.
         auto convert = [&](int m) -> bool {
             const int sm4 = m % kKqStages;
-            // PT = P Tb first: the [W; PW] product waits for it
-            bool w = t != 0 || wait_or_abort(&bars[kbPtAcc], m & 1, abort_flag, p.status);
-            if (named_bar_or(1, kPrepThreads, !w)) return false;
-            tc_fence_after();
-            convert_pt8(warp, lane, tmem, Ly::kTmPT, sbase + Ly::kTP);
-            if (lane == 0) mbar_arrive(&bars[kbPtReady]);
-            w = t != 0 || wait_or_abort(&bars[kbWaccFull], m & 1, abort_flag, p.status);
+            const bool w = t != 0 || wait_or_abort(&bars[kbWaccFull], m & 1, abort_flag, p.status);
             if (named_bar_or(1, kPrepThreads, !w)) return false;
             tc_fence_after();
             if (t == 0) KDA_TRACE1(m, 7);
@@ -486,16 +479,9 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             tc_fence_after();
             if (t == 0) KDA_TRACE1(i, 4);
             // D_AP -> L (warps 0, 1: rows 0-63) and -> the bf16 P tile (warps
-            // 2, 3: rows 64-127), side by side; the P tile is free once the
-            // previous chunk's PT product is done
-            if (sw < 2) {
-                build_l(sw, lane, tmem, Ly::kTmAP + a * 64, sL, sB + s * 64);
-            } else {
-                if (lane == 0 && i >= 1)
-                    ok = wait_or_abort(&bars[kbPtAcc], (i - 1) & 1, abort_flag, p.status);
-                if (__shfl_sync(0xffffffffu, ok, 0)) write_p(sw, lane, tmem, Ly::kTmAP + a * 64, sbase + Ly::kP);
-                ok = __shfl_sync(0xffffffffu, ok, 0);
-            }
+            // 2, 3: rows 64-127), side by side
+            if (sw < 2) build_l(sw, lane, tmem, Ly::kTmAP + a * 64, sL, sB + s * 64);
+            else write_p(sw, lane, tmem, Ly::kTmAP + a * 64, sbase + Ly::kP);
             tc_fence_before();
             if (named_bar_or(2, kSolveThreads, !ok)) break;
             if (t == 0) mbar_arrive(&bars[kbApFree + a]);
@@ -504,6 +490,9 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             if (t == 0 && i >= 1) ok = wait_or_abort(&bars[kbTpFree], (i - 1) & 1, abort_flag, p.status);
             if (named_bar_or(2, kSolveThreads, !ok)) break;
             write_tb(sw, lane, sbase + Ly::kTP, sT, sB + s * 64, 2);
+            pt_product(sw, lane, sbase + Ly::kP, sbase + Ly::kTP);
+            fence_proxy_async();
+            named_bar(2, kSolveThreads);
             if (t == 0) mbar_arrive(&bars[kbTbFull]);
             if (t == 0) KDA_TRACE1(i, 5);
         }
@@ -572,6 +561,7 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     KDA_SPAN(g_kda_span1, 1);
     tc_fence_before();
     __syncthreads();
+    if (tid == 0) report_abort(abort_flag, p.status);
     if (warp == kKsMma) {
         tc_fence_after();
         tmem_dealloc(tmem, Ly::kTmCols);
@@ -695,7 +685,8 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
             if (i == cbUbFull || i == cbD1Free || i == cbD1Free + 1) cnt = Sh::kChain / 2;
             mbar_init(&bars[i], cnt);
         }
-        *abort_flag = 0;
+        abort_flag[0] = 0;
+        abort_flag[1] = 0;
         fence_mbar_init();
     }
     if (warp == kChLoad && lane == 0) prefetch_tmap(&tm_v);
@@ -990,6 +981,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
     KDA_SPAN(g_kda_span2, 1);
     tc_fence_before();
     __syncthreads();
+    if (tid == 0) report_abort(abort_flag, p.status);
     if (warp == kChMma) {
         tc_fence_after();
         tmem_dealloc(tmem, Ly::kTmCols);

@@ -180,7 +180,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             if (i == bD1Free || i == bD1Free + 1) cnt = 2;
             mbar_init(&bars[i], cnt);
         }
-        *abort_flag = 0;
+        abort_flag[0] = 0;
+        abort_flag[1] = 0;
         fence_mbar_init();
     }
     if (warp == kTma && lane == 0) {
@@ -511,6 +512,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     // ------------------------------------------------------------ teardown
     tc_fence_before();
     __syncthreads();
+    if (tid == 0) report_abort(abort_flag, p.status);
     if (warp == kMmaK) {
         tc_fence_after();
         tmem_dealloc(tmem, Ly::kTmCols);

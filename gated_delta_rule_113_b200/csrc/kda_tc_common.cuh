@@ -25,48 +25,46 @@ constexpr int kPrepThreads = 256;  // threads running prep_chunk
 constexpr int kSolveThreads = 128; // threads running solve_chunk (4 warps, lane quarters 0..3)
 constexpr float kLog2e = 1.4426950408889634f;
 
-// Where a bounded wait gave up, for diagnosis: the first timeout of a call
-// stores (barrier's shared-memory offset | thread index << 16) in the word
-// after the status word's 32-byte line (status[8]) and the block index in
-// status[9].  Written only on that failure path.
-__device__ __forceinline__ void note_timeout(int32_t *status, const uint64_t *bar) {
-    if (!status) return;
-    const int32_t tag = (int32_t)((smem_u32(bar) & 0xFFFFu) | ((uint32_t)threadIdx.x << 16));
-    if (atomicCAS(status + 8, 0, tag) == 0) status[9] = (int32_t)blockIdx.x;
+// Bounded waits.  A wait that outlasts 2 s gives up: it raises the CTA's
+// abort flag (abort_flag[0], so every role winds down) and notes where it
+// gave up in abort_flag[1] (the barrier's shared-memory offset | thread index
+// << 16).  Thread 0 reports both after the kernel's last barrier
+// (report_abort): KDA_ERR_TIMEOUT in the status word, the note in status[8]
+// and the block index in status[9].  Keeping the failure path out of the
+// waits keeps the many call sites of a warp-specialised kernel small in the
+// instruction cache.
+__device__ __forceinline__ void raise_abort(volatile int *abort_flag, const uint64_t *bar) {
+    abort_flag[1] = (int)((smem_u32(bar) & 0xFFFFu) | ((uint32_t)threadIdx.x << 16));
+    abort_flag[0] = 1;
+}
+__device__ __forceinline__ void report_abort(const volatile int *abort_flag, int32_t *status) {
+    if (!abort_flag[0]) return;
+    set_status(status, KDA_ERR_TIMEOUT);
+    if (status && atomicCAS(status + 8, 0, abort_flag[1]) == 0) status[9] = (int32_t)blockIdx.x;
 }
 
-// Bounded wait on an mbarrier phase.  Waiting threads stay suspended in
-// try_wait (no issue slots taken from working warps) and wake when the phase
-// completes; a wait that outlasts 2 s gives up, records KDA_ERR_TIMEOUT and
-// raises the CTA's abort flag so every role winds down.  Only the first
-// try_wait is inlined: the loop lives in one out-of-line copy, which keeps the
-// many call sites of a warp-specialised kernel small in the instruction cache.
-static __device__ __noinline__ bool wait_or_abort_slow(uint64_t *bar, uint32_t parity,
-                                                volatile int *abort_flag, int32_t *status) {
+// Waiting threads stay suspended in try_wait (no issue slots taken from
+// working warps) and wake when the phase completes.
+__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity,
+                                              volatile int *abort_flag, int32_t *) {
+    if (mbar_try_wait(bar, parity)) return true;
     const uint64_t start = globaltimer_ns();
+#pragma unroll 1
     for (;;) {
         if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
         if (*abort_flag) return false;
         if (globaltimer_ns() - start > 2000000000ull) break;
     }
-    *abort_flag = 1;
-    set_status(status, KDA_ERR_TIMEOUT);
-    note_timeout(status, bar);
+    raise_abort(abort_flag, bar);
     return false;
 }
-__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity,
-                                              volatile int *abort_flag, int32_t *status) {
-    if (mbar_try_wait(bar, parity)) return true;
-    return wait_or_abort_slow(bar, parity, abort_flag, status);
-}
 
-// Bounded wait that polls instead of suspending: for the few threads on a
-// latency-critical chain, where the wake-up of a suspended waiter costs
-// hundreds of cycles.  Same 2 s limit and abort protocol as wait_or_abort;
-// the first 64 polls are inlined, the rest run out of line.
-static __device__ __noinline__ bool spin_or_abort_slow(uint64_t *bar, uint32_t parity,
-                                                volatile int *abort_flag, int32_t *status) {
+// Polls instead of suspending: for the few threads on a latency-critical
+// chain, where the wake-up of a suspended waiter costs hundreds of cycles.
+__device__ __forceinline__ bool spin_or_abort(uint64_t *bar, uint32_t parity,
+                                              volatile int *abort_flag, int32_t *) {
     uint64_t start = 0;
+#pragma unroll 1
     for (uint32_t n = 1;; ++n) {
         if (mbar_test_wait(bar, parity)) return true;
         if ((n & 1023u) == 0) {
@@ -76,17 +74,8 @@ static __device__ __noinline__ bool spin_or_abort_slow(uint64_t *bar, uint32_t p
             else if (now - start > 2000000000ull) break;
         }
     }
-    *abort_flag = 1;
-    set_status(status, KDA_ERR_TIMEOUT);
-    note_timeout(status, bar);
+    raise_abort(abort_flag, bar);
     return false;
-}
-__device__ __forceinline__ bool spin_or_abort(uint64_t *bar, uint32_t parity,
-                                              volatile int *abort_flag, int32_t *status) {
-#pragma unroll 1
-    for (int n = 0; n < 64; ++n)
-        if (mbar_test_wait(bar, parity)) return true;
-    return spin_or_abort_slow(bar, parity, abort_flag, status);
 }
 
 // Maps item index m (= global chunk g * H + head) to its chunk.
@@ -126,6 +115,9 @@ __device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, ui
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
                  "r"(d)
                  : "memory");
+}
+__device__ __forceinline__ void sts32(uint32_t addr, uint32_t a) {
+    asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(a) : "memory");
 }
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
     uint4 v;

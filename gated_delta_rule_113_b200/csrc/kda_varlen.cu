@@ -82,7 +82,7 @@ __global__ void __launch_bounds__(1024) varlen_index_kernel(const int32_t *__res
     __syncthreads();
     if (tid == 0) {
         *status = s_bad ? KDA_ERR_SEQLENS : KDA_OK;
-        status[8] = 0;   // where a bounded wait gave up, if one does (see note_timeout)
+        status[8] = 0;   // where a bounded wait gave up, if one does (see report_abort)
         status[9] = 0;
     }
     if (N > kSortMax) {

@@ -91,6 +91,7 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 // which may itself block for a hardware-defined interval, is seconds of
 // wall time: far beyond any legitimate wait in these kernels.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+#pragma unroll 1
     for (uint32_t i = 0; i < (1u << 22); ++i) {
         if (mbar_try_wait(bar, parity)) return true;
         if (i >= (1u << 14)) __nanosleep(128);
@@ -316,6 +317,27 @@ __device__ __forceinline__ uint32_t to_tf32(float x) {
 // tf32 operand from an fp32 value without a conversion instruction: the MMA
 // reads only the sign, exponent and top 10 mantissa bits (round toward zero).
 __device__ __forceinline__ uint32_t tf32_bits(float x) { return __float_as_uint(x); }
+
+// ldmatrix (x4, plain and transposed) and the bf16 m16n8k16 warp MMA
+__device__ __forceinline__ void ldsm_x4(uint32_t a, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(a));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t a, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(a));
+}
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
 
 __device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], const uint32_t (&a)[4],
                                                 const uint32_t (&b)[2]) {

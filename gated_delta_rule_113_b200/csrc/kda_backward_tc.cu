@@ -391,7 +391,7 @@ struct AsmParams {
 
 struct AsmLayout {
     static constexpr uint32_t kKG = 0, kQG = 16384, kKI = 32768;
-    static constexpr uint32_t kSolve = 49152;            // sL | sT | sXw, later V | dO
+    static constexpr uint32_t kSolve = 49152;            // sL | sT, later V | dO
     static constexpr uint32_t kV = 49152, kDO = 65536;
     static constexpr uint32_t kS = 90112;                // S (bf16 128 x 128); Gam, dG fp32 temps
     static constexpr uint32_t kX = 122880;               // dX (bf16 128 x 128); la temp; dT | M1 | dAf
@@ -442,7 +442,6 @@ __global__ void __launch_bounds__(kAsmThreads, 1) assemble_kernel(AsmParams p) {
     __nv_bfloat16 *sLa = reinterpret_cast<__nv_bfloat16 *>(sm + Ly::kX);   // bf16 [64][128] temp
     float *sL = reinterpret_cast<float *>(sm + Ly::kSolve);
     float *sT = sL + 64 * kLDL;
-    float *sXw = sT + 64 * kLDL;
 
     // tile ownership: 64 x 128 outputs: rows m0 .. m0 + 15, columns n0 .. n0 + 63;
     // 64 x 64 outputs: the same rows, columns n6 .. n6 + 31
@@ -540,7 +539,7 @@ __global__ void __launch_bounds__(kAsmThreads, 1) assemble_kernel(AsmParams p) {
     // warps 0-3: T = (I + L)^{-1}; warps 4-7: S_j and dX_j as bf16 tiles and
     // rowsum(S * dX), one row per warp and step
     if (w < 4) {
-        invert_unit_lower(w, lane, sL, sT, sXw, 1);
+        invert_unit_lower(w, lane, sL, sT, 1);
     } else {
         const float *Sg = p.ckpt + (size_t)m * kDK * kDV;
         const float *Xg = p.dxs + (size_t)m * kDK * kDV;

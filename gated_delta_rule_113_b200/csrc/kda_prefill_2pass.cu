@@ -186,8 +186,7 @@ struct KsLayout {
     static constexpr uint32_t kP = kTP + 16384;                       // 8 KB: P
     static constexpr uint32_t kL = kP + 8192;
     static constexpr uint32_t kT = kL + 64 * kLDL * 4;
-    static constexpr uint32_t kXw = kT + 64 * kLDL * 4;     // fp32 4 x [16][17]
-    static constexpr uint32_t kGL = kXw + 4 * 16 * 17 * 4;  // [2][128], per gate stage
+    static constexpr uint32_t kGL = kT + 64 * kLDL * 4;     // [2][128], per gate stage
     static constexpr uint32_t kB = kGL + kKiStages * 128 * 4;       // [4][64], per key-query stage
     static constexpr uint32_t kBar = kB + kKqStages * 64 * 4;
     static constexpr uint32_t kMisc = kBar + kbNum * 8;
@@ -222,7 +221,6 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + Ly::kMisc + 4);
     float *sL = reinterpret_cast<float *>(sm + Ly::kL);
     float *sT = reinterpret_cast<float *>(sm + Ly::kT);
-    float *sXw = reinterpret_cast<float *>(sm + Ly::kXw);
     float *sGL = reinterpret_cast<float *>(sm + Ly::kGL);
     float *sB = reinterpret_cast<float *>(sm + Ly::kB);
 
@@ -302,50 +300,54 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         auto warm = [&](const Item &it) {   // L2 prefetch of an item's tiles
             if (it.m >= 0 && lane < 6) tma_prefetch_3d(tm, a * 64, it.h, it.c0);
         };
-        Item nx0 = claim(true);
-        Item nx1 = claim(false);
-        warm(nx1);
-        Item nx2 = claim(false);
-        warm(nx2);
+        // nx0..nx2: the next three items; iterations -3..-1 only fill them,
+        // so claim() and warm() have one call site each
+        Item nx0, nx1, nx2;
+        nx0.m = nx1.m = nx2.m = -1;
+        nx0.h = nx1.h = nx2.h = nx0.c0 = nx1.c0 = nx2.c0 = nx0.L = nx1.L = nx2.L = 0;
         int n_loaded = 0;
         bool ended = false;
 #pragma unroll 1
-        for (int i = 0;; ++i) {
-            const int s = i % kKqStages, si = i % kKiStages;
-            const Item it = nx0;
-            nx0 = nx1;
-            nx1 = nx2;
-            // the packet of item i-4 must have left key-query stage s
-            bool ok = true;
-            if (lane == 0 && i >= kKqStages)
-                ok = wait_or_abort(&bars[kbStored + s], ((i / kKqStages) - 1) & 1, abort_flag, p.status);
-            // and item i-2 must be done with gate stage si
-            if (lane == 0 && ok && it.m >= 0 && i >= kKiStages)
-                ok = wait_or_abort(&bars[kbKiFree + si], ((i / kKiStages) - 1) & 1, abort_flag, p.status);
-            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-            uint64_t *full = &bars[kbRawFull + s];
-            if (it.m < 0) {   // no more items: tell the prep, which tells the rest
+        for (int i = -3;; ++i) {
+            if (i >= 0) {
+                const int s = i % kKqStages, si = i % kKiStages;
+                const Item it = nx0;
+                // the packet of item i-4 must have left key-query stage s
+                bool ok = true;
+                if (lane == 0 && i >= kKqStages)
+                    ok = wait_or_abort(&bars[kbStored + s], ((i / kKqStages) - 1) & 1, abort_flag,
+                                       p.status);
+                // and item i-2 must be done with gate stage si
+                if (lane == 0 && ok && it.m >= 0 && i >= kKiStages)
+                    ok = wait_or_abort(&bars[kbKiFree + si], ((i / kKiStages) - 1) & 1, abort_flag,
+                                       p.status);
+                if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+                uint64_t *full = &bars[kbRawFull + s];
+                if (it.m < 0) {   // no more items: tell the prep, which tells the rest
+                    if (lane == 0) {
+                        items[s] = it;
+                        mbar_arrive(full);
+                    }
+                    ended = true;
+                    break;
+                }
                 if (lane == 0) {
                     items[s] = it;
-                    mbar_arrive(full);
+                    mbar_arrive_expect_tx(full, 6 * 8192);
                 }
-                ended = true;
-                break;
+                __syncwarp();
+                if (lane < 6) {
+                    const uint32_t dst = which < 2 ? Ly::kKQ + s * 32768 + a * 16384 + which * 8192
+                                                   : Ly::kKI + si * 16384 + a * 8192;
+                    tma_load_3d(sm + dst, tm, full, a * 64, it.h, it.c0);
+                }
+                if (lane == 0) KDA_TRACE1(i, 0);
+                n_loaded = i + 1;
             }
-            if (lane == 0) {
-                items[s] = it;
-                mbar_arrive_expect_tx(full, 6 * 8192);
-            }
-            __syncwarp();
-            if (lane < 6) {
-                const uint32_t dst = which < 2 ? Ly::kKQ + s * 32768 + a * 16384 + which * 8192
-                                               : Ly::kKI + si * 16384 + a * 8192;
-                tma_load_3d(sm + dst, tm, full, a * 64, it.h, it.c0);
-            }
-            if (lane == 0) KDA_TRACE1(i, 0);
-            n_loaded = i + 1;
-            nx2 = claim(false);
-            warm(nx2);
+            nx0 = nx1;
+            nx1 = nx2;
+            nx2 = claim(i == -3);
+            if (i > -3) warm(nx2);
         }
         // Armed loads must land before the CTA may exit.  The end marker went
         // to the stage of item n_loaded - 4, whose load the Stored wait above
@@ -411,7 +413,7 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     } else if (warp >= kKsPrep0 && warp < kKsPrep0 + kPrepThreads / 32) {
         // ----------------------------------------------------------- prep
         const int t = tid - kKsPrep0 * 32;
-        // After preparing chunk i these warps turn chunk i-1's [W; PW] product
+        // After preparing chunk i these warps turn chunk i-2's [W; PW] product
         // into the bf16 -W and Qe operands.
         // Thread 0 waits on each mbarrier and named_bar_or() shares the
         // outcome: the eight warps leave together on a failed wait, so none is
@@ -428,8 +430,11 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             return true;
         };
         // Iteration i prepares item i (while there is one) and then converts
-        // item i-1; the end marker stops the preps, one more pass converts
-        // the last item.  One call site each keeps the code small.
+        // item i-2: the conversion waits for that item's solve and W product,
+        // and lagging it two items keeps the preps (which the next solves
+        // wait for) off that path.  The end marker stops the preps; two more
+        // passes convert the last items.  One call site each keeps the code
+        // small.
         int n_items = 0;
         bool more = true;
 #pragma unroll 1
@@ -454,8 +459,8 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars[kbKqFull + s]);
             }
-            if (i >= 1 && i - 1 < n_items && !convert(i - 1)) break;
-            if (!more) break;
+            if (i >= 2 && i - 2 < n_items && !convert(i - 2)) break;
+            if (!more && i - 1 >= n_items) break;
         }
     } else if (warp >= kKsSolve0 && warp < kKsSolve0 + 4) {
         // ---------------------------------------------------------- solve
@@ -485,7 +490,7 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             tc_fence_before();
             if (named_bar_or(2, kSolveThreads, !ok)) break;
             if (t == 0) mbar_arrive(&bars[kbApFree + a]);
-            invert_unit_lower(sw, lane, sL, sT, sXw, 2);
+            invert_unit_lower(sw, lane, sL, sT, 2);
             // the previous chunk's Tb|PT tile must have been read
             if (t == 0 && i >= 1) ok = wait_or_abort(&bars[kbTpFree], (i - 1) & 1, abort_flag, p.status);
             if (named_bar_or(2, kSolveThreads, !ok)) break;

@@ -78,8 +78,7 @@ struct Layout {
     static constexpr uint32_t kUB = kSB + 128 * VS * 2;     // bf16 U operand
     static constexpr uint32_t kL = kUB + 64 * VS * 2;       // fp32 [64][kLDL]
     static constexpr uint32_t kT = kL + 64 * kLDL * 4;      // fp32 [64][kLDL]
-    static constexpr uint32_t kXw = kT + 64 * kLDL * 4;     // fp32 4 x [16][17]
-    static constexpr uint32_t kGP = kXw + 4 * 16 * 17 * 4;  // fp32 [16][128] group products / prefix
+    static constexpr uint32_t kGP = kT + 64 * kLDL * 4;     // fp32 [16][128] group products / prefix
     static constexpr uint32_t kSUF = kGP + 16 * 128 * 4;    // fp32 [16][128] suffix
     static constexpr uint32_t kGL = kSUF + 16 * 128 * 4;    // fp32 [2][128]
     static constexpr uint32_t kB = kGL + 2 * 128 * 4;       // fp32 [2][64]
@@ -149,7 +148,6 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + Ly::kMisc + 4);
     float *sL = reinterpret_cast<float *>(sm + Ly::kL);
     float *sT = reinterpret_cast<float *>(sm + Ly::kT);
-    float *sXw = reinterpret_cast<float *>(sm + Ly::kXw);
     float *sGP = reinterpret_cast<float *>(sm + Ly::kGP);
     float *sSUF = reinterpret_cast<float *>(sm + Ly::kSUF);
     float *sGL = reinterpret_cast<float *>(sm + Ly::kGL);
@@ -268,7 +266,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             if (!wait_or_abort(&bars[bApFull], n & 1, abort_flag, p.status)) break;
             tc_fence_after();
             if (t == 0) KDA_TRACE_EVENT(n, 4);
-            solve_chunk(sw, lane, tmem, Ly::kTmAP, sbase + Ly::kTP + s * 24576 + 16384, sL, sT, sXw,
+            solve_chunk(sw, lane, tmem, Ly::kTmAP, sbase + Ly::kTP + s * 24576 + 16384, sL, sT,
                         sB + s * 64, &bars[bApFree], kBarSolve);
             write_tb(sw, lane, sbase + Ly::kTP + s * 24576, sT, sB + s * 64, kBarSolve);
             if (t == 0) mbar_arrive(&bars[bTbFull + s]);

@@ -295,11 +295,9 @@ __device__ __forceinline__ void prep_chunk(int t, uint32_t kq_stage, uint32_t ki
 // synchronise on named barrier `bar_id`.  Reads D_AP from TMEM (column
 // tm_ap), writes L = strict_lower(diag(b) A) to sL and the masked bf16 P as a
 // 64-row K-major tile at `p_tile`, arrives once on `ap_free` when D_AP may be
-// overwritten, then builds T = (I + L)^{-1} in sT (16x16 diagonal blocks by
-// substitution, then a block forward substitution by 8-column strips with
-// mma.sync tf32).  Blocks of sT above the diagonal blocks must be zero on
-// entry (they are never written).  sXw is 4 x [16][17] fp32 warp-private
-// scratch.  write_tb() then turns T into the bf16 Tb tile.
+// overwritten, then builds T = (I + L)^{-1} in sT (invert_unit_lower).
+// Blocks of sT above the diagonal blocks must be zero on entry (they are
+// never written).  write_tb() then turns T into the bf16 Tb tile.
 // ---------------------------------------------------------------------------
 // P = lower_incl(Q K^T) rows (TMEM lanes 64..127 of the A/P accumulator at
 // column tm_ap) -> masked bf16 64-row K-major tile at `p_tile`.  Run by the
@@ -308,36 +306,68 @@ __device__ __forceinline__ void write_p(int sw, int lane, uint32_t tmem, uint32_
                                        uint32_t p_tile) {
     if (sw < 2) return;
     const int r = 32 * (sw & 1) + lane;
-    uint32_t v0[32], v1[32];
-    tmem_ld32(tmem_addr(tmem, 32 * sw, tm_ap), v0);
-    tmem_ld32(tmem_addr(tmem, 32 * sw, tm_ap + 32), v1);
-    tmem_wait_ld();
+#pragma unroll 1
+    for (int j2 = 0; j2 < 8; j2 += 2) {
+        uint32_t v[16];
+        tmem_ld16(tmem_addr(tmem, 32 * sw, tm_ap + 8 * j2), v);
+        tmem_wait_ld();
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        uint32_t o[4];
+        for (int jj = 0; jj < 2; ++jj) {
+            uint32_t o[4];
 #pragma unroll
-        for (int e2 = 0; e2 < 4; ++e2) {
-            const int c = 8 * j + 2 * e2;
-            const uint32_t *src = c < 32 ? &v0[c] : &v1[c - 32];
-            const float x0 = (c <= r) ? __uint_as_float(src[0]) : 0.f;
-            const float x1 = (c + 1 <= r) ? __uint_as_float(src[1]) : 0.f;
-            o[e2] = pack2(x0, x1);
+            for (int e2 = 0; e2 < 4; ++e2) {
+                const int cl = 8 * jj + 2 * e2, c = 8 * j2 + cl;
+                const float x0 = (c <= r) ? __uint_as_float(v[cl]) : 0.f;
+                const float x1 = (c + 1 <= r) ? __uint_as_float(v[cl + 1]) : 0.f;
+                o[e2] = pack2(x0, x1);
+            }
+            sts128(p_tile + sw128_off(r, j2 + jj), o[0], o[1], o[2], o[3]);
         }
-        sts128(p_tile + sw128_off(r, j), o[0], o[1], o[2], o[3]);
     }
 }
 
 // ---------------------------------------------------------------------------
 // T = (I + L)^{-1} for a strictly lower 64 x 64 fp32 L in sL (row stride
 // kLDL), run by 4 warps (sw = 0..3) that synchronise on named barrier
-// `bar_id`: the four 16x16 diagonal blocks by substitution, then a block
-// forward substitution by 8-column strips with mma.sync tf32.  Blocks of sT
-// above the diagonal blocks must be zero on entry (they are never written).
-// sXw is 4 x [16][17] fp32 warp-private scratch.  On return each warp has
-// written its strips; the caller orders them before any other reader.
+// `bar_id`.  With 16x16 blocks, D_i = (I + L_ii)^{-1} and M_ik = D_i L_ik:
+//   phase 1: the four D_i by substitution (one block per warp, one column
+//            per lane);
+//   phase 2: the six M_ik (i > k), written over L_ik;
+//   phase 3: block forward substitution T_ij = -sum_{j <= k < i} M_ik T_kj
+//            (T_jj = D_j) by 8-column strips with mma.sync tf32.
+// Scaling the blocks first keeps every step of the substitution one product
+// whose operands are already in shared memory.  Blocks of sT above the
+// diagonal must be zero on entry (they are never written); sL's off-diagonal
+// blocks are overwritten.  On return each warp has written its strips (warps
+// 0, 1: block column 0; warps 2, 3: block columns 1 and 2; D_3 since phase
+// 1); the caller orders them before any other reader.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void invert_unit_lower(int sw, int lane, const float *sL, float *sT,
-                                                  float *sXw, uint32_t bar_id) {
+// acc += A_blk B_blk over one 16-wide k block: A rows 16 ai (row stride kLDL)
+// from column 16 ak, B rows 16 ak .. from column c0 (an 8-column strip).
+__device__ __forceinline__ void blk_mma(float (&acc)[4], const float *A, int ai, int ak,
+                                        const float *B, int c0, int g, int tq) {
+#pragma unroll
+    for (int kk = 0; kk < 16; kk += 8) {
+        const float *Ar = A + (16 * ai + g) * kLDL + 16 * ak + kk + tq;
+        const uint32_t af[4] = {tf32_bits(Ar[0]), tf32_bits(Ar[8 * kLDL]), tf32_bits(Ar[4]),
+                                tf32_bits(Ar[8 * kLDL + 4])};
+        const float *Bc = B + (16 * ak + kk + tq) * kLDL + c0 + g;
+        const uint32_t bfr[2] = {tf32_bits(Bc[0]), tf32_bits(Bc[4 * kLDL])};
+        mma_tf32_16x8x8(acc, af, bfr);
+    }
+}
+// C fragment (16 x 8) -> -C at rows 16 i of the strip at column c0 of sT
+__device__ __forceinline__ void store_neg(float *sT, int i, int c0, const float (&d)[4], int g,
+                                          int tq) {
+    float *o = sT + (16 * i) * kLDL + c0;
+    o[g * kLDL + 2 * tq] = -d[0];
+    o[g * kLDL + 2 * tq + 1] = -d[1];
+    o[(g + 8) * kLDL + 2 * tq] = -d[2];
+    o[(g + 8) * kLDL + 2 * tq + 1] = -d[3];
+}
+
+__device__ __forceinline__ void invert_unit_lower(int sw, int lane, float *sL, float *sT,
+                                                  uint32_t bar_id) {
     const int g = lane >> 2, tq = lane & 3;
     // phase 1: invert the four 16x16 diagonal blocks, one block per warp, one
     // column per lane (lanes 0-15)
@@ -365,58 +395,78 @@ __device__ __forceinline__ void invert_unit_lower(int sw, int lane, const float 
     }
     named_bar(bar_id, kSolveThreads);
 
-    // phase 2: block forward substitution by 8-column strips.  Block rows
-    // above a strip's block column cb are zero, block row cb is D_cb, and for
-    // i > cb:  T_i = -D_i * sum_{cb <= j < i} L_ij T_j.  Column block 0 costs
-    // the most (three block rows), so its two strips go to warps 0 and 1 and
-    // warps 2 and 3 take the strips of blocks 1 and 2; block 3 is D_3 alone.
-    // A strip only reads L, the diagonal blocks and its own columns, so no
-    // barrier is needed until Tb is written.  X goes through a warp-private
-    // [16][17] scratch to turn accumulator fragments into B fragments.
+    // phase 2: M_ik = D_i L_ik for the six blocks below the diagonal, twelve
+    // 8-column halves, three per warp: unit u -> block (i, k) and half h
     {
-        float *xw = sXw + sw * 16 * 17;
-        const int q = sw & 1;
-#pragma unroll 1
-        for (int pass = 0; pass < 2; ++pass) {
-            const int cb = sw < 2 ? (pass == 0 ? 0 : 4) : 1 + pass;
-            const int c0 = 16 * cb + 8 * q;
-            for (int i = cb + 1; i < 4; ++i) {
-                // two accumulators (k halves of each block) halve the mma chain
-                float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-                for (int jb = cb; jb < i; ++jb) {
+        float m[3][4];
 #pragma unroll
-                    for (int kk = 0; kk < 16; kk += 8) {
-                        const float *Lr = sL + (16 * i + g) * kLDL + 16 * jb + kk + tq;
-                        const uint32_t af[4] = {tf32_bits(Lr[0]), tf32_bits(Lr[8 * kLDL]),
-                                                tf32_bits(Lr[4]), tf32_bits(Lr[8 * kLDL + 4])};
-                        const float *Tc = sT + (16 * jb + kk + tq) * kLDL + c0 + g;
-                        const uint32_t bfr[2] = {tf32_bits(Tc[0]), tf32_bits(Tc[4 * kLDL])};
-                        mma_tf32_16x8x8(acc[kk >> 3], af, bfr);
-                    }
-                }
-                xw[g * 17 + 2 * tq] = acc[0][0] + acc[1][0];
-                xw[g * 17 + 2 * tq + 1] = acc[0][1] + acc[1][1];
-                xw[(g + 8) * 17 + 2 * tq] = acc[0][2] + acc[1][2];
-                xw[(g + 8) * 17 + 2 * tq + 1] = acc[0][3] + acc[1][3];
-                __syncwarp();
-                float d[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int v = 0; v < 3; ++v) {
+            const int u = sw + 4 * v;                 // 0..11
+            const int blk = u >> 1, h = u & 1;        // blocks (1,0) (2,0) (2,1) (3,0) (3,1) (3,2)
+            const int i = blk < 1 ? 1 : blk < 3 ? 2 : 3;
+            const int k = blk < 1 ? 0 : blk < 3 ? blk - 1 : blk - 3;
 #pragma unroll
-                for (int kk = 0; kk < 16; kk += 8) {
-                    const float *Dr = sT + (16 * i + g) * kLDL + 16 * i + kk + tq;
-                    const uint32_t af[4] = {tf32_bits(Dr[0]), tf32_bits(Dr[8 * kLDL]),
-                                            tf32_bits(Dr[4]), tf32_bits(Dr[8 * kLDL + 4])};
-                    const uint32_t bfr[2] = {tf32_bits(xw[(kk + tq) * 17 + g]),
-                                             tf32_bits(xw[(kk + tq + 4) * 17 + g])};
-                    mma_tf32_16x8x8(d, af, bfr);
-                }
-                float *o = sT + (16 * i) * kLDL + c0;
-                o[g * kLDL + 2 * tq] = -d[0];
-                o[g * kLDL + 2 * tq + 1] = -d[1];
-                o[(g + 8) * kLDL + 2 * tq] = -d[2];
-                o[(g + 8) * kLDL + 2 * tq + 1] = -d[3];
-                __syncwarp();
+            for (int e = 0; e < 4; ++e) m[v][e] = 0.f;
+            // D_i (rows and columns of block i in sT) times L_ik (rows of block i in sL)
+#pragma unroll
+            for (int kk = 0; kk < 16; kk += 8) {
+                const float *Ar = sT + (16 * i + g) * kLDL + 16 * i + kk + tq;
+                const uint32_t af[4] = {tf32_bits(Ar[0]), tf32_bits(Ar[8 * kLDL]), tf32_bits(Ar[4]),
+                                        tf32_bits(Ar[8 * kLDL + 4])};
+                const float *Bc = sL + (16 * i + kk + tq) * kLDL + 16 * k + 8 * h + g;
+                const uint32_t bfr[2] = {tf32_bits(Bc[0]), tf32_bits(Bc[4 * kLDL])};
+                mma_tf32_16x8x8(m[v], af, bfr);
             }
         }
+        named_bar(bar_id, kSolveThreads);   // every L_ik read before M_ik lands on it
+#pragma unroll
+        for (int v = 0; v < 3; ++v) {
+            const int u = sw + 4 * v;
+            const int blk = u >> 1, h = u & 1;
+            const int i = blk < 1 ? 1 : blk < 3 ? 2 : 3;
+            const int k = blk < 1 ? 0 : blk < 3 ? blk - 1 : blk - 3;
+            float *o = sL + (16 * i) * kLDL + 16 * k + 8 * h;
+            o[g * kLDL + 2 * tq] = m[v][0];
+            o[g * kLDL + 2 * tq + 1] = m[v][1];
+            o[(g + 8) * kLDL + 2 * tq] = m[v][2];
+            o[(g + 8) * kLDL + 2 * tq + 1] = m[v][3];
+        }
+        named_bar(bar_id, kSolveThreads);
+    }
+
+    // phase 3: each strip only reads M, the diagonal blocks and its own
+    // columns, so a warp needs no barrier until Tb is written.  Products that
+    // do not wait on the strip's latest block are issued a step early.
+    const int q = sw & 1;
+    if (sw < 2) {
+        const int c0 = 8 * q;   // block column 0
+        float t1[4] = {0.f, 0.f, 0.f, 0.f}, t2[4] = {0.f, 0.f, 0.f, 0.f},
+              t3[4] = {0.f, 0.f, 0.f, 0.f};
+        blk_mma(t1, sL, 1, 0, sT, c0, g, tq);
+        blk_mma(t2, sL, 2, 0, sT, c0, g, tq);
+        blk_mma(t3, sL, 3, 0, sT, c0, g, tq);
+        store_neg(sT, 1, c0, t1, g, tq);
+        __syncwarp();
+        blk_mma(t2, sL, 2, 1, sT, c0, g, tq);
+        blk_mma(t3, sL, 3, 1, sT, c0, g, tq);
+        store_neg(sT, 2, c0, t2, g, tq);
+        __syncwarp();
+        blk_mma(t3, sL, 3, 2, sT, c0, g, tq);
+        store_neg(sT, 3, c0, t3, g, tq);
+        __syncwarp();
+    } else {
+        const int c1 = 16 + 8 * q, c2 = 32 + 8 * q;   // block columns 1 and 2
+        float t21[4] = {0.f, 0.f, 0.f, 0.f}, t31[4] = {0.f, 0.f, 0.f, 0.f},
+              t32[4] = {0.f, 0.f, 0.f, 0.f};
+        blk_mma(t21, sL, 2, 1, sT, c1, g, tq);
+        blk_mma(t31, sL, 3, 1, sT, c1, g, tq);
+        blk_mma(t32, sL, 3, 2, sT, c2, g, tq);
+        store_neg(sT, 2, c1, t21, g, tq);
+        store_neg(sT, 3, c2, t32, g, tq);
+        __syncwarp();
+        blk_mma(t31, sL, 3, 2, sT, c1, g, tq);
+        store_neg(sT, 3, c1, t31, g, tq);
+        __syncwarp();
     }
 }
 
@@ -425,21 +475,22 @@ __device__ __forceinline__ void invert_unit_lower(int sw, int lane, const float 
 __device__ __forceinline__ void build_l(int sw, int lane, uint32_t tmem, uint32_t tm_ap, float *sL,
                                         const float *sB_s) {
     const int r = 32 * sw + lane;
-    uint32_t v0[32], v1[32];
-    tmem_ld32(tmem_addr(tmem, 32 * sw, tm_ap), v0);
-    tmem_ld32(tmem_addr(tmem, 32 * sw, tm_ap + 32), v1);
-    tmem_wait_ld();
     const float br = sB_s[r];
     float *Lr = sL + r * kLDL;
+#pragma unroll 1
+    for (int c0 = 0; c0 < 64; c0 += 16) {
+        uint32_t v[16];
+        tmem_ld16(tmem_addr(tmem, 32 * sw, tm_ap + c0), v);
+        tmem_wait_ld();
 #pragma unroll
-    for (int c = 0; c < 64; c += 4) {
-        const uint32_t *src = c < 32 ? &v0[c] : &v1[c - 32];
-        float4 w;
-        w.x = (c + 0 < r) ? br * __uint_as_float(src[0]) : 0.f;
-        w.y = (c + 1 < r) ? br * __uint_as_float(src[1]) : 0.f;
-        w.z = (c + 2 < r) ? br * __uint_as_float(src[2]) : 0.f;
-        w.w = (c + 3 < r) ? br * __uint_as_float(src[3]) : 0.f;
-        *reinterpret_cast<float4 *>(Lr + c) = w;
+        for (int c = 0; c < 16; c += 4) {
+            float4 w;
+            w.x = (c0 + c + 0 < r) ? br * __uint_as_float(v[c]) : 0.f;
+            w.y = (c0 + c + 1 < r) ? br * __uint_as_float(v[c + 1]) : 0.f;
+            w.z = (c0 + c + 2 < r) ? br * __uint_as_float(v[c + 2]) : 0.f;
+            w.w = (c0 + c + 3 < r) ? br * __uint_as_float(v[c + 3]) : 0.f;
+            *reinterpret_cast<float4 *>(Lr + c0 + c) = w;
+        }
     }
 }
 
@@ -448,7 +499,7 @@ __device__ __forceinline__ void build_l(int sw, int lane, uint32_t tmem, uint32_
 // and arrives on `ap_free` itself, later.
 template <bool kEarlyP = true>
 __device__ __forceinline__ void solve_chunk(int sw, int lane, uint32_t tmem, uint32_t tm_ap,
-                                            uint32_t p_tile, float *sL, float *sT, float *sXw,
+                                            uint32_t p_tile, float *sL, float *sT,
                                             const float *sB_s, uint64_t *ap_free,
                                             uint32_t bar_id) {
     const int t = sw * 32 + lane;
@@ -461,7 +512,7 @@ __device__ __forceinline__ void solve_chunk(int sw, int lane, uint32_t tmem, uin
     named_bar(bar_id, kSolveThreads);
     if (kEarlyP && t == 0) mbar_arrive(ap_free);
 
-    invert_unit_lower(sw, lane, sL, sT, sXw, bar_id);
+    invert_unit_lower(sw, lane, sL, sT, bar_id);
 }
 
 // Tb = T diag(b) -> bf16 into rows 0..63 of the K-major tile at `tp`, one

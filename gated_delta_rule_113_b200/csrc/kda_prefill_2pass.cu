@@ -948,7 +948,10 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
                 if (c == 0) KDA_TRACE2(j, 10);
                 if (j > 0) store_snapshot(j);
             } else {
-                // O rows: D1 lanes 64..127 -> bf16 output
+                // O rows: D1 lanes 64..127 -> bf16 output, once U is converted:
+                // these global stores share the load/store pipe with the U rows'
+                // shared-memory stores on the chain's critical path
+                if (!wait_or_abort(&bars[cbUbFull], j & 1, abort_flag, p.status)) { ok = false; break; }
                 const int c0 = t0 + j * kChunk, L = min(kChunk, t1 - c0);
                 const int r = c - 64;
 #pragma unroll

@@ -2,6 +2,8 @@
 // prefill kernel relies on.  One CTA stages A (M x K) and B (K x N) in shared
 // memory in a chosen major-ness / swizzle, issues K/16 MMAs into TMEM, and
 // copies every TMEM lane x column back, so the host can compare D with A*B.
+// With a_tmem, A is first written into tensor memory (columns 128 ..) by the
+// four warps and the MMAs read it from there.
 // Built and run only by tests/test_gpu_tcgen05_layouts.py.
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -16,6 +18,7 @@ struct ProbeCfg {
     int b_mn;      // B stored MN-major (1) or K-major (0)
     int b_swz;     // B swizzle: 128 or 64 (64 only for MN-major with N == 32)
     int neg_a;
+    int a_tmem;    // A staged in tensor memory (packed bf16 pairs, lane = row) instead
 };
 
 // byte offset of A(m, k) and B(k, n) inside their tiles
@@ -64,6 +67,23 @@ __global__ void __launch_bounds__(128) probe_kernel(ProbeCfg c, const uint16_t *
     }
     fence_proxy_async();
     if (warp == 0) tmem_alloc(&tbase, 256);
+    __syncthreads();
+    if (c.a_tmem) {
+        // lane m = tid holds row m of A: column 128 + j packs (A[m][2j], A[m][2j+1]),
+        // the even element in the low half
+        tc_fence_after();
+        const int m = tid;
+        for (int j0 = 0; j0 < c.K / 2; j0 += 16) {
+            uint32_t r[16];
+            for (int j = 0; j < 16; ++j) {
+                const uint32_t lo = m < c.M ? A[m * c.K + 2 * (j0 + j)] : 0u;
+                const uint32_t hi = m < c.M ? A[m * c.K + 2 * (j0 + j) + 1] : 0u;
+                r[j] = lo | (hi << 16);
+            }
+            tmem_st16(tmem_addr(tbase, warp * 32, 128 + j0), r);
+        }
+        tmem_wait_st();
+    }
     if (tid == 0) {
         mbar_init(&bar, 1);
         fence_mbar_init();
@@ -77,7 +97,7 @@ __global__ void __launch_bounds__(128) probe_kernel(ProbeCfg c, const uint16_t *
         const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
         const uint32_t idesc = idesc_bf16(c.M, c.N, c.a_mn, c.b_mn, c.neg_a);
         for (int ks = 0; ks < c.K / 16; ++ks) {
-            uint64_t ad, bd;
+            uint64_t ad = 0, bd;
             if (!c.a_mn) {
                 ad = smem_desc(a0 + (ks / 4) * (c.M * 128) + (ks % 4) * 32, 16, 1024, kSw128);
             } else {
@@ -90,7 +110,8 @@ __global__ void __launch_bounds__(128) probe_kernel(ProbeCfg c, const uint16_t *
             } else {
                 bd = smem_desc(b0 + ks * 2048, c.K * 128, 1024, kSw128);
             }
-            mma_bf16(tm, ad, bd, idesc, ks > 0 ? 1u : 0u);
+            if (c.a_tmem) mma_bf16_ta(tm, tm + 128 + 8 * ks, bd, idesc, ks > 0 ? 1u : 0u);
+            else mma_bf16(tm, ad, bd, idesc, ks > 0 ? 1u : 0u);
         }
         mma_commit(&bar);
     }
@@ -118,9 +139,10 @@ __global__ void __launch_bounds__(128) probe_kernel(ProbeCfg c, const uint16_t *
 }
 
 extern "C" int umma_probe(int M, int N, int K, int a_mn, int b_mn, int b_swz, int neg_a,
-                          const uint16_t *A_h, const uint16_t *B_h, float *D_h) {
+                          int a_tmem, const uint16_t *A_h, const uint16_t *B_h, float *D_h) {
     if (M * K * 2 > 32768 || K * N * 2 > 32768 || N % 32 != 0 || N > 256) return -1;
-    ProbeCfg c{M, N, K, a_mn, b_mn, b_swz, neg_a};
+    if (a_tmem && (M != 128 || N > 128 || K % 32 != 0 || K > 128 || a_mn)) return -1;
+    ProbeCfg c{M, N, K, a_mn, b_mn, b_swz, neg_a, a_tmem};
     uint16_t *A, *B;
     float *D;
     int *err;

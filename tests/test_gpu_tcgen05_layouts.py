@@ -33,18 +33,21 @@ def _bf16(x):
     return t.view(torch.int16).numpy().astype(np.uint16), t.float().double().numpy()
 
 
-def _run(lib, M, N, K, a_mn, b_mn, b_swz, neg_a=0, seed=0):
+def _run(lib, M, N, K, a_mn, b_mn, b_swz, neg_a=0, seed=0, a_tmem=0):
     rng = np.random.default_rng(seed)
     A_bits, A = _bf16(rng.standard_normal((M, K)))
     B_bits, B = _bf16(rng.standard_normal((K, N)))
     D = np.zeros((128, N), dtype=np.float32)
     p16 = ctypes.POINTER(ctypes.c_uint16)
-    rc = lib.umma_probe(M, N, K, a_mn, b_mn, b_swz, neg_a,
+    rc = lib.umma_probe(M, N, K, a_mn, b_mn, b_swz, neg_a, a_tmem,
                         np.ascontiguousarray(A_bits).ctypes.data_as(p16),
                         np.ascontiguousarray(B_bits).ctypes.data_as(p16),
                         D.ctypes.data_as(ctypes.POINTER(ctypes.c_float)))
     assert rc == 0, f"probe returned {rc}"
     ref = (-1.0 if neg_a else 1.0) * (A @ B)
+    if a_tmem:   # also the product with each column pair of A swapped
+        Asw = A.reshape(M, K // 2, 2)[:, :, ::-1].reshape(M, K)
+        return D.astype(np.float64), ref, Asw @ B
     return D.astype(np.float64), ref
 
 
@@ -72,3 +75,18 @@ def test_umma_m64_lane_layout(probe):
     split = np.max(np.abs(D[rows] - ref)) / np.max(np.abs(ref))
     print(f"M=64 layout: dense lanes 0-63 err {dense:.3e}; 16-per-quarter err {split:.3e}")
     assert min(dense, split) < 1e-5
+
+
+@pytest.mark.parametrize("N,K,b_mn,b_swz", [
+    (128, 128, 0, 128),   # S^T x [-W;Qe]^T  (B K-major, two K atoms)
+    (128, 64, 1, 128),    # U^T x Ki          (B MN-major, two N blocks)
+    (64, 64, 1, 128),
+])
+def test_umma_a_from_tensor_memory(probe, N, K, b_mn, b_swz):
+    """A staged in tensor memory as packed bf16 pairs (lane = row, column j =
+    elements 2j and 2j+1, the even one in the low half) for M = 128."""
+    D, ref, ref_swapped = _run(probe, 128, N, K, 0, b_mn, b_swz, a_tmem=1)
+    err = np.max(np.abs(D - ref)) / np.max(np.abs(ref))
+    err_sw = np.max(np.abs(D - ref_swapped)) / np.max(np.abs(ref_swapped))
+    print(f"A in TMEM: even-low err {err:.3e}, odd-low err {err_sw:.3e}")
+    assert err < 1e-5, f"max rel err {err:.3e} (swapped pairs: {err_sw:.3e})"

@@ -996,6 +996,346 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
     }
 }
 
+// ------------------------------------------------ pass 2, transposed chain
+// For full-width (128-column) value slices the chain runs transposed, with
+// TMEM lane = value column v:
+//   D1^T  = V^T [Tb; PT]^T        (columns 0-63: U^T, 64-127: P U0 parts)
+//   D1^T += S^T [-W; Qe]^T        (columns 0-63: U^T, 64-127: O^T)
+//   dS^T  = U^T Ki ;  S^T <- (S^T + dS^T) Diag(Gam_L)
+// S^T (bf16) and U^T (bf16) are the A operands of the two products on the
+// chain and go to tensor memory with tcgen05.st, so nothing on the chain
+// passes through shared memory except the packet and V tiles, which every
+// product reads as its B operand (or A, for V^T) exactly as they landed.
+// Warp w (of 8) keeps lane quarter w % 4 (v = 32 (w % 4) + lane) and half
+// w / 4: key channels 64 (w / 4) .. + 63 of the state, positions
+// 32 (w / 4) .. + 31 of U and O.
+constexpr int kCtChain = 8, kCtLoad = 8, kCtMma = 9, kCtThreads = 10 * 32;
+struct ChTLayout {
+    static constexpr uint32_t kKQ = kPkKQ, kKI = kPkKI, kTP = kPkTP, kGL = kPkGL;
+    static constexpr uint32_t kV = (kPkGL + 512 + 1023) / 1024 * 1024;   // two 64-column atoms
+    static constexpr uint32_t kStage = (kV + 64 * 128 * 2 + 1023) / 1024 * 1024;
+    static constexpr int kStages = 2;
+    static constexpr uint32_t kOS = kStages * kStage;   // 8 x [32 positions][32 columns] bf16
+    static constexpr uint32_t kBar = kOS + kCtChain * 2048;
+    static constexpr uint32_t kMisc = kBar + 16 * 8;
+    static constexpr uint32_t kAlloc = kMisc + 16 + 1024;
+    static_assert(kAlloc <= 232448, "shared memory budget exceeded");
+    static constexpr uint32_t kTmD1 = 0;     // + 128 d, d = chunk & 1
+    static constexpr uint32_t kTmD2 = 256;   // dS^T, 128 columns
+    static constexpr uint32_t kTmAS = 384;   // S^T as bf16 pairs, 64 columns
+    static constexpr uint32_t kTmAU = 448;   // U^T as bf16 pairs, 32 columns
+    static constexpr uint32_t kTmCols = 512;
+};
+
+__global__ void __launch_bounds__(kCtThreads, 1)
+chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
+    using Ly = ChTLayout;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const uint32_t sbase = smem_u32(sm);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + Ly::kBar);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + Ly::kMisc);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + Ly::kMisc + 4);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // a programmatic dependent of the key-side pass: packets and the work
+    // order are read only after that pass is done
+    grid_dependency_wait();
+    const int seq = p.order[blockIdx.x / p.H];
+    const int h = blockIdx.x % p.H;
+    int t0, t1;
+    if (!seq_range(p.cu, seq, p.T, t0, t1)) {
+        if (tid == 0) set_status(p.status, KDA_ERR_SEQLENS);
+        return;
+    }
+    const int nchunks = (t1 - t0 + kChunk - 1) / kChunk;
+    const int g0 = p.chunk_off[seq];
+    if (g0 < 0 || ((long long)g0 + nchunks) * p.H > p.slots) {
+        if (tid == 0) set_status(p.status, KDA_ERR_SEQLENS);
+        return;
+    }
+    const size_t sbase_g = ((size_t)seq * p.H + h) * kDK * kDV;
+
+    if (tid == 0) {
+        for (int i = 0; i < cbNum; ++i) {
+            uint32_t cnt = 1;
+            if (i == cbSbFull || i == cbUbFull || i == cbD1Free || i == cbD1Free + 1) cnt = kCtChain;
+            if (i >= cbStageFree && i < cbStageFree + Ly::kStages) cnt = 1 + kCtChain;
+            mbar_init(&bars[i], cnt);
+        }
+        abort_flag[0] = 0;
+        abort_flag[1] = 0;
+        fence_mbar_init();
+    }
+    if (warp == kCtLoad && lane == 0) prefetch_tmap(&tm_v);
+    if (warp == kCtMma) {
+        tmem_alloc(tmem_slot, Ly::kTmCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    KDA_SPAN(g_kda_span2, 0);
+
+    auto packet = [&](int j) {
+        return p.packets + ((size_t)(g0 + j) * p.H + h) * kPacketBytes;
+    };
+
+    if (warp == kCtLoad) {
+        // ------------------------------------------------------- loader
+        int n_issued = 0;
+#pragma unroll 1
+        for (int j = 0; j < nchunks; ++j) {
+            const int s = j % Ly::kStages;
+            bool ok = true;
+            if (lane == 0 && j >= Ly::kStages)
+                ok = wait_or_abort(&bars[cbStageFree + s], (j / Ly::kStages - 1) & 1, abort_flag, p.status);
+            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+            unsigned char *st = sm + s * Ly::kStage;
+            uint64_t *full = &bars[cbFull + s];
+            if (lane == 0) mbar_arrive_expect_tx(full, (uint32_t)kPacketBytes + 64 * 128 * 2);
+            __syncwarp();
+            if (lane < 4) {   // the packet in four pieces, one per lane
+                const uint32_t off = lane * 16384u;
+                const uint32_t len = lane < 3 ? 16384u : (uint32_t)kPacketBytes - 3 * 16384u;
+                bulk_load(st + off, packet(j) + off, len, full);
+            }
+            if (lane == 4) tma_load_3d(st + Ly::kV, &tm_v, full, 0, h, t0 + j * kChunk);
+            if (lane == 7) tma_load_3d(st + Ly::kV + 64 * 128, &tm_v, full, 64, h, t0 + j * kChunk);
+            if (j + Ly::kStages < nchunks) {   // warm L2 for the copies of chunk j + 2
+                if (lane == 5) bulk_prefetch_l2(packet(j + Ly::kStages), (uint32_t)kPacketBytes);
+                if (lane == 8) tma_prefetch_3d(&tm_v, 0, h, t0 + (j + Ly::kStages) * kChunk);
+                if (lane == 9) tma_prefetch_3d(&tm_v, 64, h, t0 + (j + Ly::kStages) * kChunk);
+            }
+            n_issued = j + 1;
+            if (lane == 0) KDA_TRACE2(j, 0);
+#ifdef KDA_TRACE
+            if (lane == 6) {
+                mbar_wait(full, (j / Ly::kStages) & 1);
+                KDA_TRACE2(j, 11);
+            }
+#endif
+        }
+        if (lane == 0)
+            for (int j = max(0, n_issued - Ly::kStages); j < n_issued; ++j)
+                mbar_wait(&bars[cbFull + j % Ly::kStages], (j / Ly::kStages) & 1);
+    } else if (warp == kCtMma) {
+        // ------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t kIdU0 = idesc_bf16(128, 128, 1, 0);   // V^T (MN-major) x [Tb;PT]^T
+            constexpr uint32_t kIdS = idesc_bf16(128, 128, 0, 0);    // S^T (TMEM) x [-W;Qe]^T
+            constexpr uint32_t kIdDs = idesc_bf16(128, 128, 0, 1);   // U^T (TMEM) x Ki (MN-major)
+            auto issue_u0 = [&](int j) -> bool {
+                const int s = j % Ly::kStages, d = j & 1;
+                const uint32_t st = sbase + s * Ly::kStage;
+                if (!spin_or_abort(&bars[cbFull + s], (j / Ly::kStages) & 1, abort_flag, p.status))
+                    return false;
+                KDA_TRACE2(j, 12);
+                if (j >= 2 && !spin_or_abort(&bars[cbD1Free + d], ((j - 2) >> 1) & 1, abort_flag,
+                                             p.status))
+                    return false;
+                KDA_TRACE2(j, 1);
+                tc_fence_after();
+                const uint64_t d_v = smem_desc(st + Ly::kV, 64 * 128, 1024, kSw128);
+                const uint64_t d_tp = smem_desc(st + Ly::kTP, 16, 1024, kSw128);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16(tmem + Ly::kTmD1 + d * 128, d_v + ((uint64_t)(ks * 2048) >> 4),
+                             d_tp + ((uint64_t)(ks * 32) >> 4), kIdU0, ks > 0);
+                return true;
+            };
+            bool ok = !p.test_stall || spin_or_abort(&bars[cbNever], 0, abort_flag, p.status);
+            ok = ok && nchunks > 0 && issue_u0(0);
+#pragma unroll 1
+            for (int j = 0; j < nchunks && ok; ++j) {
+                const int s = j % Ly::kStages, d = j & 1;
+                const uint32_t st = sbase + s * Ly::kStage;
+                const uint32_t d1 = tmem + Ly::kTmD1 + d * 128;
+                if (!spin_or_abort(&bars[cbSbFull], j & 1, abort_flag, p.status)) break;
+                KDA_TRACE2(j, 2);
+                tc_fence_after();
+                const uint64_t d_kq = smem_desc(st + Ly::kKQ, 16, 1024, kSw128);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)   // D1^T += S^T [-W; Qe]^T
+                    mma_bf16_ta(d1, tmem + Ly::kTmAS + 8 * ks, d_kq + kmaj_step(ks, 16384), kIdS, 1);
+                mma_commit(&bars[cbUFull]);
+                KDA_TRACE2(j, 3);
+                // the next chunk's V^T [Tb; PT]^T now if its tiles have landed,
+                // otherwise after dS
+                bool u0_next = j + 1 >= nchunks;
+                if (!u0_next) {
+                    const int s1 = (j + 1) % Ly::kStages, d1n = (j + 1) & 1;
+                    if (mbar_test_wait(&bars[cbFull + s1], ((j + 1) / Ly::kStages) & 1) &&
+                        (j + 1 < 2 || mbar_test_wait(&bars[cbD1Free + d1n], ((j - 1) >> 1) & 1))) {
+                        if (!issue_u0(j + 1)) break;
+                        u0_next = true;
+                    }
+                }
+                if (!spin_or_abort(&bars[cbUbFull], j & 1, abort_flag, p.status)) break;
+                KDA_TRACE2(j, 4);
+                tc_fence_after();
+                const uint64_t d_ki = smem_desc(st + Ly::kKI, 64 * 128, 1024, kSw128);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)   // dS^T = U^T Ki
+                    mma_bf16_ta(tmem + Ly::kTmD2, tmem + Ly::kTmAU + 8 * ks,
+                                d_ki + ((uint64_t)(ks * 2048) >> 4), kIdDs, ks > 0);
+                mma_commit(&bars[cbDsFull]);
+                mma_commit(&bars[cbStageFree + s]);
+                KDA_TRACE2(j, 5);
+                if (!u0_next && !issue_u0(j + 1)) break;
+            }
+            mma_commit(&bars[cbDrain]);
+            mbar_wait(&bars[cbDrain], 0);
+        }
+    } else {
+        // ------------------------------------------------------ chain warps
+        const int wq = warp & 3, hf = warp >> 2;
+        const int v = 32 * wq + lane;           // value column (TMEM lane)
+        const int cb = 64 * hf;                 // first key channel of this thread's state
+        float S[64];                            // S[c] = state[cb + c][v]
+        {
+            const float *src = p.S0 ? p.S0 + sbase_g : nullptr;
+            if (p.s0_slot) {   // resume from a pool slot (prefix-cache hit)
+                const long long slot = p.s0_slot[seq];
+                if (slot >= p.snap_slots) {
+                    if (tid == 0) set_status(p.status, KDA_ERR_SLOT);
+                    src = nullptr;
+                } else if (slot >= 0) {
+                    src = p.snap_pool + ((size_t)slot * p.H + h) * kDK * kDV;
+                }
+            }
+#pragma unroll
+            for (int c = 0; c < 64; ++c) S[c] = src ? src[(size_t)(cb + c) * kDV + v] : 0.f;
+        }
+        auto store_state = [&](float *dst) {   // dst: a [Dk][Dv] state
+#pragma unroll
+            for (int c = 0; c < 64; ++c) dst[(size_t)(cb + c) * kDV + v] = S[c];
+        };
+        bool ok = true;
+        const long long snap_base = (p.snap_every > 0 && p.snap_base) ? p.snap_base[seq] : -1;
+        auto store_snapshot = [&](int j) {
+            if (j <= 0 || snap_base < 0 || j % p.snap_every != 0 || j * kChunk > t1 - t0) return;
+            const long long slot = snap_base + j / p.snap_every - 1;
+            if (slot < p.snap_slots && KDA_IN_RANGE(slot >= 0, p.status))
+                store_state(p.snap_pool + ((size_t)slot * p.H + h) * kDK * kDV);
+            else if (tid == 0)
+                set_status(p.status, KDA_ERR_SLOT);
+        };
+#pragma unroll 1
+        for (int j = 0; j <= nchunks && ok; ++j) {
+            if (j > 0) {
+                // S^T <- (S^T + dS^T) Diag(Gam_L) for chunk j-1; then its stage
+                // may be refilled
+                const int sp = (j - 1) % Ly::kStages;
+                if (!spin_or_abort(&bars[cbDsFull], (j - 1) & 1, abort_flag, p.status)) { ok = false; break; }
+                if (tid == 0) KDA_TRACE2(j - 1, 6);
+                tc_fence_after();
+                const float4 *gl = reinterpret_cast<const float4 *>(sm + sp * Ly::kStage + Ly::kGL) + cb / 4;
+#pragma unroll
+                for (int jj = 0; jj < 64; jj += 32) {
+                    uint32_t dv[32];
+                    tmem_ld32(tmem_addr(tmem, 32 * wq, Ly::kTmD2 + cb + jj), dv);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; e += 4) {
+                        const float4 g = gl[(jj + e) / 4];
+                        S[jj + e] = g.x * (S[jj + e] + __uint_as_float(dv[e]));
+                        S[jj + e + 1] = g.y * (S[jj + e + 1] + __uint_as_float(dv[e + 1]));
+                        S[jj + e + 2] = g.z * (S[jj + e + 2] + __uint_as_float(dv[e + 2]));
+                        S[jj + e + 3] = g.w * (S[jj + e + 3] + __uint_as_float(dv[e + 3]));
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars[cbStageFree + sp]);
+                if (tid == 0) KDA_TRACE2(j - 1, 14);
+            }
+            if (j == nchunks) {
+                store_snapshot(j);
+                break;
+            }
+            const int s = j % Ly::kStages, d = j & 1;
+            if (!spin_or_abort(&bars[cbFull + s], (j / Ly::kStages) & 1, abort_flag, p.status)) { ok = false; break; }
+            if (tid == 0) KDA_TRACE2(j, 7);
+            {   // S^T as bf16 pairs -> the A operand of D1^T += S^T [-W; Qe]^T
+#pragma unroll
+                for (int jj = 0; jj < 64; jj += 32) {
+                    uint32_t w[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) w[e] = pack2(S[jj + 2 * e], S[jj + 2 * e + 1]);
+                    tmem_st16(tmem_addr(tmem, 32 * wq, Ly::kTmAS + cb / 2 + jj / 2), w);
+                }
+                tmem_wait_st();
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[cbSbFull]);
+            if (tid == 0) KDA_TRACE2(j, 8);
+            // the state entering chunk j, for the chunked backward
+            if (p.ckpt && KDA_IN_RANGE(((long long)g0 + j) * p.H + h < p.slots, p.status))
+                store_state(p.ckpt + ((size_t)(g0 + j) * p.H + h) * kDK * kDV);
+            if (j > 0) store_snapshot(j);
+
+            if (!spin_or_abort(&bars[cbUFull], j & 1, abort_flag, p.status)) { ok = false; break; }
+            if (tid == 0) KDA_TRACE2(j, 9);
+            tc_fence_after();
+            {   // U^T positions 32 hf .. + 31 -> bf16 pairs, the A operand of dS^T
+                uint32_t u[32];
+                tmem_ld32(tmem_addr(tmem, 32 * wq, Ly::kTmD1 + d * 128 + 32 * hf), u);
+                tmem_wait_ld();
+                uint32_t w[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    w[e] = pack2(__uint_as_float(u[2 * e]), __uint_as_float(u[2 * e + 1]));
+                tmem_st16(tmem_addr(tmem, 32 * wq, Ly::kTmAU + 16 * hf), w);
+                tmem_wait_st();
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[cbUbFull]);
+            if (tid == 0) KDA_TRACE2(j, 10);
+            {   // O^T positions 32 hf .. + 31, columns 32 wq .. + 31 -> bf16 output
+                // rows, through a per-warp transpose in shared memory so that the
+                // global stores are 16-byte
+                const int c0 = t0 + j * kChunk, L = min(kChunk, t1 - c0);
+                uint32_t o[32];
+                tmem_ld32(tmem_addr(tmem, 32 * wq, Ly::kTmD1 + d * 128 + 64 + 32 * hf), o);
+                tmem_wait_ld();
+                const uint32_t ob = sbase + Ly::kOS + warp * 2048;
+#pragma unroll
+                for (int e = 0; e < 32; ++e) sts16(ob + e * 64 + lane * 2, bf16_bits(__uint_as_float(o[e])));
+                __syncwarp();
+                if (p.out) {
+#pragma unroll
+                    for (int r4 = 0; r4 < 4; ++r4) {
+                        const int e = (lane >> 2) + 8 * r4, vg = lane & 3, r = 32 * hf + e;
+                        const uint4 val = lds128(ob + e * 64 + vg * 16);
+                        if (r < L && KDA_IN_RANGE(c0 + r < p.T, p.status))
+                            *reinterpret_cast<uint4 *>(p.out + ((size_t)(c0 + r) * p.H + h) * kDV +
+                                                       32 * wq + 8 * vg) = val;
+                    }
+                }
+                __syncwarp();   // read out before the next chunk's rows land
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[cbD1Free + d]);
+            if (tid == 0) KDA_TRACE2(j, 13);
+        }
+        if (ok && p.Sf && KDA_IN_RANGE(seq < p.N, p.status)) store_state(p.Sf + sbase_g);
+    }
+
+    KDA_SPAN(g_kda_span2, 1);
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) report_abort(abort_flag, p.status);
+    if (warp == kCtMma) {
+        tc_fence_after();
+        tmem_dealloc(tmem, Ly::kTmCols);
+    }
+}
+
 int sm_count() {
     static int n = 0;
     if (!n) {
@@ -1041,6 +1381,16 @@ cudaError_t launch_chain(const ChParams &cp, int T, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     const unsigned grid2 = (unsigned)cp.N * cp.H * (kDV / VS);
     return launch_dependent(kern, grid2, ChShape<VS>::kThreads, ChLayout<VS>::kAlloc, s, mv, cp);
+}
+
+cudaError_t launch_chain_t(const ChParams &cp, int T, cudaStream_t s) {
+    CUtensorMap mv;   // the V tile as two 64-column boxes
+    if (!make_tmap_bf16_3d(&mv, cp.v_base, T, cp.H, kDV, 64, 128)) return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(chain_t_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)ChTLayout::kAlloc);
+    if (e != cudaSuccess) return e;
+    const unsigned grid2 = (unsigned)cp.N * cp.H;
+    return launch_dependent(chain_t_kernel, grid2, kCtThreads, ChTLayout::kAlloc, s, mv, cp);
 }
 
 }  // namespace
@@ -1101,7 +1451,7 @@ cudaError_t launch_prefill_two_pass(const ForwardArgs &a, cudaStream_t s) {
     const long long chains = (long long)a.N * a.H;
     if (chains * (kDV / 32) <= sm_count()) return launch_chain<32>(cp, T, s);
     if (chains * (kDV / 64) <= sm_count()) return launch_chain<64>(cp, T, s);
-    return launch_chain<128>(cp, T, s);
+    return launch_chain_t(cp, T, s);
 }
 
 }  // namespace kda

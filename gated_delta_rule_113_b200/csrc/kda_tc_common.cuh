@@ -116,6 +116,12 @@ __device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, ui
                  "r"(d)
                  : "memory");
 }
+__device__ __forceinline__ void sts16(uint32_t addr, uint16_t a) {
+    asm volatile("st.shared.b16 [%0], %1;" ::"r"(addr), "h"(a) : "memory");
+}
+__device__ __forceinline__ uint16_t bf16_bits(float x) {
+    return __bfloat16_as_ushort(__float2bfloat16_rn(x));
+}
 __device__ __forceinline__ void sts32(uint32_t addr, uint32_t a) {
     asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(a) : "memory");
 }

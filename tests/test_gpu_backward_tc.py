@@ -66,6 +66,7 @@ def _check(inp, g, tol=TOL_BF16):
     ([300, 201], 2, True, True),             # ragged multi-chunk
     ([1, 63, 64, 65, 0, 130], 2, True, False),   # edge lengths and an empty sequence
     ([129], 3, False, False),
+    ([200, 77, 64], 30, True, True),         # enough chains for the transposed forward chain
 ])
 def test_chunked_backward_matches_oracle(lengths, H, s0, dsf):
     inp = _case(lengths, H, s0, dsf)

@@ -181,6 +181,16 @@ def test_many_heads_spread_over_the_grid():
     _check(inp, out, sf, torch.bfloat16)
 
 
+def test_full_width_chain():
+    """More chains than half the SMs: the chain pass runs one transposed CTA
+    per (sequence, head) over all 128 value columns; ragged and empty
+    sequences, with an initial state."""
+    w = WORKLOADS[1]
+    inp = forward_inputs(w, lengths=[300, 1, 64, 129, 0, 200], H=20, s0=True)
+    out, sf = _run(inp)
+    _check(inp, out, sf, torch.bfloat16)
+
+
 def test_malformed_seqlens_reported_not_faulting():
     w = WORKLOADS[1]
     inp = forward_inputs(w, lengths=[64, 64], H=2)

@@ -48,6 +48,7 @@ def _workspace(inp):
     (512, [1100, 600, 100, 1536, 0, 513], 3),
     (128, [1100, 600, 100, 1536, 0, 513], 3),
     (512, [1100, 600], 80),          # enough chains for the 64-wide chain slices
+    (128, [700, 300, 130], 40),      # more: the transposed full-width chain
     (512, [0, 700, 0, 1024], 3),     # empty sequences own no slot, first one included
 ])
 def test_snapshots_match_oracle(every, lengths, H):

@@ -574,13 +574,15 @@ kside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 }
 
 // ============================================================ pass 2
-// Warp roles of the chain pass: kChain chain warps (4, or 8 for 128-wide
-// slices: warp w keeps rows 32 (w % 4) .. + 31 and columns (w / 4) kCols ..
-// + kCols - 1 of the slice), then the loader and the MMA issuer.
+// Warp roles of the narrow-slice chain pass (32- or 64-column value slices;
+// full-width chains take the transposed kernel further down): 4 chain warps
+// (warp w keeps rows 32 w .. + 31 of the slice), then the loader and the MMA
+// issuer.
 template <int VS>
 struct ChShape {
-    static constexpr int kChain = VS == 128 ? 8 : 4;
-    static constexpr int kCols = VS * 4 / kChain;
+    static_assert(VS == 32 || VS == 64, "narrow value slices only");
+    static constexpr int kChain = 4;
+    static constexpr int kCols = VS;
     static constexpr int kLoad = kChain, kMma = kChain + 1;
     static constexpr int kThreads = (kChain + 2) * 32;
 };
@@ -731,12 +733,9 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_v, ChParams p) {
                 bulk_load(st + off, packet(j) + off, len, full);
             }
             if (lane == 4) tma_load_3d(st + Ly::kV, &tm_v, full, vs * VS, h, t0 + j * kChunk);
-            if (VS == 128 && lane == 7)   // the second 64-wide atom of the slice
-                tma_load_3d(st + Ly::kV + 64 * 128, &tm_v, full, 64, h, t0 + j * kChunk);
             if (j + Ly::kStages < nchunks) {   // warm L2 for the copies of chunk j + kStages
                 if (lane == 5) bulk_prefetch_l2(packet(j + Ly::kStages), (uint32_t)kPacketBytes);
                 if (lane == 8) tma_prefetch_3d(&tm_v, vs * VS, h, t0 + (j + Ly::kStages) * kChunk);
-                if (VS == 128 && lane == 9) tma_prefetch_3d(&tm_v, 64, h, t0 + (j + Ly::kStages) * kChunk);
             }
             n_issued = j + 1;
             if (lane == 0) KDA_TRACE2(j, 0);
@@ -1372,9 +1371,8 @@ cudaError_t launch_dependent(void (*kern)(KArgs...), unsigned grid, unsigned blo
 
 template <int VS>
 cudaError_t launch_chain(const ChParams &cp, int T, cudaStream_t s) {
-    CUtensorMap mv;   // 128-wide slices load their V tile as two 64-wide boxes
-    constexpr int box = VS < 64 ? VS : 64;
-    if (!make_tmap_bf16_3d(&mv, cp.v_base, T, cp.H, kDV, box, box * 2)) return cudaErrorInvalidValue;
+    CUtensorMap mv;
+    if (!make_tmap_bf16_3d(&mv, cp.v_base, T, cp.H, kDV, VS, VS * 2)) return cudaErrorInvalidValue;
     auto kern = chain_kernel<VS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)ChLayout<VS>::kAlloc);

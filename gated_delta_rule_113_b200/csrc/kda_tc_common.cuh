@@ -136,19 +136,16 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
 
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) { return pack_bf16(lo, hi); }
 
-// Byte offset of 16-byte chunk `chunk` of row `row` in a VS-wide MN-major tile
-// of `rows` rows (a 128-wide tile is two 64-wide atoms `rows` x 128 bytes apart).
+// Byte offset of 16-byte chunk `chunk` of row `row` in a VS-wide (32 or 64)
+// MN-major tile.
 template <int VS>
-__device__ __forceinline__ uint32_t vs_off(uint32_t row, uint32_t chunk, uint32_t rows = 0) {
-    if (VS == 32) return sw64_off(row, chunk);
-    if (VS == 64) return sw128_off(row, chunk);
-    return (chunk >> 3) * rows * 128u + sw128_off(row, chunk & 7u);
+__device__ __forceinline__ uint32_t vs_off(uint32_t row, uint32_t chunk, uint32_t = 0) {
+    static_assert(VS == 32 || VS == 64, "narrow value slices only");
+    return VS == 32 ? sw64_off(row, chunk) : sw128_off(row, chunk);
 }
 
 // B-operand descriptor of a VS-wide MN-major tile (rows = K) at K step 0;
-// step ks adds vs_step(ks) (start address field, in 16-byte units).  Wider
-// than 64 columns, the leading-dimension offset is the distance between the
-// 64-wide atoms.
+// step ks adds vs_step(ks) (start address field, in 16-byte units).
 template <int VS>
 __device__ __forceinline__ uint64_t vs_desc(uint32_t base, uint32_t rows) {
     return VS == 32 ? smem_desc(base, rows * 64, 512, kSw64)

@@ -100,12 +100,13 @@ def test_snapshots_leave_outputs_bit_identical():
     assert torch.equal(pool2[1], sf2[0])
 
 
-def test_resume_from_snapshot_matches_uninterrupted_run():
+@pytest.mark.parametrize("H", [None, 40])   # 40 heads: the transposed full-width chain
+def test_resume_from_snapshot_matches_uninterrupted_run(H):
     """Prefill a prefix with snapshots, then prefill the rest of each sequence
     starting from a pool slot: outputs and final states match the oracle's
     uninterrupted run."""
     lengths = [1300, 700]
-    inp = _inputs(lengths)
+    inp = _inputs(lengths) if H is None else _inputs(lengths, H=H)
     H = inp["q"].shape[1]
     every = 512
     ro, rs = oracle.forward(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"],

@@ -2,8 +2,9 @@
 problems: every checked global index stays inside its buffer (the device
 status word stays KDA_OK; an index that left its buffer would be skipped and
 recorded as KDA_ERR_BOUNDS, without a trap), and the results are those of the
-regular build.  Covered: the two-pass prefill with snapshots, the fused and
-CUDA-core prefills, and both backward paths."""
+regular build.  Covered: the two-pass prefill with snapshots (narrow and
+full-width chains), the fused and CUDA-core prefills, and both backward
+paths."""
 import contextlib
 
 import numpy as np
@@ -43,13 +44,14 @@ def _forward(d, lens, H, **kw):
     return out, sf, kda.workspace_status(ws)
 
 
-@pytest.mark.parametrize("path", ["two_pass", "fused_tc", "simt"])
+@pytest.mark.parametrize("path", ["two_pass", "two_pass_full_width", "fused_tc", "simt"])
 def test_debug_bounds_build_prefill(path):
-    lens, H = [300, 1, 64, 0, 130], 2
+    # 40 heads: enough chains for the transposed full-width chain kernel
+    lens, H = [300, 1, 64, 0, 130], (40 if path == "two_pass_full_width" else 2)
     inp = forward_inputs(WORKLOADS[1], lengths=lens, H=H, s0=True)
     d = to_dev(inp)
     kw = {"fused_tc": path == "fused_tc", "force_simt": path == "simt"}
-    if path == "two_pass":
+    if path.startswith("two_pass"):
         n_snap = sum(n // 64 for n in lens)
         pool = torch.zeros((n_snap, H, 128, 128), device="cuda")
         base = torch.tensor([sum(n // 64 for n in lens[:i]) for i in range(len(lens))],

@@ -275,20 +275,21 @@ def test_decode_equals_prefill():
     assert rel_fro(as_np(S), as_np(p_s)) < 1e-2
 
 
-def test_bounded_wait_times_out_and_the_context_stays_usable():
+@pytest.mark.parametrize("H", [2, 40])   # 40 heads: the transposed full-width chain
+def test_bounded_wait_times_out_and_the_context_stays_usable(H):
     """KDA_FLAG_TEST_STALL makes the chain pass wait on a barrier nothing
     arrives on: the wait gives up after its 2 s bound, the call records
     KDA_ERR_TIMEOUT, and the next call on the same context is correct."""
     import time
     w = WORKLOADS[1]
-    inp = forward_inputs(w, lengths=[300, 129], H=2)
+    inp = forward_inputs(w, lengths=[300, 129], H=H)
     d = to_dev(inp)
-    ws = torch.empty(kda.forward_workspace_size(2, 429, 2, 128, 128), dtype=torch.uint8,
+    ws = torch.empty(kda.forward_workspace_size(2, 429, H, 128, 128), dtype=torch.uint8,
                      device="cuda")
     lib = kda.load_library()
-    out = torch.empty((429, 2, 128), dtype=torch.bfloat16, device="cuda")
-    sf = torch.empty((2, 2, 128, 128), dtype=torch.float32, device="cuda")
-    p = kda.Params(2, 429, 2, 128, 128, 64, 1, 1, 4)   # KDA_FLAG_TEST_STALL
+    out = torch.empty((429, H, 128), dtype=torch.bfloat16, device="cuda")
+    sf = torch.empty((2, H, 128, 128), dtype=torch.float32, device="cuda")
+    p = kda.Params(2, 429, H, 128, 128, 64, 1, 1, 4)   # KDA_FLAG_TEST_STALL
     t0 = time.time()
     rc = lib.kda_forward(*(kda._ptr(x) for x in (d["q"], d["k"], d["v"], d["log_alpha"],
                                                  d["beta"], d["S0"], d["cu_seqlens"], out, sf)),
